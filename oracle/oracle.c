@@ -1,0 +1,489 @@
+/*
+ * CPU oracle for selective mixed-precision block attention (FP16 / NVFP4).
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this library.  It shares no code with the CUDA
+ * library and must never sit on the product path.
+ *
+ * What it computes (page: "ThriftAttention: Selective Mixed Precision for
+ * Long-Context FP4 Attention", abstract, and the same page's summary,
+ * "technical approach" items 2-5):
+ *   stage 1  a cheap heuristic picks a small fraction of (query block, key
+ *            block) pairs to be computed in FP16;
+ *   stage 2  the picked pairs are computed in FP16, every other pair in
+ *            block-scaled FP4, and both are merged by one online softmax into
+ *            one output.
+ * The pages leave the format, the heuristic, the block size and the handling
+ * of P open.  The readings taken here (one comment per function says which):
+ *   - NVFP4: E2M1 values, one E4M3 scale per 16 consecutive elements along the
+ *     contracted dimension, round to nearest even, scale = E4M3(amax/6) with
+ *     amax/6 formed in FP32; a zero scale encodes the whole group as +0.
+ *   - Q and K are quantised along D, V along the key axis, P per 16 keys.
+ *   - P is encoded at a fixed power-of-two pre-scale 2^c (c = 11 by default,
+ *     0 gives the literal reading); the same pre-scale is used for the FP16
+ *     encoding of P and is divided out of the output.
+ *   - Heuristic: score(i,j) = fl32(sm_scale * fl32(mean_q(i) . mean_k(j)));
+ *     per (batch, query head) keep ceil(rho * #valid - 1e-9) pairs; the
+ *     diagonal pairs (i,i) and the key-block-0 pairs (i,0) come first, then
+ *     higher scores, then the lower linear index i*nb + j.
+ *   - Online softmax with an integer running maximum M = ceil(max t), t the
+ *     log2-domain logit; rescales are exact powers of two.
+ *   - l sums the unquantised P; quantisation only encodes the P.V operand.
+ * All arithmetic is FP64 with FP32/FP16/FP4 rounding at the points the
+ * readings name.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* IEEE binary16                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Value of an fp16 bit pattern (1 sign, 5 exponent bits with bias 15, 10
+ * mantissa bits; exponent 0 = subnormal; exponent 31 = inf/NaN). */
+double orc_f16_value(uint16_t h) {
+    int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp(1024.0 + m, e - 25);
+    return s ? -v : v;
+}
+
+/* The same map as a table, filled once when the library loads; used on the
+ * hot loops of the attention rows. */
+static double F16_TABLE[65536];
+static double E4M3_TABLE[256];
+double orc_e4m3_value(uint8_t code);
+__attribute__((constructor)) static void orc_init_tables(void) {
+    for (int h = 0; h < 65536; ++h) F16_TABLE[h] = orc_f16_value((uint16_t)h);
+    for (int c = 0; c < 256; ++c) E4M3_TABLE[c] = orc_e4m3_value((uint8_t)c);
+}
+
+/* Nearest fp16 to v (ties to even mantissa), overflow to inf.  Written as a
+ * search over the representable neighbours so it reads as the definition. */
+uint16_t orc_f16_encode(double v) {
+    if (isnan(v)) return 0x7E00;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a >= 65520.0) return sign | 0x7C00;
+    /* quantum of the binade containing a (subnormal quantum below 2^-14) */
+    int e = (a < 0x1p-14) ? -14 : ilogb(a);
+    double q = ldexp(1.0, e - 10);
+    double lo = floor(a / q) * q, hi = lo + q;
+    double pick;
+    if (a - lo < hi - a) pick = lo;
+    else if (a - lo > hi - a) pick = hi;
+    else pick = (fmod(lo / q, 2.0) == 0.0) ? lo : hi; /* tie: even multiple of the quantum */
+    /* rebuild the bit pattern of pick */
+    if (pick == 0) return sign;
+    if (pick < 0x1p-14) return sign | (uint16_t)(pick / 0x1p-24);
+    int pe = ilogb(pick);
+    if (pe > 15) return sign | 0x7C00;
+    uint16_t mant = (uint16_t)(ldexp(pick, 10 - pe) - 1024.0);
+    return sign | (uint16_t)((pe + 15) << 10) | mant;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 (FP4) and E4M3 (FP8) used by NVFP4                                   */
+/* ------------------------------------------------------------------------ */
+
+/* E2M1 magnitudes by 3-bit code: exponent bias 1, one mantissa bit,
+ * code 1 is the subnormal 0.5.  Bit 3 of a code is the sign. */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double orc_e2m1_value(uint8_t code) {
+    double m = E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* Round v to the E2M1 grid: nearest magnitude, ties to the even code,
+ * magnitudes above 6 saturate to 6; the sign is kept (so -0.1 -> code 8). */
+uint8_t orc_e2m1_encode(double v) {
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs(v);
+    if (a >= 6.0) return sign | 7;
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        double dc = fabs(a - E2M1_MAG[c]), db = fabs(a - E2M1_MAG[best]);
+        if (dc < db || (dc == db && (c % 2 == 0))) best = c;
+    }
+    return sign | (uint8_t)best;
+}
+
+/* E4M3 (OCP FP8): 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * exponent 0 = subnormal (m/8 * 2^-6), pattern S.1111.111 = NaN, no inf;
+ * largest finite 448. */
+double orc_e4m3_value(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(8.0 + m, e - 10);
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 to v, ties to even mantissa, finite saturation at 448. */
+uint8_t orc_e4m3_encode(double v) {
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs(v);
+    uint8_t best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 127; ++c) { /* 0x7F is NaN; 0x7E = 448 is the largest */
+        double d = fabs(a - orc_e4m3_value((uint8_t)c));
+        if (d < bestd || (d == bestd && (c % 2 == 0))) { bestd = d; best = (uint8_t)c; }
+    }
+    return sign | best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 group quantisation                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Encode 16 values (held exactly as doubles) as one E4M3 scale and sixteen
+ * E2M1 codes.  scale = E4M3(fl32(amax/6)); code = E2M1(x / scale); a zero
+ * scale encodes every element as +0.  (float)(amax/6.0) equals the FP32
+ * quotient: amax has at most 24 significant bits, so amax/6 is never within
+ * 2^-53 of an FP32 rounding boundary without being on it.) */
+static void quant_group16(const double* x, uint8_t* codes, uint8_t* scale) {
+    double amax = 0;
+    for (int i = 0; i < 16; ++i) amax = fmax(amax, fabs(x[i]));
+    float s32 = (float)(amax / 6.0);
+    uint8_t sc = orc_e4m3_encode((double)s32);
+    double s = orc_e4m3_value(sc);
+    *scale = sc;
+    for (int i = 0; i < 16; ++i) codes[i] = (s == 0.0) ? 0 : orc_e2m1_encode(x[i] / s);
+}
+
+/* Quantise `rows` rows of `len` fp16 values along the row.
+ * codes: [rows][len/2], element 2k in the low nibble of byte k.
+ * scales: [rows][len/16] E4M3 bytes.  len must be a multiple of 16. */
+int orc_quantize_rows(const uint16_t* x, long rows, int len, uint8_t* codes, uint8_t* scales) {
+    if (len <= 0 || len % 16) return 1;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (int g = 0; g < len / 16; ++g) {
+            double v[16];
+            uint8_t c[16];
+            for (int i = 0; i < 16; ++i) v[i] = orc_f16_value(x[r * len + g * 16 + i]);
+            quant_group16(v, c, &scales[r * (len / 16) + g]);
+            for (int i = 0; i < 8; ++i)
+                codes[r * (len / 2) + g * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+/* V is quantised along the key axis: V [BH][N][D] -> codes [BH][D][N/2],
+ * scales [BH][D][N/16] (keys contiguous). */
+int orc_quantize_v(const uint16_t* V, long BH, int N, int D, uint8_t* codes, uint8_t* scales) {
+    if (N <= 0 || N % 16 || D <= 0) return 1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (long bh = 0; bh < BH; ++bh) {
+        for (int d = 0; d < D; ++d) {
+            for (int g = 0; g < N / 16; ++g) {
+                double v[16];
+                uint8_t c[16];
+                for (int i = 0; i < 16; ++i) v[i] = orc_f16_value(V[(bh * N + g * 16 + i) * (long)D + d]);
+                quant_group16(v, c, &scales[(bh * D + d) * (long)(N / 16) + g]);
+                for (int i = 0; i < 8; ++i)
+                    codes[(bh * D + d) * (long)(N / 2) + g * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+static double deq(const uint8_t* codes, const uint8_t* scales, long row, int len, int i) {
+    uint8_t byte = codes[row * (len / 2) + i / 2];
+    uint8_t c = (i & 1) ? (byte >> 4) : (byte & 15);
+    return orc_e2m1_value(c) * E4M3_TABLE[scales[row * (len / 16) + i / 16]];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stage 1: block-pair selection                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct { int forced; float score; long idx; } cand;
+
+static int cand_cmp(const void* a, const void* b) {
+    const cand* x = (const cand*)a;
+    const cand* y = (const cand*)b;
+    if (x->forced != y->forced) return y->forced - x->forced;     /* forced first */
+    if (x->score != y->score) return (x->score > y->score) ? -1 : 1; /* higher score first */
+    return (x->idx < y->idx) ? -1 : (x->idx > y->idx);             /* lower index first */
+}
+
+/* Number of pairs kept: ceil(rho * valid - 1e-9), clamped to [0, valid]. */
+long orc_budget(double rho, long valid) {
+    double k = ceil(rho * (double)valid - 1e-9);
+    if (k < 0) k = 0;
+    if (k > (double)valid) k = (double)valid;
+    return (long)k;
+}
+
+/* Block means in FP32: the FP64 sum of the block's fp16 rows (exact), divided
+ * by blk, rounded once to FP32.  out: [nb][D]. */
+static void block_means(const uint16_t* x, int N, int D, int blk, float* out) {
+    int nb = N / blk;
+    for (int i = 0; i < nb; ++i)
+        for (int d = 0; d < D; ++d) {
+            double s = 0;
+            for (int r = i * blk; r < (i + 1) * blk; ++r) s += orc_f16_value(x[(long)r * D + d]);
+            out[(long)i * D + d] = (float)(s / blk);
+        }
+}
+
+/* Pooled scores of one (batch, query head): scores [nb][nb] (invalid pairs
+ * are left untouched). */
+int orc_pooled_scores(const uint16_t* Qh, const uint16_t* Kh, int N, int D, int blk, int causal,
+                      float sm_scale, float* scores) {
+    if (blk <= 0 || N % blk) return 1;
+    int nb = N / blk;
+    float* qm = (float*)malloc(sizeof(float) * (size_t)nb * D);
+    float* km = (float*)malloc(sizeof(float) * (size_t)nb * D);
+    if (!qm || !km) { free(qm); free(km); return 2; }
+    block_means(Qh, N, D, blk, qm);
+    block_means(Kh, N, D, blk, km);
+    for (int i = 0; i < nb; ++i)
+        for (int j = 0; j < nb; ++j) {
+            if (causal && j > i) continue;
+            double dot = 0;
+            for (int d = 0; d < D; ++d) dot += (double)qm[(long)i * D + d] * (double)km[(long)j * D + d];
+            scores[(long)i * nb + j] = (float)((double)sm_scale * (double)(float)dot);
+        }
+    free(qm); free(km);
+    return 0;
+}
+
+/* Selection mask for every (batch, query head): mask [B][Hq][nb][nb],
+ * 1 = FP16 pair, 0 = FP4 pair or invalid pair.  Query head h uses key head
+ * h / (Hq/Hkv). */
+int orc_select(const uint16_t* Q, const uint16_t* K, int B, int Hq, int Hkv, int N, int D, int blk,
+               int causal, float sm_scale, double rho, uint8_t* mask) {
+    if (blk <= 0 || N % blk || Hq % Hkv) return 1;
+    int nb = N / blk, G = Hq / Hkv;
+    int fail = 0;
+    #pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            const uint16_t* Qh = Q + ((long)b * Hq + h) * (long)N * D;
+            const uint16_t* Kh = K + ((long)b * Hkv + h / G) * (long)N * D;
+            float* sc = (float*)malloc(sizeof(float) * (size_t)nb * nb);
+            cand* cs = (cand*)malloc(sizeof(cand) * (size_t)nb * nb);
+            uint8_t* m = mask + ((long)b * Hq + h) * (long)nb * nb;
+            if (!sc || !cs || orc_pooled_scores(Qh, Kh, N, D, blk, causal, sm_scale, sc)) {
+                #pragma omp atomic write
+                fail = 1;
+                free(sc); free(cs);
+                continue;
+            }
+            long nv = 0;
+            for (int i = 0; i < nb; ++i)
+                for (int j = 0; j < nb; ++j) {
+                    m[(long)i * nb + j] = 0;
+                    if (causal && j > i) continue;
+                    cs[nv].forced = (i == j) || (j == 0);
+                    cs[nv].score = sc[(long)i * nb + j];
+                    cs[nv].idx = (long)i * nb + j;
+                    ++nv;
+                }
+            long k = orc_budget(rho, nv);
+            qsort(cs, (size_t)nv, sizeof(cand), cand_cmp);
+            for (long t = 0; t < k; ++t) m[cs[t].idx] = 1;
+            free(sc); free(cs);
+        }
+    return fail;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stage 2: mixed-precision attention, one output row at a time              */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *Q, *K, *V;                 /* fp16 [B,H,N,D] */
+    const uint8_t *q4, *qs, *k4, *ks;          /* NVFP4 along D: [B,H,N,D/2], [B,H,N,D/16] */
+    const uint8_t *v4, *vs;                    /* NVFP4 along keys: [B,Hkv,D,N/2], [B,Hkv,D,N/16] */
+    int B, Hq, Hkv, N, D, blk, causal;
+    float sm_scale;
+    int p_log2;                                /* pre-scale exponent c of P */
+} orc_problem;
+
+/* log2-domain logit: t = fl32(fl32(S) * fl32(sm_scale * log2 e)). */
+static float logit_log2(double S, float sm_scale) {
+    float c = (float)((double)sm_scale * 1.4426950408889634073599246810019);
+    return (float)((double)(float)S * (double)c);
+}
+
+/* Raw score S of (query row r of head h, key k of key head hk) in the given
+ * precision: FP16 operands, or dequantised NVFP4 operands.  FP64 sum. */
+static double score(const orc_problem* p, int b, int h, int hk, int r, int k, int fp16) {
+    const int D = p->D;
+    long qrow = ((long)b * p->Hq + h) * p->N + r;
+    long krow = ((long)b * p->Hkv + hk) * p->N + k;
+    double s = 0;
+    for (int d = 0; d < D; ++d) {
+        double qv = fp16 ? F16_TABLE[p->Q[qrow * D + d]] : deq(p->q4, p->qs, qrow, D, d);
+        double kv = fp16 ? F16_TABLE[p->K[krow * D + d]] : deq(p->k4, p->ks, krow, D, d);
+        s += qv * kv;
+    }
+    return s;
+}
+
+/* V element (key k, channel d) in the given precision. */
+static double v_elem(const orc_problem* p, int b, int hk, int k, int d, int fp16) {
+    if (fp16) return F16_TABLE[p->V[(((long)b * p->Hkv + hk) * p->N + k) * p->D + d]];
+    long vrow = ((long)b * p->Hkv + hk) * p->D + d;
+    return deq(p->v4, p->vs, vrow, p->N, k);
+}
+
+/* Encode the P of one key block: FP16 (nearest fp16 of P*2^c) or NVFP4 per
+ * aligned group of 16 keys of P*2^c; returns the decoded values times 2^-c.
+ * Masked keys carry P = 0. */
+static void encode_p(const double* P, int n, int fp16, int p_log2, double* out) {
+    double pre = ldexp(1.0, p_log2), post = ldexp(1.0, -p_log2);
+    if (fp16) {
+        for (int i = 0; i < n; ++i) out[i] = orc_f16_value(orc_f16_encode(P[i] * pre)) * post;
+        return;
+    }
+    for (int g = 0; g < n; g += 16) {
+        double x[16];
+        uint8_t c[16], sc;
+        for (int i = 0; i < 16; ++i) x[i] = P[g + i] * pre;
+        quant_group16(x, c, &sc);
+        double s = orc_e4m3_value(sc);
+        for (int i = 0; i < 16; ++i) out[g + i] = orc_e2m1_value(c[i]) * s * post;
+    }
+}
+
+/* One output row by the online merge: key blocks are visited in `order`
+ * (a permutation of 0..nb-1; invalid blocks are skipped).  The running max M
+ * is an integer; when it grows, l and the accumulator are scaled by the exact
+ * power of two 2^(M_old - M_new).  out: D values of O (FP64, before the
+ * final fp16 rounding). */
+static void attention_row(const orc_problem* p, const uint8_t* mask, int b, int h, int r, const int* order,
+                          double* out) {
+    const int N = p->N, D = p->D, blk = p->blk, nb = N / blk;
+    const int hk = h / (p->Hq / p->Hkv), qb = r / blk;
+    double* acc = (double*)calloc((size_t)D, sizeof(double));
+    double* P = (double*)malloc(sizeof(double) * blk);
+    double* Pt = (double*)malloc(sizeof(double) * blk);
+    float* t = (float*)malloc(sizeof(float) * blk);
+    double M = -INFINITY, l = 0;
+    for (int oi = 0; oi < nb; ++oi) {
+        int j = order ? order[oi] : oi;
+        if (p->causal && j > qb) continue;
+        int fp16 = mask[(((long)b * p->Hq + h) * nb + qb) * nb + j] != 0;
+        float tmax = -INFINITY;
+        for (int i = 0; i < blk; ++i) {
+            int k = j * blk + i;
+            if (p->causal && k > r) { t[i] = -INFINITY; continue; }
+            t[i] = logit_log2(score(p, b, h, hk, r, k, fp16), p->sm_scale);
+            if (t[i] > tmax) tmax = t[i];
+        }
+        double Mn = fmax(M, ceil((double)tmax));
+        if (Mn > M && M != -INFINITY) {
+            double a = ldexp(1.0, (int)(M - Mn));
+            l *= a;
+            for (int d = 0; d < D; ++d) acc[d] *= a;
+        }
+        M = Mn;
+        for (int i = 0; i < blk; ++i) {
+            P[i] = (t[i] == -INFINITY) ? 0.0 : (double)(float)exp2((double)t[i] - M);
+            l += P[i];
+        }
+        encode_p(P, blk, fp16, p->p_log2, Pt);
+        for (int i = 0; i < blk; ++i) {
+            if (Pt[i] == 0.0) continue;
+            int k = j * blk + i;
+            for (int d = 0; d < D; ++d) acc[d] += Pt[i] * v_elem(p, b, hk, k, d, fp16);
+        }
+    }
+    for (int d = 0; d < D; ++d) out[d] = acc[d] / l;
+    free(acc); free(P); free(Pt); free(t);
+}
+
+static int check_problem(const orc_problem* p) {
+    if (p->B <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Hq % p->Hkv) return 1;
+    if (p->blk <= 0 || p->blk % 16 || p->N % p->blk || p->D % 16) return 1;
+    return 0;
+}
+
+/* Mixed-precision attention for a list of rows (b, h, r): out [nrows][D].
+ * order: NULL (ascending key blocks) or one permutation of 0..nb-1 used for
+ * every row. */
+int orc_attention_rows(const orc_problem* p, const uint8_t* mask, const int64_t* rows, long nrows,
+                       const int* order, double* out) {
+    if (check_problem(p)) return 1;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (long i = 0; i < nrows; ++i)
+        attention_row(p, mask, (int)rows[3 * i], (int)rows[3 * i + 1], (int)rows[3 * i + 2], order,
+                      out + i * p->D);
+    return 0;
+}
+
+/* Pure-FP4 attention written directly (two passes, no mask, no online merge):
+ * the reference point for rho = 0. */
+int orc_attention_fp4_rows(const orc_problem* p, const int64_t* rows, long nrows, double* out) {
+    if (check_problem(p)) return 1;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (long i = 0; i < nrows; ++i) {
+        int b = (int)rows[3 * i], h = (int)rows[3 * i + 1], r = (int)rows[3 * i + 2];
+        int hk = h / (p->Hq / p->Hkv);
+        int nk = p->causal ? (r / p->blk + 1) * p->blk : p->N;   /* keys of the visited blocks */
+        double* P = (double*)calloc((size_t)nk, sizeof(double));
+        double* Pt = (double*)malloc(sizeof(double) * (size_t)nk);
+        float* t = (float*)malloc(sizeof(float) * (size_t)nk);
+        float tmax = -INFINITY;
+        for (int k = 0; k < nk; ++k) {
+            t[k] = (p->causal && k > r) ? -INFINITY : logit_log2(score(p, b, h, hk, r, k, 0), p->sm_scale);
+            if (t[k] > tmax) tmax = t[k];
+        }
+        double M = ceil((double)tmax), l = 0;
+        for (int k = 0; k < nk; ++k) {
+            P[k] = (t[k] == -INFINITY) ? 0.0 : (double)(float)exp2((double)t[k] - M);
+            l += P[k];
+        }
+        encode_p(P, nk, 0, p->p_log2, Pt);
+        for (int d = 0; d < p->D; ++d) {
+            double s = 0;
+            for (int k = 0; k < nk; ++k) s += Pt[k] * v_elem(p, b, hk, k, d, 0);
+            out[i * p->D + d] = s / l;
+        }
+        free(P); free(Pt); free(t);
+    }
+    return 0;
+}
+
+/* Exact attention softmax(Q K^T sm_scale) V in FP64 from the fp16 inputs. */
+int orc_exact_rows(const orc_problem* p, const int64_t* rows, long nrows, double* out) {
+    if (check_problem(p)) return 1;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (long i = 0; i < nrows; ++i) {
+        int b = (int)rows[3 * i], h = (int)rows[3 * i + 1], r = (int)rows[3 * i + 2];
+        int hk = h / (p->Hq / p->Hkv);
+        int nk = p->causal ? r + 1 : p->N;
+        double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+        double mx = -INFINITY, l = 0;
+        for (int k = 0; k < nk; ++k) {
+            s[k] = score(p, b, h, hk, r, k, 1) * (double)p->sm_scale;
+            if (s[k] > mx) mx = s[k];
+        }
+        for (int k = 0; k < nk; ++k) { s[k] = exp(s[k] - mx); l += s[k]; }
+        for (int d = 0; d < p->D; ++d) {
+            double a = 0;
+            for (int k = 0; k < nk; ++k) a += s[k] * v_elem(p, b, hk, k, d, 1);
+            out[i * p->D + d] = a / l;
+        }
+        free(s);
+    }
+    return 0;
+}
+
+/* Round an array of doubles to fp16 bit patterns. */
+void orc_to_f16(const double* x, long n, uint16_t* out) {
+    #pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i) out[i] = orc_f16_encode(x[i]);
+}
