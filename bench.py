@@ -1,0 +1,399 @@
+"""Benchmark of the selective mixed-precision (FP16 / NVFP4) attention hot path.
+
+One step = one pass of the whole path on one synthetic batch:
+NVFP4 quantisation of Q, K, V -> block-pair selection (rho = 5%) -> fused
+mixed-precision attention, all through the library's C ABI.  Workload: causal
+GQA prefill, B=1, Hq=32, Hkv=8, N=32768, D=128, fp16 inputs, 128x128
+selection blocks.  Inputs (Q alone is 268 MB) are larger than the 126 MB L2,
+so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line on rank 0.  For N > 1 (torchrun) every rank runs its own
+independent problem (weak scaling, no data-path collective); the timed
+region is bracketed by a barrier and the slowest rank's time is reported.
+`--impl reference` times the CPU oracle on a bounded row sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "effective attn TFLOPS (ρ=5%, causal prefill) & % of blended FP4/FP16 roofline"
+WORKLOAD = synth.GQA_N32K
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attention_gqa_n32k_traffic.json")
+KERNEL_SOURCES = ["attention.cu", "ptx.cuh", "common.h"]
+LAUNCHES_PER_STEP = 8        # quantize Q, K, V; pool Q, K; scores; top-k; attention
+
+
+# ---------------------------------------------------------------- helpers ---
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max over ranks of a float (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "fp16_block_attention_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    try:
+        with open(PROFILE_FILE) as f:
+            prof = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if prof.get("kernel_hash") != kernel_hash():
+        return None
+    return prof.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def flop_split(w, mask_np):
+    """Effective FLOPs of the FP16 and FP4 block pairs (diagonal pairs count their
+    causal triangle), from the selection mask [B, Hq, nb, nb]."""
+    nb = w.N // w.blk
+    full = 4.0 * w.blk * w.blk * w.D
+    diag = 4.0 * w.D * w.blk * (w.blk + 1) / 2 if w.causal else full
+    eye = np.eye(nb, dtype=bool)
+    valid = np.tril(np.ones((nb, nb), bool)) if w.causal else np.ones((nb, nb), bool)
+    weight = np.where(eye, diag, full) * valid
+    f16 = float((weight[None, None] * (mask_np == 1)).sum())
+    total = float(weight.sum()) * w.B * w.Hq
+    return f16, total - f16
+
+
+# ------------------------------------------------------------------ our arm ---
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp16_block_attention_b200 as thrift
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    w = WORKLOAD.with_(seed=WORKLOAD.seed + 1000 * rank) if world > 1 else WORKLOAD
+    Q, K, V = synth.generate(w)
+    sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+    Od = torch.empty_like(Qd)
+    ws = torch.empty(thrift.fused_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # The fused entry point's stages as separate C-ABI calls on the same
+    # workspace, so the attention kernel can be timed on its own.
+    nc = [thrift.quant_bytes(sh, op) for op in (0, 1, 2)]
+    nb = sh.nb
+    offs, o = [], 0
+    for size in (nc[0][0], nc[0][1], nc[1][0], nc[1][1], nc[2][0], nc[2][1], w.B * w.Hq * nb * nb,
+                 thrift.select_workspace_bytes(sh)):
+        offs.append(o)
+        o += (size + 255) // 256 * 256
+    part = [ws[offs[i]:offs[i + 1]] if i + 1 < len(offs) else ws[offs[i]:] for i in range(len(offs))]
+    qz = thrift.Quantised(part[0], part[1], part[2], part[3], part[4], part[5])
+    mask = part[6][:w.B * w.Hq * nb * nb].view(w.B, w.Hq, nb, nb)
+    sel_ws = part[7]
+
+    def step(ev_a=None, ev_b=None):
+        thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, stream)
+        thrift.quantize_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, stream)
+        thrift.quantize_nvfp4(Vd, thrift.V, sh, qz.v4, qz.vs, stream)
+        thrift.select_blocks(Qd, Kd, sh, w.rho, mask, sel_ws, stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if thrift.last_device_error(stream) != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(*ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if thrift.last_device_error(stream) != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout during timing")
+    ms_total = reduce_max(ms_total, dev)
+    attn_ms = reduce_max(attn_ms, dev)
+    ms_step = ms_total / args.steps
+
+    # ---- end to end through the public API: host buffers, copies inside the timed region
+    Qh, Kh, Vh = (torch.from_numpy(a).pin_memory() for a in (Q, K, V))
+    Oh = torch.empty(Qh.shape, dtype=torch.float16).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        Qd.copy_(Qh, non_blocking=True)
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        thrift.attention_fused(Qd, Kd, Vd, sh, w.rho, out=Od, ws=ws, stream=stream)
+        Oh.copy_(Od, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, dev)
+
+    # ---- roofline of the attention kernel (blended FP16 / NVFP4 tensor peak)
+    peaks, peak_kind = load_peaks()
+    p16 = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    p4 = FP4_OVER_BF16 * p16
+    f16, f4 = flop_split(w, mask.cpu().numpy())
+    flops = w.flops()
+    t_tensor = f16 / p16 + f4 / p4
+    bytes_alg = attention_bytes(w, mask.cpu().numpy())
+    t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
+    t_bound = max(t_tensor, t_hbm)
+    blended_peak = flops / t_bound / 1e12
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    n = world
+    value = n * flops / (ms_step * 1e-3) / 1e12
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4+fp16 (fp32 accum)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D, "causal": w.causal,
+                   "rho": w.rho, "blk": w.blk, "l2": "inputs larger than L2 (Q alone 268 MB), no flush",
+                   "parallelism": f"independent problem per GPU x{n}",
+                   "step": "quantize Q,K,V + select + attention (C ABI)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(blended_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / blended_peak, 4), "traffic": profiled_traffic(),
+                     "peak_source": f"{peak_kind}: blended from bf16 sustained {p16 / 1e12:.1f} TF (FP16 pairs) "
+                                    f"and {FP4_OVER_BF16:g}x that (FP4 pairs), HBM {peaks['hbm_gbs']} GB/s",
+                     "fp16_pair_flop_share": round(f16 / flops, 4), "attention_ms": round(attn_ms, 4),
+                     "t_tensor_ms": round(t_tensor * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
+                     "algorithmic_bytes": int(bytes_alg)},
+        "clocks": clocks,
+        "e2e": {"value": round(n * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": int(Qh.numel() * 2 + Kh.numel() * 2 + Vh.numel() * 2),
+                "d2h_bytes_per_step": int(Oh.numel() * 2)},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def attention_bytes(w, mask_np):
+    """Algorithmic HBM bytes of one attention launch: NVFP4 Q, K, V (0.5625 B per
+    element) read once, fp16 K/V of FP16 key tiles once per query head that
+    selects them, fp16 Q of query tiles with an FP16 pair, and O (2 B/elt)."""
+    e_q = w.B * w.Hq * w.N * w.D
+    e_kv = w.B * w.Hkv * w.N * w.D
+    per_tile = w.blk * w.D * 2 * 2  # fp16 K and V of one key block
+    q_tiles16 = int((mask_np.reshape(w.B, w.Hq, w.N // w.blk, -1).max(-1) == 1).sum())
+    return 0.5625 * e_q + 2 * 0.5625 * e_kv + float((mask_np == 1).sum()) * per_tile + \
+        q_tiles16 * w.blk * w.D * 2 + 2 * e_q
+
+
+# --------------------------------------------------------- the CPU oracle ---
+class OracleRows:
+    """The oracle (plain C, FP64, OpenMP over rows) on a bounded sample of the
+    workload: the mixed-precision attention of seeded rows (random heads and
+    positions).  The O(N*D) quantisation and selection stages are run once in
+    the set-up, outside the timing (under 1% of the path's work); the FLOPs
+    counted are the sampled rows' effective attention FLOPs (4*D per key)."""
+
+    def __init__(self, w):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        self.Q, self.K, self.V = synth.generate(w)
+        self.mask = oracle.select(self.Q, self.K, w.blk, w.causal, w.sm_scale, w.rho)
+        self.qz = oracle.Quantised(self.Q, self.K, self.V)
+        self.rng = np.random.default_rng(11)
+
+    def run(self, n_rows):
+        w = self.w
+        rows = np.stack([self.rng.integers(0, w.B, n_rows), self.rng.integers(0, w.Hq, n_rows),
+                         self.rng.integers(0, w.N, n_rows)], 1).astype(np.int64)
+        t = time.perf_counter()
+        self.oracle.attention_rows(self.Q, self.K, self.V, self.mask, rows, w.blk, w.causal, w.sm_scale, self.qz)
+        dt = time.perf_counter() - t
+        keys = (rows[:, 2] + 1) if w.causal else np.full(n_rows, w.N)
+        return float(4.0 * w.D * keys.sum()), dt
+
+
+def cores_used():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(w, n_rows):
+    orc = OracleRows(w)
+    flops, dt = orc.run(n_rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+            "sample": f"{n_rows} seeded rows (random heads/positions) of {w.name}, attention stage, {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = WORKLOAD
+    orc = OracleRows(w)
+    for _ in range(args.warmup):
+        orc.run(args.ref_rows)
+    flops = secs = 0.0
+    for _ in range(args.steps):
+        f, dt = orc.run(args.ref_rows)
+        flops += f
+        secs += dt
+    v = flops / secs / 1e12
+    cb = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+          "sample": f"{args.ref_rows} seeded rows per step of {w.name}, attention stage", "seconds": round(secs, 2)}
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic",
+            "config": {"workload": w.name, "rho": w.rho, "blk": w.blk,
+                       "step": f"oracle attention on {args.ref_rows} sampled rows"},
+            "cpu_baseline": cb, "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                       "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

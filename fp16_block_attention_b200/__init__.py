@@ -1,0 +1,236 @@
+"""Python binding of ``libthrift.so``: selective mixed-precision (FP16 / NVFP4)
+block attention on B200 (sm_100a).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch supplies device memory and the stream.  The functions mirror the C ABI
+in ``include/thrift.h``:
+
+    quantize_nvfp4(x, op, shape)            -> (codes, scales)
+    select_blocks(Q, K, shape, rho)         -> mask [B, Hq, nb, nb] (u8, 1 = FP16 pair)
+    attention(Q, K, V, mask, qz, shape)     -> O
+    attention_fused(Q, K, V, shape, rho)    -> O
+
+There is no CPU fallback: importing fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libthrift.so")
+
+Q, K, V = 0, 1, 2  # thrift_operand
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA runtime error",
+           4: "a kernel gave up a bounded wait", 5: "workspace missing or too small"}
+
+
+class ThriftError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {_STATUS.get(status, 'unknown status')} (status {status})")
+        self.status = status
+
+
+class CShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("N", ctypes.c_int),
+                ("D", ctypes.c_int), ("blk", ctypes.c_int), ("causal", ctypes.c_int), ("sm_scale", ctypes.c_float)]
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    D: int
+    blk: int = 128
+    causal: bool = True
+    sm_scale: float | None = None
+
+    def c(self) -> CShape:
+        sm = self.sm_scale if self.sm_scale is not None else 1.0 / math.sqrt(self.D)
+        return CShape(self.B, self.Hq, self.Hkv, self.N, self.D, self.blk, int(self.causal), sm)
+
+    @property
+    def nb(self) -> int:
+        return self.N // self.blk
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fp16_block_attention_b200.build` "
+                          "(there is no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, st, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    psh = ctypes.POINTER(CShape)
+    sig = {
+        "thrift_quant_bytes": ([psh, st, ctypes.POINTER(sz), ctypes.POINTER(sz)], st),
+        "thrift_quantize_nvfp4": ([vp, st, psh, vp, vp, vp], st),
+        "thrift_select_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
+        "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
+        "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
+        "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_last_device_error": ([vp], st),
+        "thrift_strerror": ([st], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+# C-ABI symbols the header declares (checked by the tests).
+EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
+           "thrift_attention", "thrift_fused_workspace_bytes", "thrift_attention_fused", "thrift_last_device_error",
+           "thrift_strerror")
+
+
+def lib():
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise ThriftError(fn, status)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return t
+
+
+def shape_of(Q: torch.Tensor, K: torch.Tensor, blk: int = 128, causal: bool = True,
+             sm_scale: float | None = None) -> Shape:
+    B, Hq, N, D = Q.shape
+    return Shape(B, Hq, K.shape[1], N, D, blk, causal, sm_scale)
+
+
+def quant_bytes(shape: Shape, op: int):
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("thrift_quant_bytes", _lib.thrift_quant_bytes(ctypes.byref(shape.c()), op, ctypes.byref(c),
+                                                         ctypes.byref(s)))
+    return c.value, s.value
+
+
+def quantize_nvfp4(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=None, stream=None):
+    """NVFP4 copy of Q/K (along D) or V (along keys): (codes u8, scales u8)."""
+    _dev(x, "x", torch.float16)
+    nc, ns = quant_bytes(shape, op)
+    if codes is None:
+        codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
+    _check("thrift_quantize_nvfp4", _lib.thrift_quantize_nvfp4(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
+                                                               _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def select_workspace_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check("thrift_select_workspace_bytes", _lib.thrift_select_workspace_bytes(ctypes.byref(shape.c()),
+                                                                               ctypes.byref(n)))
+    return n.value
+
+
+def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, mask=None, ws=None, stream=None):
+    """Selection mask [B, Hq, nb, nb] (u8): 1 = FP16 block pair."""
+    _dev(Qt, "Q", torch.float16)
+    _dev(Kt, "K", torch.float16)
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
+    if ws is None:
+        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
+                                                             float(rho), _ptr(mask), _ptr(ws), ws.numel(),
+                                                             _stream(stream)))
+    return mask
+
+
+@dataclasses.dataclass
+class Quantised:
+    q4: torch.Tensor
+    qs: torch.Tensor
+    k4: torch.Tensor
+    ks: torch.Tensor
+    v4: torch.Tensor
+    vs: torch.Tensor
+
+
+def quantize_all(Qt, Kt, Vt, shape: Shape, stream=None) -> Quantised:
+    q4, qs = quantize_nvfp4(Qt, Q, shape, stream=stream)
+    k4, ks = quantize_nvfp4(Kt, K, shape, stream=stream)
+    v4, vs = quantize_nvfp4(Vt, V, shape, stream=stream)
+    return Quantised(q4, qs, k4, ks, v4, vs)
+
+
+def attention(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None):
+    """Mixed FP16/NVFP4 attention output O (fp16, shaped like Q)."""
+    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    _dev(mask, "mask", torch.uint8)
+    if out is None:
+        out = torch.empty_like(Qt)
+    _check("thrift_attention", _lib.thrift_attention(
+        _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
+        _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
+    return out
+
+
+def fused_workspace_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check("thrift_fused_workspace_bytes", _lib.thrift_fused_workspace_bytes(ctypes.byref(shape.c()),
+                                                                             ctypes.byref(n)))
+    return n.value
+
+
+def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, stream=None):
+    """Quantise, select (budget rho) and attend in one call."""
+    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    if out is None:
+        out = torch.empty_like(Qt)
+    if ws is None:
+        ws = torch.empty(fused_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_attention_fused", _lib.thrift_attention_fused(
+        _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return out
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise and read/clear the device error word (0 = none, 4 = a bounded wait timed out)."""
+    return int(_lib.thrift_last_device_error(_stream(stream)))
+
+
+def qk_scale_index(bh, n, g, NT, D):
+    """Byte offset of the scale of (row n, group g) in the Q/K scale layout (see thrift.h)."""
+    return ((bh * NT + n // 128) * (D // 64) + g // 4) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + (g % 4)
+
+
+def v_scale_index(bh, d, n, NT):
+    """Byte offset of the scale of (channel d, key group n//16) in the V scale layout."""
+    return (bh * 2 * NT + n // 64) * 512 + (d % 32) * 16 + (d // 32) * 4 + (n % 64) // 16

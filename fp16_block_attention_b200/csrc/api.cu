@@ -1,0 +1,222 @@
+// C ABI of the library (declared in include/thrift.h): argument checks,
+// workspace carving and kernel launches.  Nothing here allocates device
+// memory.
+#include <cmath>
+#include <cstdint>
+
+#include "common.h"
+
+namespace thrift {
+
+namespace {
+
+// Device error word: one per device, in the library's static device memory.
+__device__ uint32_t g_device_error;
+
+constexpr int kMaxDevices = 64;
+uint32_t* g_err_ptr[kMaxDevices] = {nullptr};
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+thrift_status from_cuda(cudaError_t e) { return e == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA; }
+
+struct QuantSizes {
+  size_t codes, scales;
+};
+
+QuantSizes quant_sizes(const thrift_shape& s, thrift_operand op) {
+  const size_t NT = static_cast<size_t>(num_tiles(s.N));
+  const size_t H = (op == THRIFT_Q) ? s.Hq : s.Hkv;
+  const size_t BH = static_cast<size_t>(s.B) * H;
+  QuantSizes q;
+  q.codes = BH * s.N * (s.D / 2);
+  if (op == THRIFT_V)
+    q.scales = BH * 2 * NT * 512;
+  else
+    q.scales = BH * NT * (s.D / 64) * 512;
+  return q;
+}
+
+struct FusedWs {
+  uint8_t *q4, *qs, *k4, *ks, *v4, *vs, *mask;
+  void* sel;
+  size_t total;
+};
+
+FusedWs carve_fused(void* base, const thrift_shape& s) {
+  FusedWs w;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* r = p ? p + off : nullptr;
+    off += align_up(bytes);
+    return reinterpret_cast<uint8_t*>(r);
+  };
+  const QuantSizes q = quant_sizes(s, THRIFT_Q), k = quant_sizes(s, THRIFT_K), v = quant_sizes(s, THRIFT_V);
+  w.q4 = take(q.codes);
+  w.qs = take(q.scales);
+  w.k4 = take(k.codes);
+  w.ks = take(k.scales);
+  w.v4 = take(v.codes);
+  w.vs = take(v.scales);
+  const size_t nb = s.N / s.blk;
+  w.mask = take(static_cast<size_t>(s.B) * s.Hq * nb * nb);
+  w.sel = take(select_workspace_bytes(s));
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+uint32_t* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+thrift_status check_shape(const thrift_shape* s) {
+  if (!s) return THRIFT_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->N <= 0 || s->D <= 0 || s->blk <= 0) return THRIFT_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return THRIFT_ERR_INVALID_ARG;
+  if (!std::isfinite(s->sm_scale)) return THRIFT_ERR_INVALID_ARG;
+  if (s->causal != 0 && s->causal != 1) return THRIFT_ERR_INVALID_ARG;
+  if (s->D != 64 && s->D != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (s->blk != 64 && s->blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  if (s->N % s->blk != 0) return THRIFT_ERR_UNSUPPORTED;
+  if (s->N > 131072) return THRIFT_ERR_UNSUPPORTED;                       // key tiles per query tile <= 1024
+  if (static_cast<long long>(s->B) * s->Hq > 65535) return THRIFT_ERR_UNSUPPORTED;  // grid y/z extents
+  return THRIFT_OK;
+}
+
+}  // namespace thrift
+
+using namespace thrift;
+
+extern "C" {
+
+thrift_status thrift_quant_bytes(const thrift_shape* shape, thrift_operand op, size_t* codes_bytes,
+                                 size_t* scales_bytes) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (op != THRIFT_Q && op != THRIFT_K && op != THRIFT_V) return THRIFT_ERR_INVALID_ARG;
+  if (!codes_bytes || !scales_bytes) return THRIFT_ERR_INVALID_ARG;
+  const QuantSizes q = quant_sizes(*shape, op);
+  *codes_bytes = q.codes;
+  *scales_bytes = q.scales;
+  return THRIFT_OK;
+}
+
+thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
+                                    void* scales, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (op != THRIFT_Q && op != THRIFT_K && op != THRIFT_V) return THRIFT_ERR_INVALID_ARG;
+  if (!x || !codes || !scales) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return THRIFT_ERR_INVALID_ARG;
+  const thrift_shape& s = *shape;
+  const size_t H = (op == THRIFT_Q) ? s.Hq : s.Hkv;
+  const size_t BH = static_cast<size_t>(s.B) * H;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (op == THRIFT_V) return from_cuda(launch_quantize_v(x, BH, s.N, s.D, codes, scales, cs));
+  return from_cuda(launch_quantize_qk(x, BH * s.N, s.N, s.D, codes, scales, cs));
+}
+
+thrift_status thrift_select_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!bytes) return THRIFT_ERR_INVALID_ARG;
+  *bytes = select_workspace_bytes(*shape);
+  return THRIFT_OK;
+}
+
+thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
+                                   uint8_t* mask, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!Q || !K || !mask || !(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return THRIFT_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < select_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  return from_cuda(launch_select(Q, K, *shape, rho, mask, ws, static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
+                               const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
+                               const thrift_shape* shape, void* O, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  const void* ptrs[] = {Q, K, V, q4, qs, k4, ks, v4, vs, O};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return THRIFT_ERR_INVALID_ARG;
+  if (!mask) return THRIFT_ERR_INVALID_ARG;
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  return from_cuda(
+      launch_attention(Q, K, V, mask, q4, qs, k4, ks, v4, vs, *shape, O, err, static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!bytes) return THRIFT_ERR_INVALID_ARG;
+  *bytes = carve_fused(nullptr, *shape).total;
+  return THRIFT_OK;
+}
+
+thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V, const thrift_shape* shape,
+                                     double rho, void* O, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!Q || !K || !V || !O || !(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return THRIFT_ERR_INVALID_ARG;
+  const FusedWs need = carve_fused(nullptr, *shape);
+  if (!ws || ws_bytes < need.total || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  const FusedWs w = carve_fused(ws, *shape);
+  const thrift_shape& s = *shape;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  if (launch_quantize_qk(Q, static_cast<size_t>(s.B) * s.Hq * s.N, s.N, s.D, w.q4, w.qs, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (launch_quantize_qk(K, static_cast<size_t>(s.B) * s.Hkv * s.N, s.N, s.D, w.k4, w.ks, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (launch_select(Q, K, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, err, cs));
+}
+
+thrift_status thrift_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return THRIFT_ERR_CUDA;
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return THRIFT_ERR_CUDA;
+    return THRIFT_ERR_TIMEOUT;
+  }
+  return THRIFT_OK;
+}
+
+const char* thrift_strerror(thrift_status status) {
+  switch (status) {
+    case THRIFT_OK: return "ok";
+    case THRIFT_ERR_INVALID_ARG: return "invalid argument";
+    case THRIFT_ERR_UNSUPPORTED: return "unsupported shape";
+    case THRIFT_ERR_CUDA: return "CUDA runtime error";
+    case THRIFT_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case THRIFT_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

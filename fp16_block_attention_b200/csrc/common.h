@@ -1,0 +1,47 @@
+// Shared host/device definitions of the library: shape checks, buffer sizes,
+// the scale-factor layout and the kernel launch entry points.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/thrift.h"
+
+namespace thrift {
+
+constexpr int kTile = 128;        // rows of a query tile and keys of a key tile
+constexpr int kPLog2 = 11;        // pre-scale 2^11 of P before its FP16 / NVFP4 encoding
+constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every in-kernel wait (2 s)
+
+__host__ __device__ inline int num_tiles(int N) { return (N + kTile - 1) / kTile; }
+
+// Validate a shape; returns THRIFT_OK, INVALID_ARG or UNSUPPORTED.
+thrift_status check_shape(const thrift_shape* s);
+
+// Byte offset of the scale of (row n, 16-group g) of a Q/K operand.
+__host__ __device__ inline size_t qk_scale_index(size_t bh, int n, int g, int NT, int D) {
+  return ((bh * NT + static_cast<size_t>(n / kTile)) * (D / 64) + g / 4) * 512 + (n % 32) * 16 +
+         ((n % kTile) / 32) * 4 + (g % 4);
+}
+// Byte offset of the scale of (channel d, key group n/16) of V.
+__host__ __device__ inline size_t v_scale_index(size_t bh, int d, int n, int NT) {
+  return (bh * 2 * NT + static_cast<size_t>(n / 64)) * 512 + (d % 32) * 16 + (d / 32) * 4 + (n % 64) / 16;
+}
+
+// Device error word of the current device (allocated statically in the library).
+uint32_t* device_error_word();
+
+// ---- launchers (return cudaError_t of the launch) --------------------------
+cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* codes, void* scales,
+                               cudaStream_t st);
+cudaError_t launch_quantize_v(const void* v, size_t bh, int N, int D, void* codes, void* scales, cudaStream_t st);
+
+size_t select_workspace_bytes(const thrift_shape& s);
+cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
+                          cudaStream_t st);
+
+cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
+                             const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
+                             const thrift_shape& s, void* O, uint32_t* err, cudaStream_t st);
+
+}  // namespace thrift

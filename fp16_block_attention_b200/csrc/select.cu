@@ -1,0 +1,199 @@
+// Stage 1 of the method: "a heuristic rapidly selects a small number of
+// important query-key block pairs for FP16 precision" (ThriftAttention
+// abstract).  Reading used here: pooled scores from FP32 block means,
+// score(i,j) = fl32(sm_scale * fl32(mean_q(i) . mean_k(j))), and per
+// (batch, query head) the top k = ceil(rho * #valid - 1e-9) pairs, with the
+// diagonal pairs (i,i) and the key-block-0 pairs (i,0) ranked first and ties
+// broken by the lower linear index i*nb + j.
+//
+// Three kernels:
+//   pool     block means: the FP64 sum of a block's fp16 rows is exact in any
+//            order (40-bit span + log2(blk) bits < 53), divided by blk and
+//            rounded once to FP32;
+//   scores   the FP64 dot product of two FP32 means (products exact in FP64),
+//            rounded to FP32, times sm_scale in FP32;
+//   top-k    one CTA per head: radix select of the k-th largest 64-bit key
+//            (forced bit | order-preserving score bits | inverted index), so
+//            the selection is exactly k pairs, then the mask.
+#include <cuda_fp16.h>
+
+#include "common.h"
+
+namespace thrift {
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct SelectWs {
+  float* qm;      // [B*Hq][nb][D]
+  float* km;      // [B*Hkv][nb][D]
+  float* scores;  // [B*Hq][nb][nb]
+};
+
+SelectWs carve(void* ws, const thrift_shape& s) {
+  const int nb = s.N / s.blk;
+  char* p = static_cast<char*>(ws);
+  SelectWs w;
+  w.qm = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * static_cast<size_t>(s.B) * s.Hq * nb * s.D);
+  w.km = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * static_cast<size_t>(s.B) * s.Hkv * nb * s.D);
+  w.scores = reinterpret_cast<float*>(p);
+  return w;
+}
+
+// grid (nb, BH), block D/2 threads, two channels per thread.
+__global__ void pool_kernel(const __half* __restrict__ x, int N, int D, int blk, float* __restrict__ out) {
+  const int nb = N / blk;
+  const size_t bh = blockIdx.y;
+  const int i = blockIdx.x;
+  const int c = threadIdx.x;  // channel pair
+  const __half2* src = reinterpret_cast<const __half2*>(x + (bh * N + static_cast<size_t>(i) * blk) * D) + c;
+  double s0 = 0.0, s1 = 0.0;
+  for (int r = 0; r < blk; ++r) {
+    const float2 f = __half22float2(src[static_cast<size_t>(r) * (D / 2)]);
+    s0 += static_cast<double>(f.x);
+    s1 += static_cast<double>(f.y);
+  }
+  float* dst = out + (bh * nb + i) * D + 2 * c;
+  dst[0] = static_cast<float>(s0 / blk);
+  dst[1] = static_cast<float>(s1 / blk);
+}
+
+// grid (ceil(nb/32), ceil(nb/32), B*Hq), block 256: a 32x32 tile of scores,
+// each thread a 2x2 sub-tile.
+__global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qm, const float* __restrict__ km,
+                                                    int Hq, int Hkv, int nb, int D, int causal, float sm_scale,
+                                                    float* __restrict__ scores) {
+  __shared__ float qs[32][129];
+  __shared__ float ks[32][129];
+  const int bi = blockIdx.y * 32, bj = blockIdx.x * 32;
+  if (causal && bj > bi + 31) return;
+  const size_t bh = blockIdx.z;
+  const size_t b = bh / Hq, hq = bh % Hq;
+  const size_t bhk = b * Hkv + hq / (Hq / Hkv);
+  for (int t = threadIdx.x; t < 32 * D; t += blockDim.x) {
+    const int r = t / D, d = t % D;
+    qs[r][d] = (bi + r < nb) ? qm[(bh * nb + bi + r) * D + d] : 0.0f;
+    ks[r][d] = (bj + r < nb) ? km[(bhk * nb + bj + r) * D + d] : 0.0f;
+  }
+  __syncthreads();
+  const int ti = (threadIdx.x / 16) * 2, tj = (threadIdx.x % 16) * 2;
+  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  for (int d = 0; d < D; ++d) {
+    const double q0 = qs[ti][d], q1 = qs[ti + 1][d], k0 = ks[tj][d], k1 = ks[tj + 1][d];  // exact widening
+    acc[0][0] = fma(q0, k0, acc[0][0]);
+    acc[0][1] = fma(q0, k1, acc[0][1]);
+    acc[1][0] = fma(q1, k0, acc[1][0]);
+    acc[1][1] = fma(q1, k1, acc[1][1]);
+  }
+  for (int a = 0; a < 2; ++a)
+    for (int c = 0; c < 2; ++c) {
+      const int i = bi + ti + a, j = bj + tj + c;
+      if (i < nb && j < nb && (!causal || j <= i))
+        scores[(bh * nb + i) * nb + j] = __fmul_rn(sm_scale, static_cast<float>(acc[a][c]));
+    }
+}
+
+__device__ __forceinline__ uint64_t pair_key(float score, int i, int j, int nb) {
+  if (score == 0.0f) score = 0.0f;  // one zero
+  uint32_t u = __float_as_uint(score);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint64_t forced = (i == j || j == 0) ? 1ull : 0ull;
+  const uint64_t idx = static_cast<uint64_t>(i) * nb + j;
+  return (forced << 63) | (static_cast<uint64_t>(u) << 31) | (0x7FFFFFFFull - idx);
+}
+
+// One CTA (1024 threads) per (batch, query head).
+__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int nb, int causal,
+                                                    long long k, uint8_t* __restrict__ mask) {
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ long long s_remaining;
+  __shared__ int s_done;
+  const size_t bh = blockIdx.x;
+  const float* sc = scores + bh * nb * static_cast<size_t>(nb);
+  uint8_t* m = mask + bh * nb * static_cast<size_t>(nb);
+  const size_t total = static_cast<size_t>(nb) * nb;
+  const long long valid = causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(total);
+
+  uint64_t threshold;  // select keys >= threshold
+  bool select_none = (k <= 0);
+  if (k >= valid) {
+    threshold = 0;  // every valid pair
+  } else if (select_none) {
+    threshold = ~0ull;
+  } else {
+    if (threadIdx.x == 0) {
+      s_prefix = 0;
+      s_remaining = k;
+      s_done = 0;
+    }
+    uint64_t pmask = 0;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
+      __syncthreads();
+      const uint64_t prefix = s_prefix;
+      for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
+        const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
+        if (causal && j > i) continue;
+        const uint64_t key = pair_key(sc[idx], i, j, nb);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        long long rem = s_remaining, cum = 0;
+        int digit = 0;
+        for (int d = 255; d >= 0; --d) {
+          if (cum + hist[d] >= rem) {
+            digit = d;
+            break;
+          }
+          cum += hist[d];
+        }
+        rem -= cum;
+        s_prefix = prefix | (static_cast<uint64_t>(digit) << shift);
+        s_remaining = rem;
+        s_done = (static_cast<long long>(hist[digit]) == rem);
+      }
+      __syncthreads();
+      pmask |= 255ull << shift;
+      if (s_done) break;
+    }
+    threshold = s_prefix;
+  }
+  for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
+    uint8_t v = 0;
+    if (!(causal && j > i) && !select_none) v = pair_key(sc[idx], i, j, nb) >= threshold ? 1 : 0;
+    m[idx] = v;
+  }
+}
+
+}  // namespace
+
+size_t select_workspace_bytes(const thrift_shape& s) {
+  const size_t nb = s.N / s.blk;
+  return align_up(sizeof(float) * s.B * s.Hq * nb * s.D) + align_up(sizeof(float) * s.B * s.Hkv * nb * s.D) +
+         align_up(sizeof(float) * s.B * s.Hq * nb * nb);
+}
+
+cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
+                          cudaStream_t st) {
+  const int nb = s.N / s.blk;
+  SelectWs w = carve(ws, s);
+  pool_kernel<<<dim3(nb, s.B * s.Hq), s.D / 2, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
+  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
+  const int tiles = (nb + 31) / 32;
+  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
+                                                               s.sm_scale, w.scores);
+  const long long valid = s.causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
+  double kk = ceil(rho * static_cast<double>(valid) - 1e-9);
+  if (kk < 0) kk = 0;
+  if (kk > static_cast<double>(valid)) kk = static_cast<double>(valid);
+  topk_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, static_cast<long long>(kk), mask);
+  return cudaGetLastError();
+}
+
+}  // namespace thrift

@@ -1,0 +1,149 @@
+/*
+ * thrift.h -- C ABI of the selective mixed-precision (FP16 / NVFP4) block
+ * attention library for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "ThriftAttention: Selective Mixed Precision for
+ * Long-Context FP4 Attention", abstract; same page's summary, "technical
+ * approach" items 2-5) computes prefill attention in two stages:
+ *   1. a cheap heuristic picks a small fraction rho of (query block, key
+ *      block) pairs to run in FP16                 -> thrift_select_blocks
+ *   2. the picked pairs run in FP16, all other pairs in block-scaled FP4, and
+ *      one online softmax merges both into one output -> thrift_attention
+ * The FP4 operands come from                       -> thrift_quantize_nvfp4
+ * and thrift_attention_fused chains all of them.
+ *
+ * Readings of points the pages leave open (each is fixed, not tunable):
+ *   - NVFP4: E2M1 codes with one E4M3 scale per 16 consecutive elements along
+ *     the contracted axis, scale = E4M3_rn(amax/6) with amax/6 rounded to
+ *     FP32, code = E2M1_rn(x/scale) (ties to even, saturating, sign kept);
+ *     a zero scale encodes the whole group as +0.
+ *   - Q and K are quantised along D, V along the key axis, P (the softmax
+ *     numerators) per 16 keys, at a fixed pre-scale of 2^11 that the output
+ *     divides out again.
+ *   - Heuristic: score(i,j) = fl32(sm_scale * fl32(mean_q(i) . mean_k(j)))
+ *     from FP32 block means; per (batch, query head) keep
+ *     k = ceil(rho * #valid_pairs - 1e-9) pairs, diagonal pairs (i,i) and
+ *     key-block-0 pairs (i,0) first, then by score, ties to the lower linear
+ *     index i*nb + j.
+ *   - Online softmax keeps an integer running maximum of the log2-domain
+ *     logits, so every rescale is an exact power of two; the row sum l adds
+ *     the unquantised P.
+ *
+ * Conventions for every call:
+ *   - Pointers named Q, K, V, O, mask, codes, scales, ws are DEVICE pointers,
+ *     owned by the caller; the library allocates no device memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); calls only
+ *     enqueue work and return without synchronising.
+ *   - Arguments are validated on the host before any launch; on error nothing
+ *     is launched and the status says why.
+ *   - Device-side faults are never raised on purpose: every wait inside a
+ *     kernel is bounded; a timeout sets a device error word that
+ *     thrift_last_device_error() reads (and clears).
+ *   - Tensors are contiguous, row-major:
+ *       Q [B][Hq][N][D] fp16, K and V [B][Hkv][N][D] fp16, O like Q.
+ *     Query head h reads key/value head h / (Hq/Hkv).
+ *   - Supported shapes: D in {64, 128}; blk in {64, 128}; N a positive
+ *     multiple of blk; Hq a multiple of Hkv; all sizes positive.  Other
+ *     shapes return THRIFT_ERR_UNSUPPORTED.
+ */
+#ifndef THRIFT_H_
+#define THRIFT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define THRIFT_API __attribute__((visibility("default")))
+#else
+#define THRIFT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  THRIFT_OK = 0,
+  THRIFT_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, rho outside [0,1] */
+  THRIFT_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (see above) */
+  THRIFT_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, attribute, copy) */
+  THRIFT_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait (device error word) */
+  THRIFT_ERR_WORKSPACE = 5    /* workspace pointer null or too small */
+} thrift_status;
+
+typedef enum { THRIFT_Q = 0, THRIFT_K = 1, THRIFT_V = 2 } thrift_operand;
+
+/* Problem shape.  sm_scale multiplies Q K^T (usually 1/sqrt(D)); causal = 1
+ * masks key > query.  blk is the selection block (square, blk x blk). */
+typedef struct {
+  int B, Hq, Hkv, N, D, blk, causal;
+  float sm_scale;
+} thrift_shape;
+
+/* Sizes of the NVFP4 copy of one operand.
+ * Codes (canonical, also what the attention kernel reads by TMA):
+ *   Q/K: [B][H][N][D/2] bytes, element d in the low nibble of byte d/2 when
+ *        d is even, high nibble when odd;
+ *   V:   [B][Hkv][D][N/2] bytes (keys contiguous), key n in nibble n%2.
+ * Scales (E4M3 bytes) in the tensor-core scale-factor layout, with
+ * NT = ceil(N/128):
+ *   Q/K: [B][H][NT][D/64][32][4][4]; the scale of row n, group g = d/16 sits at
+ *        ((bh*NT + n/128)*(D/64) + g/4)*512 + (n%32)*16 + ((n%128)/32)*4 + g%4;
+ *   V:   [B][Hkv][2*NT][32][4][4]; the scale of channel d, key group n/16 sits at
+ *        (bh*2*NT + n/64)*512 + (d%32)*16 + (d/32)*4 + (n%64)/16.
+ * Padding bytes (rows past N, channels past D) are written as 0.
+ * Returns INVALID_ARG / UNSUPPORTED like the calls below. */
+THRIFT_API thrift_status thrift_quant_bytes(const thrift_shape* shape, thrift_operand op, size_t* codes_bytes,
+                                 size_t* scales_bytes);
+
+/* NVFP4 quantisation of one operand (Q or K along D, V along keys).
+ * x: fp16 device tensor of the operand's shape; codes/scales: device buffers
+ * of thrift_quant_bytes() sizes.  Block-scaled FP4 as the pages' prior work
+ * on Blackwell ("ThriftAttention" abstract); the format is the NVFP4 reading
+ * above. */
+THRIFT_API thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
+                                    void* scales, void* stream);
+
+/* Workspace bytes thrift_select_blocks needs (block means and pooled scores). */
+THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape, size_t* bytes);
+
+/* Stage 1 ("a heuristic rapidly selects a small number of important
+ * query-key block pairs", ThriftAttention abstract): writes
+ * mask [B][Hq][nb][nb] (nb = N/blk) with 1 for pairs computed in FP16 and 0
+ * for FP4 pairs and for invalid (causal, j > i) pairs.
+ * rho in [0,1]; ws: device workspace of at least
+ * thrift_select_workspace_bytes() bytes (contents need not be initialised). */
+THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
+                                   uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 2 ("the selected blocks are computed in FP16 and the remaining blocks
+ * in FP4, with both paths merged via online softmax into a single output",
+ * ThriftAttention abstract): O [B][Hq][N][D] fp16.
+ * mask: as written by thrift_select_blocks; q4/qs, k4/ks, v4/vs: the NVFP4
+ * copies written by thrift_quantize_nvfp4 for Q, K and V. */
+THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
+                               const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
+                               const thrift_shape* shape, void* O, void* stream);
+
+/* Workspace bytes of thrift_attention_fused (NVFP4 copies, mask and the
+ * selection workspace, each 256-byte aligned). */
+THRIFT_API thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape, size_t* bytes);
+
+/* Both stages in one call: quantise Q, K, V, select with budget rho, attend.
+ * ws: device workspace of thrift_fused_workspace_bytes() bytes. */
+THRIFT_API thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V, const thrift_shape* shape,
+                                     double rho, void* O, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the device error word of the current
+ * device: THRIFT_OK, or THRIFT_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call, or THRIFT_ERR_CUDA if the synchronisation failed. */
+THRIFT_API thrift_status thrift_last_device_error(void* stream);
+
+/* Static, human-readable name of a status. */
+THRIFT_API const char* thrift_strerror(thrift_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THRIFT_H_ */

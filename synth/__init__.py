@@ -133,14 +133,16 @@ def f16_bits(x: float) -> int:
     return int(_load().synth_f16(float(x)))
 
 
-def sample_rows(w: Workload, count: int, seed: int = 7):
-    """Deterministic row sample (b, hq, r): every row of q-blocks {0, 1, nb/2, nb-1} of the
-    first (b, hq) plus `count` seeded random rows spread over the heads."""
+def sample_rows(w: Workload, count: int, seed: int = 7, per_block: int | None = None):
+    """Deterministic row sample (b, hq, r): rows of q-blocks {0, 1, nb/2, nb-1} of the
+    first (b, hq) (all of them, or `per_block` evenly spaced ones) plus `count`
+    seeded random rows spread over the heads."""
     rng = np.random.default_rng(seed)
     nb = w.N // w.blk
+    step = 1 if per_block is None else max(1, w.blk // per_block)
     rows = []
     for qb in sorted({0, min(1, nb - 1), nb // 2, nb - 1}):
-        for r in range(qb * w.blk, (qb + 1) * w.blk):
+        for r in range(qb * w.blk, (qb + 1) * w.blk, step):
             rows.append((0, 0, r))
     for _ in range(count):
         rows.append((int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.N))))

@@ -1,0 +1,78 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp16_block_attention_b200 as thrift
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_symbols():
+    text = open(os.path.join(ROOT, "include", "thrift.h")).read()
+    return set(re.findall(r"THRIFT_API\s+[\w\s\*]+?\b(thrift_\w+)\s*\(", text))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _header_symbols()
+    assert declared == set(thrift.EXPORTS)
+    lib = ctypes.CDLL(thrift.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def _c(**kw):
+    base = dict(B=1, Hq=2, Hkv=1, N=256, D=128, blk=128, causal=1, sm_scale=0.088)
+    base.update(kw)
+    return thrift.CShape(base["B"], base["Hq"], base["Hkv"], base["N"], base["D"], base["blk"], base["causal"],
+                         base["sm_scale"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0),
+    (dict(B=0), 1), (dict(N=-64), 1), (dict(Hq=3, Hkv=2), 1), (dict(causal=2), 1),
+    (dict(sm_scale=float("nan")), 1),
+    (dict(D=96), 2), (dict(blk=32), 2), (dict(N=200), 2), (dict(N=64, blk=128), 2), (dict(N=262144), 2),
+])
+def test_shape_validation(kw, status):
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    assert thrift.lib().thrift_quant_bytes(ctypes.byref(_c(**kw)), 0, ctypes.byref(c), ctypes.byref(s)) == status
+
+
+def test_quant_bytes_layout_sizes():
+    sh = thrift.Shape(2, 4, 2, 192, 128, 64, True)
+    assert thrift.quant_bytes(sh, thrift.Q) == (2 * 4 * 192 * 64, 2 * 4 * 2 * 2 * 512)
+    assert thrift.quant_bytes(sh, thrift.K) == (2 * 2 * 192 * 64, 2 * 2 * 2 * 2 * 512)
+    assert thrift.quant_bytes(sh, thrift.V) == (2 * 2 * 192 * 64, 2 * 2 * 4 * 512)
+
+
+def test_null_pointers_and_bad_rho_are_rejected_before_launch():
+    lib = thrift.lib()
+    sh = ctypes.byref(_c())
+    fake = ctypes.c_void_p(256)
+    assert lib.thrift_quantize_nvfp4(None, 0, sh, fake, fake, None) == 1
+    assert lib.thrift_quantize_nvfp4(fake, 7, sh, fake, fake, None) == 1
+    assert lib.thrift_quantize_nvfp4(ctypes.c_void_p(258), 0, sh, fake, fake, None) == 1  # misaligned
+    assert lib.thrift_select_blocks(fake, fake, sh, 1.5, fake, fake, 1 << 30, None) == 1
+    assert lib.thrift_select_blocks(fake, fake, sh, 0.05, fake, None, 0, None) == 5
+    assert lib.thrift_select_blocks(fake, fake, sh, 0.05, fake, fake, 16, None) == 5
+    args = [fake] * 10
+    assert lib.thrift_attention(None, *args[:9], sh, fake, None) == 1
+    assert lib.thrift_attention_fused(fake, fake, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1
+    assert lib.thrift_attention_fused(fake, fake, fake, sh, 0.05, fake, fake, 8, None) == 5
+
+
+def test_workspace_sizes_cover_the_parts():
+    sh = thrift.Shape(1, 4, 2, 512, 128, 64, True)
+    need = thrift.fused_workspace_bytes(sh)
+    parts = sum(sum(thrift.quant_bytes(sh, op)) for op in (0, 1, 2)) + 4 * 8 * 8 + thrift.select_workspace_bytes(sh)
+    assert need >= parts
+
+
+def test_strerror_names_every_status():
+    lib = thrift.lib()
+    names = {lib.thrift_strerror(i).decode() for i in range(6)}
+    assert len(names) == 6 and "ok" in names
