@@ -299,15 +299,20 @@ def run_gpu(args):
 
 
 def attention_bytes(w, mask_np):
-    """Algorithmic HBM bytes of one attention launch: NVFP4 Q, K, V (0.5625 B per
-    element) read once, fp16 K/V of FP16 key tiles once per query head that
-    selects them, fp16 Q of query tiles with an FP16 pair, and O (2 B/elt)."""
+    """Algorithmic (minimum) HBM bytes of one attention launch: the NVFP4 copies of
+    Q, K, V (0.5 B code + 1/16 B scale per element) read once; the fp16 K and V
+    tiles that some query head of their group computes in FP16, once each; the
+    fp16 Q tiles with at least one FP16 pair, once each; O written once (2 B per
+    element); the mask."""
+    nb = w.N // w.blk
+    G = w.Hq // w.Hkv
     e_q = w.B * w.Hq * w.N * w.D
     e_kv = w.B * w.Hkv * w.N * w.D
-    per_tile = w.blk * w.D * 2 * 2  # fp16 K and V of one key block
-    q_tiles16 = int((mask_np.reshape(w.B, w.Hq, w.N // w.blk, -1).max(-1) == 1).sum())
-    return 0.5625 * e_q + 2 * 0.5625 * e_kv + float((mask_np == 1).sum()) * per_tile + \
-        q_tiles16 * w.blk * w.D * 2 + 2 * e_q
+    m = mask_np.reshape(w.B, w.Hkv, G, nb, nb) == 1
+    kv_tiles16 = int(m.any(axis=(2, 3)).sum())          # (b, kv head, key block) used in FP16
+    q_tiles16 = int(m.any(axis=4).sum())                  # (b, q head, query block) with an FP16 pair
+    return (0.5625 * e_q + 2 * 0.5625 * e_kv + kv_tiles16 * w.blk * w.D * 2 * 2 +
+            q_tiles16 * w.blk * w.D * 2 + 2 * e_q + mask_np.size)
 
 
 # --------------------------------------------------------- the CPU oracle ---
@@ -383,8 +388,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=512)
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
