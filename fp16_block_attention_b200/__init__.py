@@ -90,8 +90,8 @@ _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
-           "thrift_attention", "thrift_fused_workspace_bytes", "thrift_attention_fused", "thrift_last_device_error",
-           "thrift_strerror")
+           "thrift_attention", "thrift_fused_workspace_bytes",
+           "thrift_attention_fused", "thrift_last_device_error", "thrift_strerror")
 
 
 def lib():

@@ -86,7 +86,7 @@ thrift_status check_shape(const thrift_shape* s) {
   if (!s) return THRIFT_ERR_INVALID_ARG;
   if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->N <= 0 || s->D <= 0 || s->blk <= 0) return THRIFT_ERR_INVALID_ARG;
   if (s->Hq % s->Hkv != 0) return THRIFT_ERR_INVALID_ARG;
-  if (!std::isfinite(s->sm_scale)) return THRIFT_ERR_INVALID_ARG;
+  if (!std::isfinite(s->sm_scale) || !(s->sm_scale > 0.0f)) return THRIFT_ERR_INVALID_ARG;  // softmax scale > 0
   if (s->causal != 0 && s->causal != 1) return THRIFT_ERR_INVALID_ARG;
   if (s->D != 64 && s->D != 128) return THRIFT_ERR_UNSUPPORTED;
   if (s->blk != 64 && s->blk != 128) return THRIFT_ERR_UNSUPPORTED;

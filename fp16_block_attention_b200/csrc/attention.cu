@@ -146,6 +146,38 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float max16(const float* v) {
+  const float a = fmax3(v[0], v[1], v[2]), b = fmax3(v[3], v[4], v[5]), c = fmax3(v[6], v[7], v[8]);
+  const float d = fmax3(v[9], v[10], v[11]), e = fmax3(v[12], v[13], v[14]);
+  return fmaxf(fmax3(a, b, c), fmax3(d, e, v[15]));
+}
+
+// Pairwise (tree) sums: short dependency chains.
+__device__ __forceinline__ float sum16(const float* v) {
+  float t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = v[i] + v[i + 8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t[i] += t[i + 4];
+  return (t[0] + t[2]) + (t[1] + t[3]);
+}
+
+__device__ __forceinline__ float sum64(const float* v) {
+  return (sum16(v) + sum16(v + 16)) + (sum16(v + 32) + sum16(v + 48));
+}
+
 // 2^e for an integer-valued e <= 0 (0 below the normal range).
 __device__ __forceinline__ float exp2_int(float e) {
   const int i = static_cast<int>(e);
@@ -401,16 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float s[64];
       if (!failed) {
-        uint32_t v[32];
+        uint32_t v[64];
         const uint32_t col = lane_base + (fp16 ? kColS16 : kColS4) + 64 * half;
-        tmem_ld32(col, v);
+        tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
-        tmem_ld32(col + 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
+        for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(v[j]);
         tc_fence_before();
         mbar_arrive(&ms.bar_s_free);
       } else {
@@ -418,27 +447,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 64; ++j) s[j] = -INFINITY;
       }
 
-      // logits in the log2 domain, masked
+      // Mask keys past N and, on the diagonal tile, keys after the query.
       const int key0 = kt * 128 + 64 * half;
-      float tmax = -INFINITY;
+      if (kt * 128 + 128 > p.N || (p.causal && kt == qt)) {
+        const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys < lim are valid
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const int k = key0 + j;
-        const bool valid = (k < p.N) && (!p.causal || k <= qrow);
-        s[j] = valid ? s[j] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[j]);
+        for (int j = 0; j < 64; ++j)
+          if (key0 + j >= lim) s[j] = -INFINITY;
       }
-      ms.red_max[kt & 1][half][r] = tmax;
+      // Group maxima of the raw scores (sm_scale > 0, so the order is that of t).
+      float gm[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) gm[g] = max16(&s[16 * g]);
+      float smax = fmax3(fmaxf(gm[0], gm[1]), gm[2], gm[3]);
+      ms.red_max[kt & 1][half][r] = smax;
       if (softmax_bar_or(failed)) break;
-      tmax = fmaxf(tmax, ms.red_max[kt & 1][half ^ 1][r]);
-      const float Mn = fmaxf(M, ceilf(tmax));
+      smax = fmaxf(smax, ms.red_max[kt & 1][half ^ 1][r]);
+      // t = fl32(S * sm_scale * log2 e) is monotone in S: the row maximum of t is
+      // fl32(max S * c).
+      const float c2 = p.scale_log2;
+      const float Mn = fmaxf(M, ceilf(smax * c2));
       const float alpha = (M == -INFINITY) ? 0.f : exp2_int(M - Mn);
       const float Mx = (Mn == -INFINITY) ? 0.f : Mn;
-      float rs = 0.f;
+      const float base = static_cast<float>(kPLog2) - Mx;  // exponent offset of P * 2^11
+
+      // P * 2^11 = 2^(S*c + 11 - M); NVFP4 groups fold 1/scale into the exponent.
+      float rs;
+      uint32_t codes[8];
+      uint32_t sfw = 0;
+      if (fp16) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        s[j] = ex2(s[j] - Mx);
-        rs += s[j];
+        for (int j = 0; j < 64; ++j) s[j] = ex2(fmaf(s[j], c2, base));
+        rs = sum64(s);
+      } else {
+        rs = 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float amax = ex2(fmaf(gm[g], c2, base));                      // max of P * 2^11
+          const uint32_t sb = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;  // E4M3(amax / 6)
+          const float sc = e4m3_to_f32(sb);
+          const float sce = sc > 0.f ? sc : 1.0f;  // zero scale: codes round to 0, l keeps P
+          const float bias = base - lg2(sce);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[16 * g + i] = ex2(fmaf(s[16 * g + i], c2, bias));
+          rs = fmaf(sum16(&s[16 * g]), sce, rs);
+          uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) w0 |= cvt_e2m1x2(s[16 * g + i], s[16 * g + i + 1]) << (i * 4);
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) w1 |= cvt_e2m1x2(s[16 * g + 8 + i], s[16 * g + 9 + i]) << (i * 4);
+          codes[2 * g] = w0;
+          codes[2 * g + 1] = w1;
+          sfw |= sb << (8 * g);
+        }
       }
       l = l * alpha + rs;
 
@@ -447,34 +508,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             !wait_or_abort(&ms.bar_o_done, (kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA));
         if (failed) continue;  // the next joint barrier ends the loop for every softmax thread
         tc_fence_after();
-        // Rows whose maximum did not move have alpha = 1; the warp rescales together.
-        if (__any_sync(0xffffffffu, Mn > M)) {
-#pragma unroll
-          for (int cc = 0; cc < D / 64; ++cc) {
-            uint32_t v[32];
-            const uint32_t col = lane_base + kColO + (D / 2) * half + 32 * cc;
-            tmem_ld32(col, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-            tmem_st32(col, v);
-          }
-          tmem_st_wait();
-        }
       }
-      M = Mn;
 
-      // encode P * 2^11 for the P V product
-      const float pre = static_cast<float>(1 << kPLog2);
+      // write the encoded P for the P V product (P * 2^11)
       if (fp16) {
         uint8_t* dst = sm + L::kP16 + half * 16384;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint4 w;
-          w.x = pack_half2(s[8 * ch + 0] * pre, s[8 * ch + 1] * pre);
-          w.y = pack_half2(s[8 * ch + 2] * pre, s[8 * ch + 3] * pre);
-          w.z = pack_half2(s[8 * ch + 4] * pre, s[8 * ch + 5] * pre);
-          w.w = pack_half2(s[8 * ch + 6] * pre, s[8 * ch + 7] * pre);
+          w.x = pack_half2(s[8 * ch + 0], s[8 * ch + 1]);
+          w.y = pack_half2(s[8 * ch + 2], s[8 * ch + 3]);
+          w.z = pack_half2(s[8 * ch + 4], s[8 * ch + 5]);
+          w.w = pack_half2(s[8 * ch + 6], s[8 * ch + 7]);
           *reinterpret_cast<uint4*>(dst + sw128_off(r, ch)) = w;
         }
         if (need4) {
@@ -484,26 +529,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint32_t*>(sm + L::kPSF + half * 512 + (r % 32) * 16 + (r / 32) * 4) = 0u;
         }
       } else {
-        uint32_t codes[8];
-        uint32_t sfw = 0;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float amax = 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, s[16 * g + i]);
-          const uint32_t sb = cvt_e4m3x2(amax * (pre / 6.0f), 0.f) & 0xFFu;
-          const float sc = e4m3_to_f32(sb);
-          const float rinv = sc > 0.f ? __fdividef(pre, sc) : 0.f;
-          uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-          for (int i = 0; i < 8; i += 2) w0 |= cvt_e2m1x2(s[16 * g + i] * rinv, s[16 * g + i + 1] * rinv) << (i * 4);
-#pragma unroll
-          for (int i = 0; i < 8; i += 2)
-            w1 |= cvt_e2m1x2(s[16 * g + 8 + i] * rinv, s[16 * g + 9 + i] * rinv) << (i * 4);
-          codes[2 * g] = w0;
-          codes[2 * g + 1] = w1;
-          sfw |= sb << (8 * g);
-        }
         uint8_t* d4 = sm + L::kP4;
         *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half)) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
         *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + 1)) =
@@ -515,6 +540,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(dst + sw128_off(r, ch)) = make_uint4(0, 0, 0, 0);
         }
       }
+      // Rescale O (after P V of the previous tile; before P V of this one).  Rows
+      // whose maximum did not move have alpha = 1; the warp acts together.
+      if (kt > 0 && __any_sync(0xffffffffu, Mn > M)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t v[32];
+          const uint32_t col = lane_base + kColO + (D / 2) * half + 32 * cc;
+          tmem_ld32(col, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+          tmem_st32(col, v);
+        }
+        tmem_st_wait();
+      }
+      M = Mn;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&ms.bar_p_full);
@@ -527,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!softmax_bar_or(failed)) {
       tc_fence_after();
       const float lt = l + ms.red_l[half ^ 1][r];
-      const float inv = 1.0f / (lt * static_cast<float>(1 << kPLog2));
+      const float inv = 1.0f / lt;  // l and O both carry the 2^11 pre-scale
       __half* orow = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + (D / 2) * half;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {

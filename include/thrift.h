@@ -73,7 +73,7 @@ typedef enum {
 
 typedef enum { THRIFT_Q = 0, THRIFT_K = 1, THRIFT_V = 2 } thrift_operand;
 
-/* Problem shape.  sm_scale multiplies Q K^T (usually 1/sqrt(D)); causal = 1
+/* Problem shape.  sm_scale > 0 multiplies Q K^T (usually 1/sqrt(D)); causal = 1
  * masks key > query.  blk is the selection block (square, blk x blk). */
 typedef struct {
   int B, Hq, Hkv, N, D, blk, causal;

@@ -34,7 +34,7 @@ def _c(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(), 0),
     (dict(B=0), 1), (dict(N=-64), 1), (dict(Hq=3, Hkv=2), 1), (dict(causal=2), 1),
-    (dict(sm_scale=float("nan")), 1),
+    (dict(sm_scale=float("nan")), 1), (dict(sm_scale=0.0), 1), (dict(sm_scale=-0.1), 1),
     (dict(D=96), 2), (dict(blk=32), 2), (dict(N=200), 2), (dict(N=64, blk=128), 2), (dict(N=262144), 2),
 ])
 def test_shape_validation(kw, status):
