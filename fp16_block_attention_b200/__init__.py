@@ -73,6 +73,7 @@ def _load():
         "thrift_quantize_nvfp4": ([vp, st, psh, vp, vp, vp], st),
         "thrift_select_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_select_blocks_static": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
@@ -90,7 +91,7 @@ _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
-           "thrift_attention", "thrift_fused_workspace_bytes",
+           "thrift_select_blocks_static", "thrift_attention", "thrift_fused_workspace_bytes",
            "thrift_attention_fused", "thrift_last_device_error", "thrift_strerror")
 
 
@@ -167,6 +168,25 @@ def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, 
     _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
                                                              float(rho), _ptr(mask), _ptr(ws), ws.numel(),
                                                              _stream(stream)))
+    return mask
+
+
+SELECT_STATIC_BYTES = 16 << 20
+
+
+def select_blocks_static(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, mask=None, stream=None):
+    """Selection mask without a workspace argument: for callers that cannot
+    allocate device memory (their GPU memory belongs to another allocator, or
+    they are hooks with no way to allocate).  Runs on the library's static
+    16 MiB scratch per device; larger selection workspaces are rejected.  Calls
+    that overlap on the GPU race on the shared scratch.  (This binding still
+    lets torch allocate the mask when none is given.)"""
+    _dev(Qt, "Q", torch.float16)
+    _dev(Kt, "K", torch.float16)
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_select_blocks_static", _lib.thrift_select_blocks_static(
+        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), _ptr(mask), _stream(stream)))
     return mask
 
 

@@ -147,6 +147,16 @@ thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_sh
   return from_cuda(launch_select(Q, K, *shape, rho, mask, ws, static_cast<cudaStream_t>(stream)));
 }
 
+thrift_status thrift_select_blocks_static(const void* Q, const void* K, const thrift_shape* shape, double rho,
+                                          uint8_t* mask, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!Q || !K || !mask || !(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return THRIFT_ERR_INVALID_ARG;
+  if (select_workspace_bytes(*shape) > kSelectStaticBytes) return THRIFT_ERR_WORKSPACE;
+  return from_cuda(launch_select_static(Q, K, *shape, rho, mask, static_cast<cudaStream_t>(stream)));
+}
+
 thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
                                const thrift_shape* shape, void* O, void* stream) {

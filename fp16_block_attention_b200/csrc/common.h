@@ -37,6 +37,10 @@ cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* c
 cudaError_t launch_quantize_v(const void* v, size_t bh, int N, int D, void* codes, void* scales, cudaStream_t st);
 
 size_t select_workspace_bytes(const thrift_shape& s);
+// Size of the library's static selection scratch (thrift_select_blocks_static).
+constexpr size_t kSelectStaticBytes = size_t(16) << 20;
+cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask,
+                                 cudaStream_t st);
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st);
 

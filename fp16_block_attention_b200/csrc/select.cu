@@ -196,4 +196,47 @@ cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, d
   return cudaGetLastError();
 }
 
+// ---- selection without a caller-supplied workspace ------------------------
+// Some callers cannot allocate device memory: their GPU memory belongs to
+// another allocator (a framework's caching pool, a serving runtime that
+// reserves the device at start-up), or they are hooks that the host program
+// calls without any way to allocate.  For them the selection can run on a
+// scratch array that lives in the library's own static device memory.  Every
+// device that loads the library holds this array until the process exits.
+// All calls share it and it keeps the last call's contents; the selection
+// kernels overwrite everything they read (block means, then the scores of
+// every valid pair), so nothing needs clearing between calls.  Calls whose
+// kernels overlap on the GPU (for example on two streams) race on it.
+namespace {
+__device__ __align__(256) unsigned char g_select_scratch[kSelectStaticBytes];
+constexpr int kMaxScratchDevices = 64;
+void* g_select_scratch_ptr[kMaxScratchDevices] = {nullptr};
+}  // namespace
+
+// Host code must not pass `g_select_scratch` itself to a kernel: on the host
+// that name is only a stand-in for the device array.  Its device address is
+// looked up once per device, with that device current, on the first call.
+cudaError_t select_static_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  if (!g_select_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    g_select_scratch_ptr[dev] = p;
+  }
+  *ptr = g_select_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask,
+                                 cudaStream_t st) {
+  void* scratch = nullptr;
+  cudaError_t e = select_static_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  return launch_select(Q, K, s, rho, mask, scratch, st);
+}
+
 }  // namespace thrift

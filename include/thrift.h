@@ -116,6 +116,30 @@ THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape
 THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
                                    uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
 
+/* thrift_select_blocks without a caller-supplied workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- their GPU memory is owned by another allocator (a
+ * framework's caching pool, a serving runtime that reserves the device at
+ * start-up), or they are hooks called by a host program that gives them no
+ * way to allocate.  It computes exactly what thrift_select_blocks computes,
+ * with the same kernels, on a scratch array held in the library's own static
+ * device memory:
+ *   - the array is THRIFT_SELECT_STATIC_BYTES (16 MiB) per device, held by
+ *     every GPU that loads the library until the process exits; shapes whose
+ *     selection workspace (thrift_select_workspace_bytes) exceeds it return
+ *     THRIFT_ERR_WORKSPACE;
+ *   - it allocates nothing (no cudaMalloc, no cudaFree);
+ *   - the first call on a device looks up the array's device address with
+ *     that device current (a one-time set-up); make that first call before
+ *     any stream capture;
+ *   - every call shares the array and it keeps the last call's contents
+ *     (nothing needs clearing: the kernels overwrite all they read); calls
+ *     whose kernels overlap on the GPU, e.g. on two streams, race on it.
+ * Arguments and the mask output are as for thrift_select_blocks. */
+#define THRIFT_SELECT_STATIC_BYTES ((size_t)16 << 20)
+THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* K, const thrift_shape* shape,
+                                                     double rho, uint8_t* mask, void* stream);
+
 /* Stage 2 ("the selected blocks are computed in FP16 and the remaining blocks
  * in FP4, with both paths merged via online softmax into a single output",
  * ThriftAttention abstract): O [B][Hq][N][D] fp16.
