@@ -16,13 +16,14 @@
 //   blocks) and O += P~ V~ accumulates both kinds into one FP32 tensor-memory
 //   accumulator; finally O = O / (l * 2^11).
 //
-// Warp roles (320 threads):
-//   warps 0-7  softmax: warp w owns rows 32*(w%4) .. +31 and keys
-//              64*(w/4) .. +63 of each tile, so every thread sees one
-//              selection block per tile.
-//   warp 8     producer: TMA / bulk copies of Q once, then K/V tiles into a
-//              ring of FP4 slots and a ring of FP16 slots.
-//   warp 9     MMA issuer (lane 0) and tensor-memory owner.
+// Warp roles (576 threads):
+//   warps 0-15 softmax: warp w owns rows 32*(w%4) .. +31 and keys
+//              32*(w/4) .. +31 of each tile (four threads per row), so every
+//              thread sees one selection block per tile and four softmax
+//              warps share each SM sub-partition.
+//   warp 16    producer: TMA / bulk copies of Q once, then K/V tiles into a
+//              ring of FP4 slots and separate fp16 K and V slots.
+//   warp 17    MMA issuer (lane 0) and tensor-memory owner.
 // The S product of tile j+1 is issued as soon as the softmax has read S of
 // tile j, so it overlaps the softmax of tile j; P V of tile j follows.
 #include <cuda_fp16.h>
@@ -34,9 +35,15 @@
 namespace thrift {
 namespace {
 
-constexpr int kSoftmaxThreads = 256;
-constexpr int kThreads = 320;
-constexpr int kNS4 = 2;  // FP4 K/V ring slots
+constexpr int kSplit = 4;                              // softmax threads per row
+constexpr int kKPT = 128 / kSplit;                     // keys of a tile per softmax thread
+constexpr int kGPT = kKPT / 16;                        // NVFP4 groups of P per softmax thread
+constexpr int kSoftmaxWarps = 4 * kSplit;
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kNS4 = 4;  // FP4 K/V ring slots (loads run up to three tiles ahead)
 
 // Tensor-memory columns (512 allocated).
 constexpr uint32_t kColS16 = 0;    // S from fp16 operands, 128 columns
@@ -72,6 +79,7 @@ struct Smem {
   static constexpr uint32_t kTx4 = kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes;
   static constexpr uint32_t kTx16 = kK16Bytes;  // K16 or V16 tile
   static constexpr uint32_t kTxQ = kQ16Bytes + kQ4Bytes + kQSFBytes;
+  static_assert(kBytes + 1024 <= 232448, "shared memory above the 227 KB per-CTA limit");
 };
 
 struct Misc {
@@ -89,10 +97,12 @@ struct Misc {
   uint64_t bar_drain;
   uint32_t tmem;
   volatile int abort;
-  float red_max[2][2][128];
-  float red_l[2][128];
+  float red_max[2][kSplit][128];
+  float red_l[kSplit][128];
   uint8_t cls[1024];  // per key tile: bit (a*2 + c) = FP16 flag of block (query half a, key half c)
 };
+
+static_assert(sizeof(Misc) <= 8192, "barriers and exchange buffers must fit their shared-memory slice");
 
 struct Params {
   const uint8_t* mask;
@@ -125,20 +135,22 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   return false;
 }
 
-// Named barrier of the 256 softmax threads that also ORs a per-thread flag,
+// Named barrier of the softmax threads that also ORs a per-thread flag,
 // so that every softmax thread takes the same exit decision.
+template <int NT = kSoftmaxThreads>
 __device__ __forceinline__ bool softmax_bar_or(bool flag) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(flag))
+      : "r"(static_cast<uint32_t>(flag)), "n"(NT)
       : "memory");
   return r != 0;
 }
+
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -174,9 +186,6 @@ __device__ __forceinline__ float sum16(const float* v) {
   return (t[0] + t[2]) + (t[1] + t[3]);
 }
 
-__device__ __forceinline__ float sum64(const float* v) {
-  return (sum16(v) + sum16(v + 16)) + (sum16(v + 32) + sum16(v + 48));
-}
 
 // 2^e for an integer-valued e <= 0 (0 below the normal range).
 __device__ __forceinline__ float exp2_int(float e) {
@@ -211,11 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nb = p.N / p.blk;
 
   // ---- set-up --------------------------------------------------------------
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&ms.tmem, 512);
     tmem_relinquish();
   }
-  if (tid == 256) {
+  if (tid == kProducerWarp * 32) {
     mbar_init(&ms.bar_q, 1);
     for (int i = 0; i < kNS4; ++i) {
       mbar_init(&ms.bar_full4[i], 1);
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tm = ms.tmem;
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ======================== producer ========================
     if (lane == 0) {
       prefetch_tensormap(&mQ16);
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u16 > 0) mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, kWaitNs);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ======================== MMA issuer ========================
     if (lane == 0) {
       const uint32_t q16 = sbase + L::kQ16, q4 = sbase + L::kQ4;
@@ -417,52 +426,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================== softmax ========================
-    const int quad = warp % 4, half = warp / 4;
-    const int r = quad * 32 + lane;       // row in the tile (tensor-memory lane)
-    const int qrow = qt * 128 + r;        // query index
-    const int a = r / 64;                 // query half (selection block for blk = 64)
+    // Warp w owns rows 32*(w%4) .. +31 (its tensor-memory lane quarter) and keys
+    // kKPT*(w/4) .. +kKPT-1 of every tile: one selection block per thread.
+    constexpr int kOC = D / kSplit;        // O columns of this thread
+    const int quad = warp % 4, part = warp / 4;
+    const int r = quad * 32 + lane;        // row in the tile (tensor-memory lane)
+    const int qrow = qt * 128 + r;         // query index
+    const int a = r / 64;                  // query half (selection block for blk = 64)
+    const int koff = part * kKPT;          // first key of this thread in a tile
+    const int kh = koff / 64;              // key half (selection block for blk = 64)
     const uint32_t lane_base = tm + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t ocol = lane_base + kColO + part * kOC;
     float M = -INFINITY, l = 0.f;
     bool failed = false;  // this thread gave up a wait; the exit is taken jointly
     for (int kt = 0; kt < n_kt; ++kt) {
       const uint32_t c = ms.cls[kt];
-      const bool fp16 = (c >> (a * 2 + half)) & 1u;
+      const bool fp16 = (c >> (a * 2 + kh)) & 1u;
       const bool need16 = c != 0u, need4 = c != 0xFu;
       if (!failed) failed = !wait_or_abort(&ms.bar_s_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       tc_fence_after();
-      float s[64];
+      float s[kKPT];
       if (!failed) {
-        uint32_t v[64];
-        const uint32_t col = lane_base + (fp16 ? kColS16 : kColS4) + 64 * half;
-        tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(col + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        uint32_t v[kKPT];
+        const uint32_t col = lane_base + (fp16 ? kColS16 : kColS4) + koff;
+#pragma unroll
+        for (int q = 0; q < kKPT / 32; ++q) tmem_ld32(col + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(v[j]);
+        for (int j = 0; j < kKPT; ++j) s[j] = __uint_as_float(v[j]);
         tc_fence_before();
         mbar_arrive(&ms.bar_s_free);
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s[j] = -INFINITY;
+        for (int j = 0; j < kKPT; ++j) s[j] = -INFINITY;
       }
 
       // Mask keys past N and, on the diagonal tile, keys after the query.
-      const int key0 = kt * 128 + 64 * half;
+      const int key0 = kt * 128 + koff;
       if (kt * 128 + 128 > p.N || (p.causal && kt == qt)) {
         const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys < lim are valid
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
+        for (int j = 0; j < kKPT; ++j)
           if (key0 + j >= lim) s[j] = -INFINITY;
       }
       // Group maxima of the raw scores (sm_scale > 0, so the order is that of t).
-      float gm[4];
+      float gm[kGPT];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) gm[g] = max16(&s[16 * g]);
-      float smax = fmax3(fmaxf(gm[0], gm[1]), gm[2], gm[3]);
-      ms.red_max[kt & 1][half][r] = smax;
+      for (int g = 0; g < kGPT; ++g) gm[g] = max16(&s[16 * g]);
+      float smax = gm[0];
+#pragma unroll
+      for (int g = 1; g < kGPT; ++g) smax = fmaxf(smax, gm[g]);
+      ms.red_max[kt & 1][part][r] = smax;
       if (softmax_bar_or(failed)) break;
-      smax = fmaxf(smax, ms.red_max[kt & 1][half ^ 1][r]);
+#pragma unroll
+      for (int o = 0; o < kSplit; ++o) smax = fmaxf(smax, ms.red_max[kt & 1][o][r]);
       // t = fl32(S * sm_scale * log2 e) is monotone in S: the row maximum of t is
       // fl32(max S * c).
       const float c2 = p.scale_log2;
@@ -472,17 +490,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float base = static_cast<float>(kPLog2) - Mx;  // exponent offset of P * 2^11
 
       // P * 2^11 = 2^(S*c + 11 - M); NVFP4 groups fold 1/scale into the exponent.
-      float rs;
-      uint32_t codes[8];
+      float rs = 0.f;
+      uint32_t codes[2 * kGPT];
       uint32_t sfw = 0;
       if (fp16) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) s[j] = ex2(fmaf(s[j], c2, base));
-        rs = sum64(s);
-      } else {
-        rs = 0.f;
+        for (int j = 0; j < kKPT; ++j) s[j] = ex2(fmaf(s[j], c2, base));
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < kGPT; ++g) rs += sum16(&s[16 * g]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < kGPT; ++g) {
           const float amax = ex2(fmaf(gm[g], c2, base));                      // max of P * 2^11
           const uint32_t sb = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;  // E4M3(amax / 6)
           const float sc = e4m3_to_f32(sb);
@@ -511,47 +529,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // write the encoded P for the P V product (P * 2^11)
+      uint8_t* p16 = sm + L::kP16 + kh * 16384;
+      uint8_t* p4 = sm + L::kP4;
+      uint8_t* psf = sm + L::kPSF + kh * 512 + (r % 32) * 16 + (r / 32) * 4 + (koff % 64) / 16;
+      const int ch16 = (koff % 64) / 8;  // first 16-byte chunk of this thread in the fp16 row
+      const int ch4 = koff / 32;         // first 16-byte chunk of this thread in the NVFP4 row
+      static_assert(kGPT == 2 || kGPT == 4, "scale bytes are stored as one 16- or 32-bit word");
       if (fp16) {
-        uint8_t* dst = sm + L::kP16 + half * 16384;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < kKPT / 8; ++ch) {
           uint4 w;
           w.x = pack_half2(s[8 * ch + 0], s[8 * ch + 1]);
           w.y = pack_half2(s[8 * ch + 2], s[8 * ch + 3]);
           w.z = pack_half2(s[8 * ch + 4], s[8 * ch + 5]);
           w.w = pack_half2(s[8 * ch + 6], s[8 * ch + 7]);
-          *reinterpret_cast<uint4*>(dst + sw128_off(r, ch)) = w;
+          *reinterpret_cast<uint4*>(p16 + sw128_off(r, ch16 + ch)) = w;
         }
         if (need4) {
-          uint8_t* d4 = sm + L::kP4;
-          *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half)) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + 1)) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint32_t*>(sm + L::kPSF + half * 512 + (r % 32) * 16 + (r / 32) * 4) = 0u;
+#pragma unroll
+          for (int q = 0; q < kKPT / 32; ++q)
+            *reinterpret_cast<uint4*>(p4 + sw64_off(r, ch4 + q)) = make_uint4(0, 0, 0, 0);
+          if (kGPT == 2) *reinterpret_cast<uint16_t*>(psf) = 0;
+          else *reinterpret_cast<uint32_t*>(psf) = 0u;
         }
       } else {
-        uint8_t* d4 = sm + L::kP4;
-        *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half)) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + 1)) =
-            make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        *reinterpret_cast<uint32_t*>(sm + L::kPSF + half * 512 + (r % 32) * 16 + (r / 32) * 4) = sfw;
-        if (need16) {
-          uint8_t* dst = sm + L::kP16 + half * 16384;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(dst + sw128_off(r, ch)) = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < kKPT / 32; ++q)
+          *reinterpret_cast<uint4*>(p4 + sw64_off(r, ch4 + q)) =
+              make_uint4(codes[4 * q], codes[4 * q + 1], codes[4 * q + 2], codes[4 * q + 3]);
+        if (kGPT == 2) *reinterpret_cast<uint16_t*>(psf) = static_cast<uint16_t>(sfw);
+        else *reinterpret_cast<uint32_t*>(psf) = sfw;
+        if (need16) {
+#pragma unroll
+          for (int ch = 0; ch < kKPT / 8; ++ch)
+            *reinterpret_cast<uint4*>(p16 + sw128_off(r, ch16 + ch)) = make_uint4(0, 0, 0, 0);
         }
       }
       // Rescale O (after P V of the previous tile; before P V of this one).  Rows
       // whose maximum did not move have alpha = 1; the warp acts together.
       if (kt > 0 && __any_sync(0xffffffffu, Mn > M)) {
+        if constexpr (kOC % 32 == 0) {
 #pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
-          uint32_t v[32];
-          const uint32_t col = lane_base + kColO + (D / 2) * half + 32 * cc;
-          tmem_ld32(col, v);
+          for (int cc = 0; cc < kOC / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(ocol + 32 * cc, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+            tmem_st32(ocol + 32 * cc, v);
+          }
+        } else {
+          uint32_t v[16];
+          tmem_ld16(ocol, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-          tmem_st32(col, v);
+          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+          tmem_st16(ocol, v);
         }
         tmem_st_wait();
       }
@@ -561,30 +594,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ms.bar_p_full);
     }
 
-    // ---- epilogue: O / (l * 2^11) -> fp16 ----
+    // ---- epilogue: O / l -> fp16 (both carry the 2^11 pre-scale) ----
     if (!failed) failed = !wait_or_abort(&ms.bar_o_done, (n_kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
     failed = __any_sync(0xffffffffu, failed);
-    ms.red_l[half][r] = l;
+    ms.red_l[part][r] = l;
     if (!softmax_bar_or(failed)) {
       tc_fence_after();
-      const float lt = l + ms.red_l[half ^ 1][r];
-      const float inv = 1.0f / lt;  // l and O both carry the 2^11 pre-scale
-      __half* orow = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + (D / 2) * half;
+      float lt = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + kColO + (D / 2) * half + 32 * cc, v);
-        tmem_ld_wait();
-        if (qrow < p.N) {
+      for (int o = 0; o < kSplit; ++o) lt += ms.red_l[o][r];
+      const float inv = 1.0f / lt;
+      __half* orow = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + part * kOC;
+      uint32_t v[kOC];
+      if constexpr (kOC % 32 == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 w;
-            w.x = pack_half2(__uint_as_float(v[j + 0]) * inv, __uint_as_float(v[j + 1]) * inv);
-            w.y = pack_half2(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-            w.z = pack_half2(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
-            w.w = pack_half2(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * cc + j) = w;
-          }
+        for (int cc = 0; cc < kOC / 32; ++cc) tmem_ld32(ocol + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * cc]));
+      } else {
+        tmem_ld16(ocol, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+      }
+      tmem_ld_wait();
+      if (qrow < p.N) {
+#pragma unroll
+        for (int j = 0; j < kOC; j += 8) {
+          uint4 w;
+          w.x = pack_half2(__uint_as_float(v[j + 0]) * inv, __uint_as_float(v[j + 1]) * inv);
+          w.y = pack_half2(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+          w.z = pack_half2(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
+          w.w = pack_half2(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + j) = w;
         }
       }
     }
@@ -592,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tm, 512);
   }
@@ -628,11 +665,11 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.causal = s.causal;
   prm.NT = num_tiles(s.N);
   prm.scale_log2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
+  const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   const size_t smem = Smem<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(thrift_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   thrift_attention_kernel<D><<<grid, kThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
   return cudaGetLastError();
 }

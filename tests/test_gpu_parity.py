@@ -26,6 +26,7 @@ SMALL = [
     synth.BATCHED_GQA_N16K.with_(N=384, B=2, Hq=4, Hkv=2, blk=64),          # batched, seed per batch
     synth.TINY_NONCAUSAL_D64.with_(N=192, causal=True, n_heavy=2),          # D 64 causal, ragged
     synth.CAUSAL_MH_N8K.with_(N=64, Hq=1, Hkv=1),                           # a single 64-row tile
+    synth.TINY_NONCAUSAL_D64.with_(N=384, blk=128, Hq=2, Hkv=1),            # D 64, blk 128, non-causal
 ]
 IDS = [f"{w.name}-N{w.N}-B{w.B}-H{w.Hq}x{w.Hkv}-blk{w.blk}-c{int(w.causal)}" for w in SMALL]
 
