@@ -28,12 +28,14 @@
 // tile j, so it overlaps the softmax of tile j; P V of tile j follows.
 #include <cuda_fp16.h>
 
+#include "attention_common.cuh"
 #include "common.h"
 #include "ptx.cuh"
 #include "tmap.h"
 
 namespace thrift {
 namespace {
+using namespace attn;
 
 constexpr int kSplit = 4;                              // softmax threads per row
 constexpr int kKPT = 128 / kSplit;                     // keys of a tile per softmax thread
@@ -103,100 +105,6 @@ struct Misc {
 };
 
 static_assert(sizeof(Misc) <= 8192, "barriers and exchange buffers must fit their shared-memory slice");
-
-struct Params {
-  const uint8_t* mask;
-  const uint8_t* qs;
-  const uint8_t* ks;
-  const uint8_t* vs;
-  __half* O;
-  uint32_t* err;
-  int B, Hq, Hkv, N, blk, causal, NT;
-  float scale_log2;
-};
-
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
-                                              uint32_t code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0; i < (1u << 30); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 63u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) {
-        record_error(err, code);
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-  record_error(err, code);
-  *abort = 1;
-  return false;
-}
-
-// Named barrier of the softmax threads that also ORs a per-thread flag,
-// so that every softmax thread takes the same exit decision.
-template <int NT = kSoftmaxThreads>
-__device__ __forceinline__ bool softmax_bar_or(bool flag) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(flag)), "n"(NT)
-      : "memory");
-  return r != 0;
-}
-
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ float lg2(float x) {
-  float y;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-__device__ __forceinline__ float max16(const float* v) {
-  const float a = fmax3(v[0], v[1], v[2]), b = fmax3(v[3], v[4], v[5]), c = fmax3(v[6], v[7], v[8]);
-  const float d = fmax3(v[9], v[10], v[11]), e = fmax3(v[12], v[13], v[14]);
-  return fmaxf(fmax3(a, b, c), fmax3(d, e, v[15]));
-}
-
-// Pairwise (tree) sums: short dependency chains.
-__device__ __forceinline__ float sum16(const float* v) {
-  float t[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = v[i] + v[i + 8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) t[i] += t[i + 4];
-  return (t[0] + t[2]) + (t[1] + t[3]);
-}
-
-
-// 2^e for an integer-valued e <= 0 (0 below the normal range).
-__device__ __forceinline__ float exp2_int(float e) {
-  const int i = static_cast<int>(e);
-  return (i < -126) ? 0.f : __int_as_float((127 + i) << 23);
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -478,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int g = 1; g < kGPT; ++g) smax = fmaxf(smax, gm[g]);
       ms.red_max[kt & 1][part][r] = smax;
-      if (softmax_bar_or(failed)) break;
+      if (softmax_bar_or<kSoftmaxThreads>(failed)) break;
 #pragma unroll
       for (int o = 0; o < kSplit; ++o) smax = fmaxf(smax, ms.red_max[kt & 1][o][r]);
       // t = fl32(S * sm_scale * log2 e) is monotone in S: the row maximum of t is
@@ -598,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!failed) failed = !wait_or_abort(&ms.bar_o_done, (n_kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
     failed = __any_sync(0xffffffffu, failed);
     ms.red_l[part][r] = l;
-    if (!softmax_bar_or(failed)) {
+    if (!softmax_bar_or<kSoftmaxThreads>(failed)) {
       tc_fence_after();
       float lt = 0.f;
 #pragma unroll
@@ -665,6 +573,7 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.causal = s.causal;
   prm.NT = num_tiles(s.N);
   prm.scale_log2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
+  if (s.blk == 128) return launch_attention_pp<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
   const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   const size_t smem = Smem<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(thrift_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

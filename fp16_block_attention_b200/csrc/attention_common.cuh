@@ -1,0 +1,117 @@
+// Device helpers shared by the attention kernels: launch parameters, bounded
+// mbarrier waits that raise a CTA-wide abort flag, the softmax threads' joint
+// barrier, and small arithmetic helpers (ex2 / lg2 on the MUFU, three-input
+// max, tree sums, fp16 packing).
+#pragma once
+#include <cuda_fp16.h>
+
+#include "common.h"
+#include "ptx.cuh"
+
+namespace thrift {
+namespace attn {
+
+struct Params {
+  const uint8_t* mask;
+  const uint8_t* qs;
+  const uint8_t* ks;
+  const uint8_t* vs;
+  __half* O;
+  uint32_t* err;
+  int B, Hq, Hkv, N, blk, causal, NT;
+  float scale_log2;
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
+                                              uint32_t code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) {
+        record_error(err, code);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  record_error(err, code);
+  *abort = 1;
+  return false;
+}
+
+// Named barrier of the softmax threads that also ORs a per-thread flag,
+// so that every softmax thread takes the same exit decision.
+template <int NT>
+__device__ __forceinline__ bool softmax_bar_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(flag)), "n"(NT)
+      : "memory");
+  return r != 0;
+}
+
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float max16(const float* v) {
+  const float a = fmax3(v[0], v[1], v[2]), b = fmax3(v[3], v[4], v[5]), c = fmax3(v[6], v[7], v[8]);
+  const float d = fmax3(v[9], v[10], v[11]), e = fmax3(v[12], v[13], v[14]);
+  return fmaxf(fmax3(a, b, c), fmax3(d, e, v[15]));
+}
+
+// Pairwise (tree) sums: short dependency chains.
+__device__ __forceinline__ float sum16(const float* v) {
+  float t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = v[i] + v[i + 8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t[i] += t[i + 4];
+  return (t[0] + t[2]) + (t[1] + t[3]);
+}
+
+
+// 2^e for an integer-valued e <= 0 (0 below the normal range).
+__device__ __forceinline__ float exp2_int(float e) {
+  const int i = static_cast<int>(e);
+  return (i < -126) ? 0.f : __int_as_float((127 + i) << 23);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+
+}  // namespace attn
+
+// Ping-pong kernel for 128 x 128 selection blocks (attention_pp.cu).
+template <int D>
+cudaError_t launch_attention_pp(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
+                                const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                                const attn::Params& prm, cudaStream_t st);
+
+}  // namespace thrift
