@@ -16,11 +16,14 @@
 //   (.kind::mxf4nvf4), t = S * sm_scale * log2 e, integer running maximum
 //   M = ceil(max t) (rescales of O are exact powers of two), P * 2^11 encoded
 //   as fp16 (written to tensor memory, the A operand of a .kind::f16 product)
-//   or as NVFP4 per 16 keys (shared memory, scales via tcgen05.cp), and
-//   O += P~ V~; finally O / l.
+//   or as NVFP4 per 16 keys (codes in shared memory, scales stored by each
+//   row's thread straight into tensor memory), and O += P~ V~; finally O / l.
 //
-// Warp roles (320 threads): warps 0-3 softmax of tile A, 4-7 softmax of tile
-// B, 8 TMA producer, 9 MMA issuer and tensor-memory owner.
+// Warp roles (352 threads): warps 0-3 softmax of tile A, 4-7 softmax of tile
+// B, 8 TMA producer, 9 issues the S products (and owns tensor memory), 10
+// issues the P V products.  Two issuing threads on different SM
+// sub-partitions keep the S of one tile from queueing behind the P V of the
+// other; they meet only through mbarriers.
 #include <cuda_fp16.h>
 
 #include "attention_common.cuh"
@@ -32,9 +35,10 @@ namespace thrift {
 namespace {
 using namespace attn;
 
-constexpr int kPPThreads = 320;
+constexpr int kPPThreads = 352;
 constexpr int kPPProducer = 8;
-constexpr int kPPMma = 9;
+constexpr int kPPMmaS = 9;   // issues the S products; owns tensor memory
+constexpr int kPPMmaPV = 10;  // issues the P V products
 
 // Tensor-memory columns (512 allocated).
 constexpr uint32_t kPColS = 0;       // shared S buffer, 128 columns
@@ -43,7 +47,7 @@ constexpr uint32_t kPColP16 = 384;   // fp16 P of either tile, 64 columns (used 
 constexpr uint32_t kPColSFQ = 448;   // Q4 scales, 8 columns per tile
 constexpr uint32_t kPColSFK = 464;   // K4 scales of the current key tile
 constexpr uint32_t kPColSFV = 472;   // V4 scales of the key tile being multiplied
-constexpr uint32_t kPColSFP = 480;   // P4 scales, 8 columns per tile
+constexpr uint32_t kPColSFP = 480;   // P4 scales, 8 columns per tile: chunk c of row r at 4c + r / 32
 
 template <int D>
 struct SmemPP {
@@ -54,13 +58,12 @@ struct SmemPP {
   static constexpr uint32_t kQSFBytes = (D / 64) * 512;
   static constexpr uint32_t kQSF = kQ4 + 2 * kQ4Bytes;
   static constexpr uint32_t kP4 = (kQSF + 2 * kQSFBytes + 1023) / 1024 * 1024;  // 8 KB per tile
-  static constexpr uint32_t kPSF = kP4 + 2 * 8192;                              // 1 KB per tile
   static constexpr uint32_t kK4Bytes = 128 * D / 2;
   static constexpr uint32_t kV4Bytes = D * 64;
   static constexpr uint32_t kKSFBytes = (D / 64) * 512;
   static constexpr uint32_t kVSFBytes = 1024;
   static constexpr uint32_t kSlot4Bytes = (kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes + 1023) / 1024 * 1024;
-  static constexpr uint32_t kSlot4 = kPSF + 2048;
+  static constexpr uint32_t kSlot4 = kP4 + 2 * 8192;
   static constexpr int kNS = (D == 128) ? 3 : 4;  // NVFP4 K/V ring slots
   static constexpr uint32_t kK16Bytes = 128 * D * 2;
   static constexpr uint32_t kSlot16 = kSlot4 + kNS * kSlot4Bytes;  // K16 then V16
@@ -81,7 +84,7 @@ struct MiscPP {
   uint64_t bar_p_full[2];  // per tile: P of the tile's current key tile written
   uint64_t bar_o_done[2];  // per tile: one phase per P V product of that tile
   uint64_t bar_p16_free;   // one phase per fp16 P V product, in issue order
-  uint64_t bar_drain;
+  uint64_t bar_drain[2];   // one per issuing thread
   uint32_t tmem;
   volatile int abort;
   uint8_t cls[2][1024];  // per tile and key tile: 1 = FP16, 0 = NVFP4
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const int nmax = n0 > n1 ? n0 : n1;
   const int nb = p.NT;  // blk = 128
 
-  if (warp == kPPMma) {
+  if (warp == kPPMmaS) {
     tmem_alloc(&ms.tmem, 512);
     tmem_relinquish();
   }
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     mbar_init(&ms.bar_q, 1);
     for (int i = 0; i < L::kNS; ++i) {
       mbar_init(&ms.bar_full4[i], 1);
-      mbar_init(&ms.bar_empty4[i], 1);
+      mbar_init(&ms.bar_empty4[i], 2);  // K4 read by the S issuer, V4 by the P V issuer
     }
     mbar_init(&ms.bar_full_k16, 1);
     mbar_init(&ms.bar_empty_k16, 1);
@@ -135,7 +138,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     mbar_init(&ms.bar_s_free, 128);
     mbar_init(&ms.bar_p16_free, 1);
-    mbar_init(&ms.bar_drain, 1);
+    mbar_init(&ms.bar_drain[0], 1);
+    mbar_init(&ms.bar_drain[1], 1);
     ms.abort = 0;
     fence_mbar_init();
   }
@@ -219,12 +223,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kPPMma) {
-    // ======================== MMA issuer ========================
+  } else if (warp == kPPMmaS) {
+    // ================= S issuer: K scales, then S of tile A and tile B =================
+    // The two tiles take turns on the S buffer; each S waits until the
+    // previous one has been loaded into registers by its warpgroup.
     if (lane == 0) {
       constexpr uint32_t sbo4 = (D == 128) ? 512u : 256u;
       constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
-      const int nt[2] = {n0, n1};
       bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
       tc_fence_after();
       if (ok)
@@ -232,17 +237,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           for (int c = 0; c < D / 64; ++c)
             tmem_cp_32x128b_x4(tm + kPColSFQ + 8 * x + 4 * c,
                                make_sdesc(sbase + L::kQSF + x * L::kQSFBytes + 512 * c, 16, 128, LAYOUT_NONE));
-      int u4 = 0, uk16 = 0, uv16 = 0, seq = 0;
-      int slot_of[2] = {0, 0};
-      uint32_t o_acc[2] = {0u, 0u};
-      for (int kt = 0; ok && kt <= nmax; ++kt) {
-        // ---- operands of key tile kt ----
-        const bool t4 = kt < nmax && need4(kt), t16 = kt < nmax && need16(kt);
+      int u4 = 0, uk16 = 0, seq = 0;
+      for (int kt = 0; ok && kt < nmax; ++kt) {
+        const bool t4 = need4(kt), t16 = need16(kt);
+        int slot = 0;
         if (t4) {
-          const int slot = u4 % L::kNS, use = u4 / L::kNS;
-          if (!(ok = wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          slot = u4 % L::kNS;
+          if (!(ok = wait_or_abort(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++u4;
-          slot_of[kt & 1] = slot;
           tc_fence_after();
           const uint32_t ksf = sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK4Bytes + L::kV4Bytes;
           for (int c = 0; c < D / 64; ++c)
@@ -253,17 +255,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           ++uk16;
           tc_fence_after();
         }
-        const bool p4 = kt >= 1 && need4(kt - 1), p16 = kt >= 1 && need16(kt - 1);
-        bool v16_ready = false;
-        for (int x = 0; x < 2 && ok; ++x) {
-          // ---- S of tile x, key tile kt, into the shared S buffer ----
-          if (kt < nt[x]) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (kt < (x == 0 ? n0 : n1)) {
             if (seq > 0 && !(ok = wait_or_abort(&ms.bar_s_free, (seq - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
               break;
             tc_fence_after();
             if (ms.cls[x][kt] == 0) {
               const uint32_t q4 = sbase + L::kQ4 + x * L::kQ4Bytes;
-              const uint32_t k4 = sbase + L::kSlot4 + slot_of[kt & 1] * L::kSlot4Bytes;
+              const uint32_t k4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
 #pragma unroll
               for (int c = 0; c < D / 64; ++c)
                 mma_nvf4(tm + kPColS, make_sdesc(q4 + 32 * c, 16, sbo4, sw4), make_sdesc(k4 + 32 * c, 16, sbo4, sw4),
@@ -280,26 +280,55 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             mma_commit(&ms.bar_s_full[x]);
             ++seq;
           }
-          // ---- P V of tile x, key tile kt - 1 ----
-          const int kp = kt - 1;
-          if (kp >= 0 && kp < nt[x]) {
-            if (!(ok = wait_or_abort(&ms.bar_p_full[x], kp & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        }
+        if (!ok) break;
+        // K operands of this key tile are no longer needed (V: the P V issuer)
+        if (t4) mma_commit(&ms.bar_empty4[slot]);
+        if (t16) mma_commit(&ms.bar_empty_k16);
+      }
+      // drain: every tensor-core operation this thread issued completes before exit
+      mma_commit(&ms.bar_drain[0]);
+      mbar_wait(&ms.bar_drain[0], 0, kWaitNs);
+    }
+    __syncwarp();
+  } else if (warp == kPPMmaPV) {
+    // ================= P V issuer: O_x += P_x V for tile A, then tile B =================
+    if (lane == 0) {
+      bool ok = true;
+      int u4 = 0, uv16 = 0;
+      uint32_t acc0 = 0u, acc1 = 0u;
+      for (int kt = 0; ok && kt < nmax; ++kt) {
+        const bool t4 = need4(kt), t16 = need16(kt);
+        const int slot = u4 % L::kNS, use = u4 / L::kNS;
+        if (t4) ++u4;
+        bool v4_ready = false, v16_ready = false;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (kt < (x == 0 ? n0 : n1)) {
+            if (!(ok = wait_or_abort(&ms.bar_p_full[x], kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
             tc_fence_after();
             const uint32_t dO = tm + kPColO + 128 * x;
-            if (ms.cls[x][kp] == 0) {
-              const uint32_t st = sbase + L::kSlot4 + slot_of[kp & 1] * L::kSlot4Bytes;
+            uint32_t& acc = x == 0 ? acc0 : acc1;
+            if (ms.cls[x][kt] == 0) {
+              const uint32_t st = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
               const uint32_t v4 = st + L::kK4Bytes, vsf = st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes;
-              const uint32_t p4s = sbase + L::kP4 + x * 8192, psf = sbase + L::kPSF + x * 1024;
-              for (int c = 0; c < 2; ++c) {
-                tmem_cp_32x128b_x4(tm + kPColSFP + 8 * x + 4 * c, make_sdesc(psf + 512 * c, 16, 128, LAYOUT_NONE));
-                tmem_cp_32x128b_x4(tm + kPColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
+              if (!v4_ready) {
+                // V4 landed with K4 (one barrier phase); wait on it here too so
+                // that this thread observes the copy itself.  The producer cannot
+                // refill the slot before this thread releases it.
+                if (!(ok = wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+                tc_fence_after();
+                for (int c = 0; c < 2; ++c)
+                  tmem_cp_32x128b_x4(tm + kPColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
+                v4_ready = true;
               }
+              const uint32_t p4s = sbase + L::kP4 + x * 8192;
 #pragma unroll
               for (int c = 0; c < 2; ++c) {
                 mma_nvf4(dO, make_sdesc(p4s + 32 * c, 16, 512, LAYOUT_SW64),
                          make_sdesc(v4 + 32 * c, 16, 512, LAYOUT_SW64), idesc_nvf4(128, D),
-                         tm + kPColSFP + 8 * x + 4 * c, tm + kPColSFV + 4 * c, o_acc[x]);
-                o_acc[x] = 1;
+                         tm + kPColSFP + 8 * x + 4 * c, tm + kPColSFV + 4 * c, acc);
+                acc = 1;
               }
             } else {
               if (!v16_ready) {
@@ -312,8 +341,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
                 mma_f16_ts(dO, tm + kPColP16 + 8 * k, make_sdesc(v16 + k * 2048, 16384, 1024, LAYOUT_SW128),
-                           idesc_f16(128, D, true), o_acc[x]);
-                o_acc[x] = 1;
+                           idesc_f16(128, D, true), acc);
+                acc = 1;
               }
               mma_commit(&ms.bar_p16_free);
             }
@@ -321,14 +350,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
         }
         if (!ok) break;
-        // ---- release the operands no longer needed ----
-        if (p4) mma_commit(&ms.bar_empty4[slot_of[(kt - 1) & 1]]);
-        if (p16) mma_commit(&ms.bar_empty_v16);
-        if (t16) mma_commit(&ms.bar_empty_k16);
+        if (t4) mma_commit(&ms.bar_empty4[slot]);
+        if (t16) mma_commit(&ms.bar_empty_v16);
       }
-      // drain: every tensor-core operation of this CTA completes before exit
-      mma_commit(&ms.bar_drain);
-      mbar_wait(&ms.bar_drain, 0, kWaitNs);
+      mma_commit(&ms.bar_drain[1]);
+      mbar_wait(&ms.bar_drain[1], 0, kWaitNs);
     }
     __syncwarp();
   } else {
@@ -396,17 +422,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       // P * 2^11 = 2^(S*c + 11 - M), encoded and stored 64 (fp16) or 32 (NVFP4)
       // keys at a time; NVFP4 groups fold 1/scale into the exponent.
       float rs = 0.f;
+      const float2 c2v = make_float2(c2, c2);
       if (fp16) {
+        const float2 bb = make_float2(base, base);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t w[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float p0 = ex2(fmaf(s[64 * h + 2 * j], c2, base));
-            const float p1 = ex2(fmaf(s[64 * h + 2 * j + 1], c2, base));
-            s[64 * h + 2 * j] = p0;
-            s[64 * h + 2 * j + 1] = p1;
-            w[j] = pack_half2(p0, p1);
+            const float2 pp = ex2_fma2(s[64 * h + 2 * j], s[64 * h + 2 * j + 1], c2v, bb);
+            s[64 * h + 2 * j] = pp.x;
+            s[64 * h + 2 * j + 1] = pp.y;
+            w[j] = pack_half2(pp.x, pp.y);
           }
           rs += sum16(&s[64 * h]) + sum16(&s[64 * h + 16]) + sum16(&s[64 * h + 32]) + sum16(&s[64 * h + 48]);
           tmem_st32(lane_base + kPColP16 + 32 * h, w);
@@ -425,23 +452,24 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             const float sc = e4m3_to_f32(sbyte);
             const float sce = sc > 0.f ? sc : 1.0f;  // zero scale: codes round to 0, l keeps P
             const float bias = base - lg2(sce);
+            const float2 bb = make_float2(bias, bias);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) s[16 * g + i] = ex2(fmaf(s[16 * g + i], c2, bias));
+            for (int i = 0; i < 16; i += 2) {
+              const float2 pp = ex2_fma2(s[16 * g + i], s[16 * g + i + 1], c2v, bb);
+              s[16 * g + i] = pp.x;
+              s[16 * g + i + 1] = pp.y;
+            }
             rs = fmaf(sum16(&s[16 * g]), sce, rs);
-            uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) w0 |= cvt_e2m1x2(s[16 * g + i], s[16 * g + i + 1]) << (i * 4);
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) w1 |= cvt_e2m1x2(s[16 * g + 8 + i], s[16 * g + 9 + i]) << (i * 4);
-            code[2 * gg] = w0;
-            code[2 * gg + 1] = w1;
+            code[2 * gg] = cvt_e2m1x8(&s[16 * g]);
+            code[2 * gg + 1] = cvt_e2m1x8(&s[16 * g + 8]);
             sfw[g / 4] |= sbyte << (8 * (g % 4));
           }
           *reinterpret_cast<uint4*>(d4 + sw64_off(r, c)) = make_uint4(code[0], code[1], code[2], code[3]);
         }
-        uint8_t* psf = sm + L::kPSF + x * 1024 + (r % 32) * 16 + (r / 32) * 4;
-        *reinterpret_cast<uint32_t*>(psf) = sfw[0];
-        *reinterpret_cast<uint32_t*>(psf + 512) = sfw[1];
+        // Scale factors of a 128-row A operand: the MMA reads row r's four
+        // scales of K chunk c from lane r, column base + 4c + r / 32.
+        tmem_st1(lane_base + kPColSFP + 8 * x + quad, sfw[0]);
+        tmem_st1(lane_base + kPColSFP + 8 * x + 4 + quad, sfw[1]);
       }
       l = l * alpha + rs;
       // Rescale O when the maximum grew (rows with alpha = 1 are unchanged).
@@ -451,8 +479,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           uint32_t v[32];
           tmem_ld32(ocol + 32 * cc, v);
           tmem_ld_wait();
+          const float2 aa = make_float2(alpha, alpha);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+          for (int j = 0; j < 32; j += 2) {
+            const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), aa);
+            v[j] = __float_as_uint(o.x);
+            v[j + 1] = __float_as_uint(o.y);
+          }
           tmem_st32(ocol + 32 * cc, v);
         }
       }
@@ -494,7 +527,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kPPMma) {
+  if (warp == kPPMmaS) {
     tc_fence_after();
     tmem_dealloc(tm, 512);
   }
