@@ -40,7 +40,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
 PROFILE_FILE = os.path.join(ROOT, "profiles", "attention_gqa_n32k_traffic.json")
-KERNEL_SOURCES = ["attention.cu", "attention_pp.cu", "attention_common.cuh", "ptx.cuh", "tmap.h"]
+KERNEL_SOURCES = ["attention.cu", "attention_db.cu", "attention_common.cuh", "ptx.cuh", "tmap.h"]
 LAUNCHES_PER_STEP = 8        # quantize Q, K, V; pool Q, K; scores; top-k; attention
 
 

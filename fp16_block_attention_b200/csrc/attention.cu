@@ -573,7 +573,7 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.causal = s.causal;
   prm.NT = num_tiles(s.N);
   prm.scale_log2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
-  if (s.blk == 128) return launch_attention_pp<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
+  if (s.blk == 128) return launch_attention_db<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
   const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   const size_t smem = Smem<D>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(thrift_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

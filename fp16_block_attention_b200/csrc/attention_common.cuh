@@ -59,6 +59,14 @@ __device__ __forceinline__ bool softmax_bar_or(bool flag) {
 }
 
 
+// Named barriers among a subset of the CTA's warps (count = threads taking part).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -116,9 +124,10 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 
 }  // namespace attn
 
-// Ping-pong kernel for 128 x 128 selection blocks (attention_pp.cu).
+// Kernel with double-buffered S and P for 128 x 128 selection blocks
+// (attention_db.cu).
 template <int D>
-cudaError_t launch_attention_pp(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
+cudaError_t launch_attention_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
                                 const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
                                 const attn::Params& prm, cudaStream_t st);
 

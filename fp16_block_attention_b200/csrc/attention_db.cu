@@ -1,0 +1,564 @@
+// Stage 2 of the method for 128 x 128 selection blocks ("the selected blocks
+// are computed in FP16 and the remaining blocks in FP4, with both paths merged
+// via online softmax into a single output", ThriftAttention abstract), with
+// the S products and the P operands double-buffered.
+//
+// A CTA owns one 128-row query tile of one (batch, query head).  With blk =
+// 128 each key tile is one selection block, so it is entirely FP16 or
+// entirely NVFP4.  Per key tile k:
+//   S(k) from the fp16 operands (.kind::f16) or the NVFP4 copies
+//   (.kind::mxf4nvf4) into tensor-memory buffer k % 2; t = S * sm_scale *
+//   log2 e, integer running maximum M = ceil(max t) (rescales of O are exact
+//   powers of two); P * 2^11 encoded as fp16 (tensor memory, the A operand of
+//   a .kind::f16 product) or as NVFP4 per 16 keys (codes in shared-memory
+//   buffer k % 2, scales stored by each row's thread straight into tensor
+//   memory); O += P~ V~; finally O / l.
+//
+// While the softmax threads work on key tile k, the tensor cores compute
+// S(k + 1) into the other buffer and P(k - 1) V(k - 1) from the other P
+// buffer, so neither round trip is on the softmax's path.  The softmax waits
+// for a P V product only before reusing its P buffer (two key tiles later) or
+// before rescaling O.
+//
+// Warp roles (352 threads): warps 0-7 softmax, two threads per query row
+// (warps w and w + 4 share the tensor-memory lanes of row quadrant w % 4);
+// both threads load the whole 128-key row of S and take its maximum, so each
+// reaches the same M on its own, and each exponentiates, encodes and rescales
+// its own half (keys 64h .. 64h + 63, O columns hD/2 ..).  Their partial row
+// sums meet once, in the epilogue.  Warp 8 is the TMA producer, 9 issues the
+// S products (and owns tensor memory), 10 issues the P V products.  The two
+// issuing threads and the softmax threads meet only through mbarriers.
+#include <cuda_fp16.h>
+
+#include "attention_common.cuh"
+#include "common.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+namespace thrift {
+namespace {
+using namespace attn;
+
+constexpr int kDBThreads = 352;
+constexpr int kDBSoftmax = 256;  // softmax threads (two per query row)
+constexpr int kDBProducer = 8;
+constexpr int kDBMmaS = 9;
+constexpr int kDBMmaPV = 10;
+
+// Tensor-memory columns (512 allocated).
+constexpr uint32_t kDColS = 0;      // S of key tile k in buffer k % 2 at 128 * (k % 2)
+constexpr uint32_t kDColO = 256;    // O, D columns
+constexpr uint32_t kDColP16 = 384;  // fp16 P, 64 columns
+constexpr uint32_t kDColSFQ = 448;  // Q4 scales, 4 columns per 64-wide chunk of D
+constexpr uint32_t kDColSFK = 456;  // K4 scales of the key tile being multiplied
+constexpr uint32_t kDColSFV = 464;  // V4 scales of the key tile being multiplied
+constexpr uint32_t kDColSFP = 472;  // P4 scales of P buffer b at 8 b: chunk c of row r at 4 c + r / 32
+
+template <int D>
+struct SmemDB {
+  static constexpr uint32_t kQ16Bytes = 128 * D * 2;
+  static constexpr uint32_t kQ16 = 0;
+  static constexpr uint32_t kQ4Bytes = 128 * D / 2;
+  static constexpr uint32_t kQ4 = kQ16 + kQ16Bytes;
+  static constexpr uint32_t kQSFBytes = (D / 64) * 512;
+  static constexpr uint32_t kQSF = kQ4 + kQ4Bytes;
+  static constexpr uint32_t kP4Bytes = 8192;  // 128 rows x 128 keys of E2M1, 64B-swizzled
+  static constexpr uint32_t kP4 = (kQSF + kQSFBytes + 1023) / 1024 * 1024;  // two buffers
+  static constexpr uint32_t kK4Bytes = 128 * D / 2;
+  static constexpr uint32_t kV4Bytes = D * 64;
+  static constexpr uint32_t kKSFBytes = (D / 64) * 512;
+  static constexpr uint32_t kVSFBytes = 1024;
+  static constexpr uint32_t kSlot4Bytes = (kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes + 1023) / 1024 * 1024;
+  static constexpr uint32_t kSlot4 = kP4 + 2 * kP4Bytes;
+  static constexpr int kNS = 4;  // NVFP4 K/V ring slots
+  static constexpr uint32_t kK16Bytes = 128 * D * 2;
+  static constexpr uint32_t kSlot16 = kSlot4 + kNS * kSlot4Bytes;  // K16 then V16
+  static constexpr uint32_t kMisc = kSlot16 + 2 * kK16Bytes;
+  static constexpr uint32_t kBytes = kMisc + 4096;
+  static constexpr uint32_t kTx4 = kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes;
+  static constexpr uint32_t kTx16 = kK16Bytes;
+  static constexpr uint32_t kTxQ = kQ16Bytes + kQ4Bytes + kQSFBytes;
+  static_assert(kBytes + 1024 <= 232448, "shared memory above the 227 KB per-CTA limit");
+  static_assert(kQ4 % 1024 == 0 && kSlot4 % 1024 == 0 && kSlot16 % 1024 == 0, "TMA tiles need 1 KB alignment");
+};
+
+struct MiscDB {
+  uint64_t bar_q;
+  uint64_t bar_full4[4], bar_empty4[4];
+  uint64_t bar_full_k16, bar_empty_k16, bar_full_v16, bar_empty_v16;
+  uint64_t bar_s_full[2];  // S buffer b holds a new product (one phase per use)
+  uint64_t bar_s_free[2];  // S buffer b loaded into registers by the softmax threads
+  uint64_t bar_p_full[2];  // P buffer b written by the softmax threads
+  uint64_t bar_o_done[2];  // P buffer b multiplied into O
+  uint64_t bar_drain[2];   // one per issuing thread
+  uint32_t tmem;
+  volatile int abort;
+  float lsum[2][128];  // partial row sums of the two halves, for the epilogue
+  uint8_t cls[1024];    // per key tile: 1 = FP16, 0 = NVFP4
+};
+static_assert(sizeof(MiscDB) <= 4096, "barriers must fit their shared-memory slice");
+
+template <int D>
+__global__ void __launch_bounds__(kDBThreads, 1)
+    thrift_attention_db_kernel(const __grid_constant__ CUtensorMap mQ16, const __grid_constant__ CUtensorMap mK16,
+                               const __grid_constant__ CUtensorMap mV16, const __grid_constant__ CUtensorMap mQ4,
+                               const __grid_constant__ CUtensorMap mK4, const __grid_constant__ CUtensorMap mV4,
+                               const Params p) {
+  using L = SmemDB<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  MiscDB& ms = *reinterpret_cast<MiscDB*>(sm + L::kMisc);
+  const uint32_t sbase = smem_u32(sm);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int BH = p.B * p.Hq;
+  const int qt = p.NT - 1 - static_cast<int>(blockIdx.x) / BH;  // longest causal rows first
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.Hq, hq = bh % p.Hq;
+  const int bhk = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  const int nk = p.causal ? qt + 1 : p.NT;  // key tiles this query tile attends to
+  const int nb = p.NT;                     // blk = 128
+
+  if (warp == kDBMmaS) {
+    tmem_alloc(&ms.tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == kDBProducer * 32) {
+    mbar_init(&ms.bar_q, 1);
+    for (int i = 0; i < L::kNS; ++i) {
+      mbar_init(&ms.bar_full4[i], 1);
+      mbar_init(&ms.bar_empty4[i], 2);  // K4 read by the S issuer, V4 by the P V issuer
+    }
+    mbar_init(&ms.bar_full_k16, 1);
+    mbar_init(&ms.bar_empty_k16, 1);
+    mbar_init(&ms.bar_full_v16, 1);
+    mbar_init(&ms.bar_empty_v16, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms.bar_s_full[i], 1);
+      mbar_init(&ms.bar_s_free[i], kDBSoftmax);
+      mbar_init(&ms.bar_p_full[i], kDBSoftmax);
+      mbar_init(&ms.bar_o_done[i], 1);
+      mbar_init(&ms.bar_drain[i], 1);
+    }
+    ms.abort = 0;
+    fence_mbar_init();
+  }
+  {
+    const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
+    for (int kt = tid; kt < nk; kt += kDBThreads) ms.cls[kt] = m0[kt] ? 1 : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ms.tmem;
+
+  if (warp == kDBProducer) {
+    // ======================== producer ========================
+    if (lane == 0) {
+      prefetch_tensormap(&mQ16);
+      prefetch_tensormap(&mK4);
+      prefetch_tensormap(&mV4);
+      mbar_arrive_expect_tx(&ms.bar_q, L::kTxQ);
+      for (int pnl = 0; pnl < D / 64; ++pnl)
+        tma_load_3d(sm + L::kQ16 + pnl * 16384, &mQ16, &ms.bar_q, pnl * 64, qt * 128, bh);
+      tma_load_3d(sm + L::kQ4, &mQ4, &ms.bar_q, 0, qt * 128, bh);
+      bulk_load(sm + L::kQSF, p.qs + (static_cast<size_t>(bh) * p.NT + qt) * L::kQSFBytes, L::kQSFBytes, &ms.bar_q);
+      int u4 = 0, u16 = 0;
+      for (int kt = 0; kt < nk && !ms.abort; ++kt) {
+        if (ms.cls[kt] == 0) {
+          const int slot = u4 % L::kNS, use = u4 / L::kNS;
+          if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+            break;
+          uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
+          mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx4);
+          tma_load_3d(st, &mK4, &ms.bar_full4[slot], 0, kt * 128, bhk);
+          tma_load_3d(st + L::kK4Bytes, &mV4, &ms.bar_full4[slot], kt * 64, 0, bhk);
+          bulk_load(st + L::kK4Bytes + L::kV4Bytes, p.ks + (static_cast<size_t>(bhk) * p.NT + kt) * L::kKSFBytes,
+                    L::kKSFBytes, &ms.bar_full4[slot]);
+          bulk_load(st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes,
+                    p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * kt) * 512, L::kVSFBytes, &ms.bar_full4[slot]);
+          ++u4;
+        } else {
+          uint8_t* st = sm + L::kSlot16;
+          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+            break;
+          mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
+          for (int pnl = 0; pnl < D / 64; ++pnl)
+            tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
+          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
+            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K16 copy of this tile is in flight
+            break;
+          }
+          mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
+          for (int pnl = 0; pnl < D / 64; ++pnl)
+            tma_load_3d(st + L::kK16Bytes + pnl * 16384, &mV16, &ms.bar_full_v16, pnl * 64, kt * 128, bhk);
+          ++u16;
+        }
+      }
+      // Let every copy this thread issued land before the CTA can exit.
+      mbar_wait(&ms.bar_q, 0, kWaitNs);
+      for (int s = 0; s < L::kNS; ++s)
+        if (u4 > s) mbar_wait(&ms.bar_full4[s], ((u4 - 1 - s) / L::kNS) & 1, kWaitNs);
+      if (u16 > 0) {
+        mbar_wait(&ms.bar_full_k16, (u16 - 1) & 1, kWaitNs);
+        mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, kWaitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kDBMmaS) {
+    // ================= S issuer: K scales, then S(k) into buffer k % 2 =================
+    if (lane == 0) {
+      constexpr uint32_t sbo4 = (D == 128) ? 512u : 256u;
+      constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
+      bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
+      tc_fence_after();
+      if (ok)
+        for (int c = 0; c < D / 64; ++c)
+          tmem_cp_32x128b_x4(tm + kDColSFQ + 4 * c, make_sdesc(sbase + L::kQSF + 512 * c, 16, 128, LAYOUT_NONE));
+      int u4 = 0, uk16 = 0;
+      for (int kt = 0; ok && kt < nk; ++kt) {
+        const int bb = kt & 1;
+        const bool fp16 = ms.cls[kt] != 0;
+        int slot = 0;
+        if (!fp16) {
+          slot = u4 % L::kNS;
+          if (!(ok = wait_or_abort(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          ++u4;
+          tc_fence_after();
+          const uint32_t ksf = sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK4Bytes + L::kV4Bytes;
+          for (int c = 0; c < D / 64; ++c)
+            tmem_cp_32x128b_x4(tm + kDColSFK + 4 * c, make_sdesc(ksf + 512 * c, 16, 128, LAYOUT_NONE));
+        } else {
+          if (!(ok = wait_or_abort(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          ++uk16;
+          tc_fence_after();
+        }
+        // buffer bb was last used by S(kt - 2): wait until its threads loaded it
+        if (kt >= 2) {
+          if (!(ok = wait_or_abort(&ms.bar_s_free[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
+            break;
+          tc_fence_after();
+        }
+        const uint32_t dS = tm + kDColS + 128 * bb;
+        if (!fp16) {
+          const uint32_t q4 = sbase + L::kQ4;
+          const uint32_t k4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            mma_nvf4(dS, make_sdesc(q4 + 32 * c, 16, sbo4, sw4), make_sdesc(k4 + 32 * c, 16, sbo4, sw4),
+                     idesc_nvf4(128, 128), tm + kDColSFQ + 4 * c, tm + kDColSFK + 4 * c, c > 0);
+        } else {
+          const uint32_t q16 = sbase + L::kQ16, k16 = sbase + L::kSlot16;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+            mma_f16(dS, make_sdesc(q16 + off, 16, 1024, LAYOUT_SW128), make_sdesc(k16 + off, 16, 1024, LAYOUT_SW128),
+                    idesc_f16(128, 128, false), k > 0);
+          }
+        }
+        mma_commit(&ms.bar_s_full[bb]);
+        // the K operands of this key tile are no longer needed (V: the P V issuer)
+        if (!fp16)
+          mma_commit(&ms.bar_empty4[slot]);
+        else
+          mma_commit(&ms.bar_empty_k16);
+      }
+      // drain: every tensor-core operation this thread issued completes before exit
+      mma_commit(&ms.bar_drain[0]);
+      mbar_wait(&ms.bar_drain[0], 0, kWaitNs);
+    }
+    __syncwarp();
+  } else if (warp == kDBMmaPV) {
+    // ================= P V issuer: O += P(k) V(k) from P buffer k % 2 =================
+    if (lane == 0) {
+      bool ok = true;
+      int u4 = 0, uv16 = 0;
+      uint32_t acc = 0u;
+      for (int kt = 0; ok && kt < nk; ++kt) {
+        const int bb = kt & 1;
+        const bool fp16 = ms.cls[kt] != 0;
+        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        tc_fence_after();
+        const uint32_t dO = tm + kDColO;
+        int slot = 0;
+        if (!fp16) {
+          slot = u4 % L::kNS;
+          const int use = u4 / L::kNS;
+          ++u4;
+          // V4 landed with K4 in one barrier phase; wait on it here too so that
+          // this thread observes the copy itself.  The producer cannot refill the
+          // slot before this thread releases it.
+          if (!(ok = wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
+          const uint32_t v4 = st + L::kK4Bytes, vsf = st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes;
+          for (int c = 0; c < 2; ++c)
+            tmem_cp_32x128b_x4(tm + kDColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
+          const uint32_t p4s = sbase + L::kP4 + bb * L::kP4Bytes;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            mma_nvf4(dO, make_sdesc(p4s + 32 * c, 16, 512, LAYOUT_SW64), make_sdesc(v4 + 32 * c, 16, 512, LAYOUT_SW64),
+                     idesc_nvf4(128, D), tm + kDColSFP + 8 * bb + 4 * c, tm + kDColSFV + 4 * c, acc);
+            acc = 1;
+          }
+        } else {
+          if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          ++uv16;
+          tc_fence_after();
+          const uint32_t v16 = sbase + L::kSlot16 + L::kK16Bytes;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            mma_f16_ts(dO, tm + kDColP16 + 8 * k, make_sdesc(v16 + k * 2048, 16384, 1024, LAYOUT_SW128),
+                       idesc_f16(128, D, true), acc);
+            acc = 1;
+          }
+        }
+        mma_commit(&ms.bar_o_done[bb]);
+        if (!fp16)
+          mma_commit(&ms.bar_empty4[slot]);
+        else
+          mma_commit(&ms.bar_empty_v16);
+      }
+      mma_commit(&ms.bar_drain[1]);
+      mbar_wait(&ms.bar_drain[1], 0, kWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ======================== softmax (two threads per row) ========================
+    const int quad = warp % 4, half = warp / 4;
+    const int r = quad * 32 + lane;
+    const int qrow = qt * 128 + r;
+    const uint32_t lane_base = tm + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t ocol = lane_base + kDColO + half * (D / 2);  // this thread's half of O
+    const float c2 = p.scale_log2;
+    float M = -INFINITY, l = 0.f;
+    bool failed = false;
+    // The two halves take turns on their exponentials (named barriers 2 and 3,
+    // both halves taking part), so that one half's loads, maxima and rescales
+    // overlap the other half's MUFU work.  Every key tile passes the turn
+    // exactly once per half, on every path, so neither half can be left
+    // waiting at a named barrier.
+    const auto turn_in = [&] { named_bar_sync(2 + half, kDBSoftmax); };
+    const auto turn_out = [&] { named_bar_arrive(3 - half, kDBSoftmax); };
+    if (half == 1) named_bar_arrive(2, kDBSoftmax);  // half 0 goes first
+    for (int kt = 0; kt < nk; ++kt) {
+      const int bb = kt & 1;
+      const bool fp16 = ms.cls[kt] != 0;
+      if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
+      if (failed) {
+        turn_in();
+        turn_out();
+        continue;
+      }
+      tc_fence_after();
+      // The whole row (for its maximum): this thread's keys 64h .. 64h + 63 into
+      // s, the other half into o.
+      float s[64];
+      float gh[4];  // maxima of this thread's four groups
+      float smax;
+      {
+        uint32_t vm[64], vo[64];
+        const uint32_t sb = lane_base + kDColS + 128 * bb;
+        const uint32_t mine = 64 * half, other = 64 - mine;
+        tmem_ld32(sb + mine, *reinterpret_cast<uint32_t(*)[32]>(&vm[0]));
+        tmem_ld32(sb + mine + 32, *reinterpret_cast<uint32_t(*)[32]>(&vm[32]));
+        tmem_ld32(sb + other, *reinterpret_cast<uint32_t(*)[32]>(&vo[0]));
+        tmem_ld32(sb + other + 32, *reinterpret_cast<uint32_t(*)[32]>(&vo[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&ms.bar_s_free[bb]);
+        float o[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          s[j] = __uint_as_float(vm[j]);
+          o[j] = __uint_as_float(vo[j]);
+        }
+        // Mask keys past N and, on the diagonal tile, keys after the query.
+        if (kt * 128 + 128 > p.N || (p.causal && kt == qt)) {
+          const int lim = (p.causal ? min(qrow + 1, p.N) : p.N) - kt * 128;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            if (static_cast<int>(mine) + j >= lim) s[j] = -INFINITY;
+            if (static_cast<int>(other) + j >= lim) o[j] = -INFINITY;
+          }
+        }
+        float go[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          gh[g] = max16(&s[16 * g]);
+          go[g] = max16(&o[16 * g]);
+        }
+        smax = fmaxf(fmaxf(fmax3(gh[0], gh[1], gh[2]), fmax3(gh[3], go[0], go[1])), fmaxf(go[2], go[3]));
+      }
+      // t = fl32(S * sm_scale * log2 e) is monotone in S: max t = fl32(max S * c).
+      const float Mn = fmaxf(M, ceilf(smax * c2));
+      const float alpha = (M == -INFINITY) ? 0.f : exp2_int(M - Mn);
+      const float Mx = (Mn == -INFINITY) ? 0.f : Mn;
+      const float base = static_cast<float>(kPLog2) - Mx;  // exponent offset of P * 2^11
+
+      // P buffer bb (and its scales) was multiplied two key tiles ago; the fp16
+      // P columns are single-buffered, so an fp16 tile also waits for the
+      // previous key tile's product.
+      if (kt >= 2) failed = !wait_or_abort(&ms.bar_o_done[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (!failed && fp16 && kt >= 1)
+        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      failed = __any_sync(0xffffffffu, failed);
+      if (failed) {
+        turn_in();
+        turn_out();
+        continue;
+      }
+      tc_fence_after();
+
+      turn_in();
+      // P * 2^11 = 2^(S*c + 11 - M) for this thread's 64 keys, encoded as fp16
+      // or as NVFP4 (each group folds 1/scale into the exponent).
+      float rs = 0.f;
+      const float2 c2v = make_float2(c2, c2);
+      if (fp16) {
+        const float2 bv = make_float2(base, base);
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float2 pp = ex2_fma2(s[2 * j], s[2 * j + 1], c2v, bv);
+          s[2 * j] = pp.x;
+          s[2 * j + 1] = pp.y;
+          w[j] = pack_half2(pp.x, pp.y);
+        }
+        rs = (sum16(&s[0]) + sum16(&s[16])) + (sum16(&s[32]) + sum16(&s[48]));
+        tmem_st32(lane_base + kDColP16 + 32 * half, w);
+      } else {
+        uint8_t* d4 = sm + L::kP4 + bb * L::kP4Bytes;
+        // group scales E4M3(fl32(amax / 6)) of the four groups first (independent
+        // chains), then the exponentials with 1/scale folded in, then sums and codes
+        float sce[4], bias[4];
+        uint32_t sfw = 0u;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float amax = ex2(fmaf(gh[g], c2, base));                         // max of P * 2^11
+          const uint32_t sbyte = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;  // E4M3(amax / 6)
+          const float sc = e4m3_to_f32(sbyte);
+          sce[g] = sc > 0.f ? sc : 1.0f;  // zero scale: codes round to 0, l keeps P
+          bias[g] = base - lg2(sce[g]);
+          sfw |= sbyte << (8 * g);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float2 bv = make_float2(bias[g], bias[g]);
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const float2 pp = ex2_fma2(s[16 * g + i], s[16 * g + i + 1], c2v, bv);
+            s[16 * g + i] = pp.x;
+            s[16 * g + i + 1] = pp.y;
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) rs = fmaf(sum16(&s[16 * g]), sce[g], rs);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 w = make_uint4(cvt_e2m1x8(&s[32 * c]), cvt_e2m1x8(&s[32 * c + 8]), cvt_e2m1x8(&s[32 * c + 16]),
+                                     cvt_e2m1x8(&s[32 * c + 24]));
+          *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + c)) = w;
+        }
+        // Scale factors of a 128-row A operand: the MMA reads row r's four
+        // scales of K chunk c from lane r, column base + 4c + r / 32.
+        tmem_st1(lane_base + kDColSFP + 8 * bb + 4 * half + quad, sfw);
+      }
+      turn_out();
+      l = l * alpha + rs;
+      // Rescale this thread's half of O when the maximum grew (rows with alpha
+      // = 1 are unchanged); O is stable once the previous key tile's P V
+      // product is done.
+      if (kt > 0 && __any_sync(0xffffffffu, Mn > M)) {
+        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = __any_sync(0xffffffffu, failed);
+        if (failed) continue;
+        tc_fence_after();
+        const float2 aa = make_float2(alpha, alpha);
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(ocol + 32 * cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), aa);
+            v[j] = __float_as_uint(o.x);
+            v[j + 1] = __float_as_uint(o.y);
+          }
+          tmem_st32(ocol + 32 * cc, v);
+        }
+      }
+      tmem_st_wait();
+      M = Mn;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&ms.bar_p_full[bb]);
+    }
+
+    if (half == 0) turn_in();  // the turn half 1 passed after its last key tile
+
+    // ---- epilogue: O / l -> fp16 (both carry the 2^11 pre-scale) ----
+    if (nk > 0) {
+      if (!failed)
+        failed = !wait_or_abort(&ms.bar_o_done[(nk - 1) & 1], ((nk - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      ms.lsum[half][r] = l;
+      // every softmax thread takes the same exit decision (and sees lsum)
+      failed = softmax_bar_or<kDBSoftmax>(failed);
+      if (!failed) {
+        tc_fence_after();
+        const float inv = 1.0f / (ms.lsum[0][r] + ms.lsum[1][r]);
+        __half* orow = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + half * (D / 2);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(ocol + 32 * cc, v);
+          tmem_ld_wait();
+          if (qrow < p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 w;
+              w.x = pack_half2(__uint_as_float(v[j + 0]) * inv, __uint_as_float(v[j + 1]) * inv);
+              w.y = pack_half2(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+              w.z = pack_half2(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
+              w.w = pack_half2(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + 32 * cc + j) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kDBMmaS) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+}  // namespace
+
+template <int D>
+cudaError_t launch_attention_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
+                                const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                                const attn::Params& prm, cudaStream_t st) {
+  const size_t smem = SmemDB<D>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(thrift_attention_db_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(prm.B * prm.Hq * prm.NT);
+  thrift_attention_db_kernel<D><<<grid, kDBThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_attention_db<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                             const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                             const attn::Params&, cudaStream_t);
+template cudaError_t launch_attention_db<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                              const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                              const attn::Params&, cudaStream_t);
+
+}  // namespace thrift
