@@ -233,9 +233,14 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           ++uk16;
           tc_fence_after();
         }
-        // buffer bb was last used by S(kt - 2): wait until its threads loaded it
+        // Buffers bb were last used by key tile kt - 2: wait until its S was
+        // loaded by the softmax threads, and until its P V product is done, so
+        // that the softmax threads, once they see S(kt), may overwrite P buffer
+        // bb and its scales without waiting themselves.
         if (kt >= 2) {
           if (!(ok = wait_or_abort(&ms.bar_s_free[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
+            break;
+          if (!(ok = wait_or_abort(&ms.bar_o_done[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA)))
             break;
           tc_fence_after();
         }
@@ -397,19 +402,36 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       const float Mx = (Mn == -INFINITY) ? 0.f : Mn;
       const float base = static_cast<float>(kPLog2) - Mx;  // exponent offset of P * 2^11
 
-      // P buffer bb (and its scales) was multiplied two key tiles ago; the fp16
-      // P columns are single-buffered, so an fp16 tile also waits for the
-      // previous key tile's product.
-      if (kt >= 2) failed = !wait_or_abort(&ms.bar_o_done[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
-      if (!failed && fp16 && kt >= 1)
-        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
-      failed = __any_sync(0xffffffffu, failed);
-      if (failed) {
-        turn_in();
-        turn_out();
-        continue;
+      // NVFP4 group scales E4M3(fl32(amax / 6)) of this half's four groups
+      // (independent chains, ahead of the exponentials).
+      float sce[4], bias[4];
+      uint32_t sfw = 0u;
+      if (!fp16) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float amax = ex2(fmaf(gh[g], c2, base));                         // max of P * 2^11
+          const uint32_t sbyte = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;  // E4M3(amax / 6)
+          const float sc = e4m3_to_f32(sbyte);
+          sce[g] = sc > 0.f ? sc : 1.0f;  // zero scale: codes round to 0, l keeps P
+          bias[g] = base - lg2(sce[g]);
+          sfw |= sbyte << (8 * g);
+        }
       }
-      tc_fence_after();
+
+      // P buffer bb (and its scales) is free: the S issuer waited for the P V
+      // product of key tile kt - 2 before issuing S(kt).  The fp16 P columns
+      // are single-buffered, so an fp16 tile waits for the previous key tile's
+      // product.
+      if (fp16 && kt >= 1) {
+        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = __any_sync(0xffffffffu, failed);
+        if (failed) {
+          turn_in();
+          turn_out();
+          continue;
+        }
+        tc_fence_after();
+      }
 
       turn_in();
       // P * 2^11 = 2^(S*c + 11 - M) for this thread's 64 keys, encoded as fp16
@@ -430,19 +452,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         tmem_st32(lane_base + kDColP16 + 32 * half, w);
       } else {
         uint8_t* d4 = sm + L::kP4 + bb * L::kP4Bytes;
-        // group scales E4M3(fl32(amax / 6)) of the four groups first (independent
-        // chains), then the exponentials with 1/scale folded in, then sums and codes
-        float sce[4], bias[4];
-        uint32_t sfw = 0u;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float amax = ex2(fmaf(gh[g], c2, base));                         // max of P * 2^11
-          const uint32_t sbyte = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;  // E4M3(amax / 6)
-          const float sc = e4m3_to_f32(sbyte);
-          sce[g] = sc > 0.f ? sc : 1.0f;  // zero scale: codes round to 0, l keeps P
-          bias[g] = base - lg2(sce[g]);
-          sfw |= sbyte << (8 * g);
-        }
+        // exponentials with 1/scale folded in, then sums and codes
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const float2 bv = make_float2(bias[g], bias[g]);
