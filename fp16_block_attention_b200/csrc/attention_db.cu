@@ -485,20 +485,20 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         failed = __any_sync(0xffffffffu, failed);
         if (failed) continue;
         tc_fence_after();
+        // all of this half's D/2 columns in flight at once: one load wait
         const float2 aa = make_float2(alpha, alpha);
+        uint32_t v[D / 2];
 #pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(ocol + 32 * cc, v);
-          tmem_ld_wait();
+        for (int cc = 0; cc < D / 64; ++cc) tmem_ld32(ocol + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * cc]));
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), aa);
-            v[j] = __float_as_uint(o.x);
-            v[j + 1] = __float_as_uint(o.y);
-          }
-          tmem_st32(ocol + 32 * cc, v);
+        for (int j = 0; j < D / 2; j += 2) {
+          const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), aa);
+          v[j] = __float_as_uint(o.x);
+          v[j + 1] = __float_as_uint(o.y);
         }
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) tmem_st32(ocol + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * cc]));
       }
       tmem_st_wait();
       M = Mn;
