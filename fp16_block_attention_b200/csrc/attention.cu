@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < kKPT / 32; ++q) tmem_ld32(col + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
         tmem_ld_wait();
+        tmem_ld_fence(v);
 #pragma unroll
         for (int j = 0; j < kKPT; ++j) s[j] = __uint_as_float(v[j]);
         tc_fence_before();
@@ -482,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t v[32];
             tmem_ld32(ocol + 32 * cc, v);
             tmem_ld_wait();
+            tmem_ld_fence(v);
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
             tmem_st32(ocol + 32 * cc, v);
@@ -490,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[16];
           tmem_ld16(ocol, v);
           tmem_ld_wait();
+          tmem_ld_fence(v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
           tmem_st16(ocol, v);
@@ -521,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(ocol, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
       }
       tmem_ld_wait();
+      tmem_ld_fence(v);
       if (qrow < p.N) {
 #pragma unroll
         for (int j = 0; j < kOC; j += 8) {

@@ -371,6 +371,8 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         tmem_ld32(sb + other, *reinterpret_cast<uint32_t(*)[32]>(&vo[0]));
         tmem_ld32(sb + other + 32, *reinterpret_cast<uint32_t(*)[32]>(&vo[32]));
         tmem_ld_wait();
+        tmem_ld_fence(vm);
+        tmem_ld_fence(vo);
         tc_fence_before();
         mbar_arrive(&ms.bar_s_free[bb]);
         float o[64];
@@ -491,6 +493,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc) tmem_ld32(ocol + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * cc]));
         tmem_ld_wait();
+        tmem_ld_fence(v);
 #pragma unroll
         for (int j = 0; j < D / 2; j += 2) {
           const float2 o = __fmul2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), aa);
@@ -525,6 +528,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           uint32_t v[32];
           tmem_ld32(ocol + 32 * cc, v);
           tmem_ld_wait();
+          tmem_ld_fence(v);
           if (qrow < p.N) {
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {

@@ -257,6 +257,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Ties registers written by tcgen05.ld to the preceding tcgen05.wait::ld: the
+// load's outputs are only valid after the wait, but the compiler sees them
+// defined at the load.  Passing each one through an empty volatile asm placed
+// after the wait (volatile asm statements keep their order) makes every use
+// read the register as it is after the wait.  No instruction is emitted.
+template <int N>
+__device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------ swizzled offsets ----
