@@ -282,10 +282,12 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       for (int kt = 0; ok && kt < nk; ++kt) {
         const int bb = kt & 1;
         const bool fp16 = ms.cls[kt] != 0;
-        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
-        tc_fence_after();
-        const uint32_t dO = tm + kDColO;
+        // The V operands (and the V4 scales, copied to tensor memory) do not
+        // depend on P, so they are made ready before waiting for it.  The copy
+        // follows the previous P V product in this thread's tcgen05 order, so
+        // it cannot overwrite scales that product still reads.
         int slot = 0;
+        uint32_t v4 = 0;
         if (!fp16) {
           slot = u4 % L::kNS;
           const int use = u4 / L::kNS;
@@ -296,9 +298,18 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           if (!(ok = wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           tc_fence_after();
           const uint32_t st = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
-          const uint32_t v4 = st + L::kK4Bytes, vsf = st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes;
+          v4 = st + L::kK4Bytes;
+          const uint32_t vsf = st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes;
           for (int c = 0; c < 2; ++c)
             tmem_cp_32x128b_x4(tm + kDColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
+        } else {
+          if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          ++uv16;
+        }
+        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        tc_fence_after();
+        const uint32_t dO = tm + kDColO;
+        if (!fp16) {
           const uint32_t p4s = sbase + L::kP4 + bb * L::kP4Bytes;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -307,9 +318,6 @@ __global__ void __launch_bounds__(kDBThreads, 1)
             acc = 1;
           }
         } else {
-          if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
-          ++uv16;
-          tc_fence_after();
           const uint32_t v16 = sbase + L::kSlot16 + L::kK16Bytes;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
