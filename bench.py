@@ -167,6 +167,25 @@ def flop_split(w, mask_np):
     return f16, total - f16
 
 
+MUFU_PER_CLK_PER_SM = 16  # ex2 / lg2 throughput of compute capability 10.0 (16 per clock per SM)
+
+
+def mufu_ops(w, mask_np):
+    """MUFU operations the method needs at least: one exponential per valid
+    (query, key) pair, and per 16-key NVFP4 group of P one exponential (the
+    group maximum) and one logarithm (its scale)."""
+    f16, f4 = flop_split(w, mask_np)
+    per_elem = 4.0 * w.D
+    return (f16 + f4) / per_elem + (f4 / per_elem) * 2.0 / 16.0
+
+
+def mufu_ceiling(w, mask_np, attn_ms, sm_mhz, n_sm):
+    ops = mufu_ops(w, mask_np)
+    bound_ms = ops / (MUFU_PER_CLK_PER_SM * n_sm * sm_mhz * 1e6) * 1e3
+    return {"ops": int(ops), "per_clk_per_sm": MUFU_PER_CLK_PER_SM, "sm_mhz": sm_mhz,
+            "bound_ms": round(bound_ms, 4), "frac": round(bound_ms / attn_ms, 4)}
+
+
 # ------------------------------------------------------------------ our arm ---
 def run_gpu(args):
     import torch
@@ -319,6 +338,8 @@ def run_gpu(args):
                      "t_tensor_ms": round(t_tensor * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
                      "algorithmic_bytes": int(bytes_alg)},
         "clocks": clocks,
+        "mufu_ceiling": mufu_ceiling(w, mask.cpu().numpy(), attn_ms, clocks.get("sm_mhz") or 1965.0,
+                                     torch.cuda.get_device_properties(dev).multi_processor_count),
         "e2e": {"value": round(whole_job_tflops(flops, e2e_ms, n), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "api": "attention_fused (quantise + select + attend) per step",
@@ -421,6 +442,69 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Attention-kernel time for every workload at its rho, and for the 32k GQA
+    workload at rho in {0, 1, 5, 10, 100}%: ms, effective TFLOP/s, blended
+    roofline fraction and MUFU fraction.  Prints a markdown table."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, _ = load_peaks()
+    p16 = peaks["bf16_tflops"] * 1e12
+    p4 = FP4_OVER_BF16 * p16
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    # tensor-pipe rates of the two MMA kinds (measurement helper of the library)
+    stream = torch.cuda.current_stream(dev)
+    for kind, name, iters in ((0, "NVFP4 mxf4nvf4 M128 N256 K64", 20000), (1, "fp16 f16 M128 N256 K16", 20000)):
+        thrift.mma_rate_probe(kind, 100, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        thrift.mma_rate_probe(kind, iters, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if thrift.last_device_error(stream) != 0:
+            raise RuntimeError("the MMA rate probe reported a bounded-wait timeout")
+        tf = n_sm * iters * thrift.MMA_RATE_FLOP[kind] / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        print(f"tensor-pipe rate, {name}: {tf:.1f} TFLOP/s ({n_sm} SMs)")
+    print()
+    cases = [(w, w.rho) for w in synth.WORKLOADS] + [(synth.GQA_N32K, r) for r in (0.0, 0.01, 0.10, 1.0)]
+    print("| workload | rho | blk | attention ms | effective TFLOP/s | roofline frac | MUFU frac |")
+    print("|---|---:|---:|---:|---:|---:|---:|")
+    for w, rho in cases:
+        Q, K, V = synth.generate(w)
+        Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+        sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+        qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+        mask = thrift.select_blocks(Qd, Kd, sh, rho)
+        Od = torch.empty_like(Qd)
+        stream = torch.cuda.current_stream(dev)
+        for _ in range(args.warmup):
+            thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(2, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n):
+            thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if thrift.last_device_error(stream) != 0:
+            raise RuntimeError(f"a kernel reported a bounded-wait timeout on {w.name}")
+        ms = e0.elapsed_time(e1) / n
+        m = mask.cpu().numpy()
+        f16, f4 = flop_split(w, m)
+        t_bound = max(f16 / p16 + f4 / p4, attention_bytes(w, m) / (peaks["hbm_gbs"] * 1e9))
+        mufu = mufu_ceiling(w, m, ms, 1965.0, n_sm)
+        print(f"| {w.name} | {rho:g} | {w.blk} | {ms:.4f} | {w.flops() / (ms * 1e-3) / 1e12:.1f} | "
+              f"{t_bound * 1e3 / ms:.4f} | {mufu['frac']:.4f} |", flush=True)
+        del Qd, Kd, Vd, Od, qz, mask
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,10 +514,14 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the attention kernel on every workload and rho (markdown table), then exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

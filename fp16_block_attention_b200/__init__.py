@@ -78,6 +78,7 @@ def _load():
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_last_device_error": ([vp], st),
+        "thrift_mma_rate_probe": ([st, st, vp], st),
         "thrift_strerror": ([st], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -92,7 +93,7 @@ _lib = _load()
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
            "thrift_select_blocks_static", "thrift_attention", "thrift_fused_workspace_bytes",
-           "thrift_attention_fused", "thrift_last_device_error", "thrift_strerror")
+           "thrift_attention_fused", "thrift_last_device_error", "thrift_mma_rate_probe", "thrift_strerror")
 
 
 def lib():
@@ -239,6 +240,15 @@ def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, str
         _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(),
         _stream(stream)))
     return out
+
+
+MMA_RATE_FLOP = {0: 2 * 128 * 256 * 64, 1: 2 * 128 * 256 * 16}  # per product: NVFP4, fp16
+
+
+def mma_rate_probe(kind: int, iters: int, stream=None):
+    """Launch the tensor-pipe rate probe (measurement helper, see thrift.h):
+    one CTA per SM issues `iters` products of MMA_RATE_FLOP[kind] flop each."""
+    _check("thrift_mma_rate_probe", _lib.thrift_mma_rate_probe(int(kind), int(iters), _stream(stream)))
 
 
 def last_device_error(stream=None) -> int:

@@ -217,6 +217,16 @@ thrift_status thrift_last_device_error(void* stream) {
   return THRIFT_OK;
 }
 
+thrift_status thrift_mma_rate_probe(int kind, int iters, void* stream) {
+  if (kind < 0 || kind > 1 || iters <= 0 || iters > (1 << 24)) return THRIFT_ERR_INVALID_ARG;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return THRIFT_ERR_CUDA;
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  return from_cuda(launch_mma_rate(kind, iters, nsm, err, static_cast<cudaStream_t>(stream)));
+}
+
 const char* thrift_strerror(thrift_status status) {
   switch (status) {
     case THRIFT_OK: return "ok";

@@ -44,6 +44,9 @@ cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shap
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st);
 
+// Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
+cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);
+
 cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
                              const thrift_shape& s, void* O, uint32_t* err, cudaStream_t st);

@@ -65,6 +65,14 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert lib.thrift_attention_fused(fake, fake, fake, sh, 0.05, fake, fake, 8, None) == 5
 
 
+def test_mma_rate_probe_rejects_bad_arguments_before_launch():
+    lib = thrift.lib()
+    assert lib.thrift_mma_rate_probe(2, 10, None) == 1
+    assert lib.thrift_mma_rate_probe(-1, 10, None) == 1
+    assert lib.thrift_mma_rate_probe(0, 0, None) == 1
+    assert lib.thrift_mma_rate_probe(1, (1 << 24) + 1, None) == 1
+
+
 def test_workspace_sizes_cover_the_parts():
     sh = thrift.Shape(1, 4, 2, 512, 128, 64, True)
     need = thrift.fused_workspace_bytes(sh)

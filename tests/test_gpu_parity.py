@@ -185,3 +185,9 @@ def test_gap_recovered_agrees_with_oracle():
     g = oracle.gap_recovered(gpu[0.0], gpu[w.rho], gpu[1.0], ex)
     r = oracle.gap_recovered(ref[0.0], ref[w.rho], ref[1.0], ex)
     assert abs(g - r) <= 1.0, (g, r)
+
+
+def test_mma_rate_probe_runs_without_error():
+    thrift.mma_rate_probe(0, 64)
+    thrift.mma_rate_probe(1, 64)
+    assert thrift.last_device_error() == 0
