@@ -472,6 +472,44 @@ def run_sweep(args):
         print(f"tensor-pipe rate, {name}: {tf:.1f} TFLOP/s ({n_sm} SMs)")
     print()
     cases = [(w, w.rho) for w in synth.WORKLOADS] + [(synth.GQA_N32K, r) for r in (0.0, 0.01, 0.10, 1.0)]
+    # quantisation and selection on the 32k GQA workload: time and achieved HBM
+    # bandwidth over their algorithmic bytes
+    w = synth.GQA_N32K
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+    sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+    qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+    mask = torch.empty((w.B, w.Hq, sh.nb, sh.nb), dtype=torch.uint8, device=dev)
+    sel_ws = torch.empty(thrift.select_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+    q_el, kv_el = Qd.numel(), Kd.numel()
+    stages = [
+        ("quantise Q (NVFP4 along D)", lambda: thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, stream),
+         q_el * (2 + 0.5625)),
+        ("quantise K (NVFP4 along D)", lambda: thrift.quantize_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, stream),
+         kv_el * (2 + 0.5625)),
+        ("quantise V (NVFP4 along keys)", lambda: thrift.quantize_nvfp4(Vd, thrift.V, sh, qz.v4, qz.vs, stream),
+         kv_el * (2 + 0.5625)),
+        ("select (pool Q and K, score, top-k)", lambda: thrift.select_blocks(Qd, Kd, sh, w.rho, mask, sel_ws, stream),
+         (q_el + kv_el) * 2),
+    ]
+    print(f"| stage ({w.name}) | ms | algorithmic GB | achieved GB/s |")
+    print("|---|---:|---:|---:|")
+    for name, fn, nbytes in stages:
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 10
+        print(f"| {name} | {ms:.4f} | {nbytes / 1e9:.3f} | {nbytes / (ms * 1e-3) / 1e9:.0f} |", flush=True)
+    print()
+    del Qd, Kd, Vd, qz, mask, sel_ws
+    torch.cuda.empty_cache()
+
     print("| workload | rho | blk | attention ms | effective TFLOP/s | roofline frac | MUFU frac |")
     print("|---|---:|---:|---:|---:|---:|---:|")
     for w, rho in cases:
