@@ -1,7 +1,6 @@
-// Stage 2 of the method: "the selected blocks are computed in FP16 and the
-// remaining blocks in FP4, with both paths merged via online softmax into a
-// single output" (ThriftAttention abstract; summary, "technical approach"
-// items 3-4).
+// Stage 2 of the method (ThriftAttention abstract; summary, technical
+// approach items 3-4): picked block pairs run in FP16, all others in FP4, and
+// one online softmax folds both kinds of tile into the same output.
 //
 // One CTA computes one 128-row query tile of one (batch, query head) and walks
 // its key tiles (128 keys each).  Per key tile the selection mask gives the

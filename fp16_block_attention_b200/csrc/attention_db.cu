@@ -1,7 +1,6 @@
-// Stage 2 of the method for 128 x 128 selection blocks ("the selected blocks
-// are computed in FP16 and the remaining blocks in FP4, with both paths merged
-// via online softmax into a single output", ThriftAttention abstract), with
-// the S products and the P operands double-buffered.
+// Stage 2 of the method for 128 x 128 selection blocks (ThriftAttention
+// abstract: picked block pairs in FP16, the rest in FP4, one online softmax
+// over both), with the S products and the P operands double-buffered.
 //
 // A CTA owns one 128-row query tile of one (batch, query head).  With blk =
 // 128 each key tile is one selection block, so it is entirely FP16 or
