@@ -2,9 +2,10 @@
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It is plain C
-(``oracle.c``, FP64 arithmetic, OpenMP over rows) loaded with ctypes, and it
-shares no code with the CUDA library.  See ``oracle.c`` for what each function
-computes and which reading of the method it takes.
+(``oracle.c``, FP64 arithmetic, OpenMP over rows) loaded with ctypes, plus the
+numpy module ``vertical_window`` (the HyQuant-style selector), and it shares
+no code with the CUDA library.  See ``oracle.c`` and ``vertical_window.py``
+for what each function computes and which reading of the method it takes.
 """
 from __future__ import annotations
 
@@ -170,6 +171,21 @@ def select(Q, K, blk, causal, sm_scale, rho):
     if _load().orc_select(Q.ctypes.data, K.ctypes.data, B, Hq, Hkv, N, D, blk, int(causal),
                           float(sm_scale), float(rho), mask.ctypes.data):
         raise ValueError("orc_select rejected the shape")
+    return mask
+
+
+def select_vertical_window(Q, K, blk, causal, sm_scale, rho, window):
+    """Mask [B,Hq,nb,nb] (u8) of the vertical-line / local-window selector
+    (``vertical_window``) on the pooled scores of every (batch, query head)."""
+    from . import vertical_window as vw
+    B, Hq = Q.shape[:2]
+    group = Hq // K.shape[1]
+    nb = Q.shape[2] // blk
+    mask = np.zeros((B, Hq, nb, nb), np.uint8)
+    for b in range(B):
+        for h in range(Hq):
+            sc = pooled_scores(Q[b, h], K[b, h // group], blk, causal, sm_scale)
+            mask[b, h] = vw.select_head(sc, causal, rho, window, budget)
     return mask
 
 
