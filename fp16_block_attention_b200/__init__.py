@@ -74,6 +74,7 @@ def _load():
         "thrift_select_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_select_blocks_static": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
+        "thrift_select_blocks_vertical_window": ([vp, vp, psh, ctypes.c_double, st, vp, vp, sz, vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
@@ -92,7 +93,8 @@ _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
-           "thrift_select_blocks_static", "thrift_attention", "thrift_fused_workspace_bytes",
+           "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_attention",
+           "thrift_fused_workspace_bytes",
            "thrift_attention_fused", "thrift_last_device_error", "thrift_mma_rate_probe", "thrift_strerror")
 
 
@@ -169,6 +171,24 @@ def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, 
     _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
                                                              float(rho), _ptr(mask), _ptr(ws), ws.numel(),
                                                              _stream(stream)))
+    return mask
+
+
+def select_blocks_vertical_window(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, window: int,
+                                  mask=None, ws=None, stream=None):
+    """Selection mask [B, Hq, nb, nb] (u8) of the HyQuant-style selector: the
+    local window of `window` blocks, then whole key-block columns ranked by
+    the pooled attention mass they receive, on the same budget as
+    select_blocks."""
+    _dev(Qt, "Q", torch.float16)
+    _dev(Kt, "K", torch.float16)
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
+    if ws is None:
+        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_select_blocks_vertical_window", _lib.thrift_select_blocks_vertical_window(
+        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), int(window), _ptr(mask), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return mask
 
 

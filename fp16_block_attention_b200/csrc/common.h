@@ -43,6 +43,10 @@ cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shap
                                  cudaStream_t st);
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st);
+// Vertical-line / local-window selector (select.cu); nb = N / blk <= kMaxVWBlocks.
+constexpr int kMaxVWBlocks = 2048;
+cudaError_t launch_select_vertical_window(const void* Q, const void* K, const thrift_shape& s, double rho, int window,
+                                          uint8_t* mask, void* ws, cudaStream_t st);
 
 // Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
 cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);

@@ -1,6 +1,6 @@
-// Stage 1 of the method: "a heuristic rapidly selects a small number of
-// important query-key block pairs for FP16 precision" (ThriftAttention
-// abstract).  Reading used here: pooled scores from FP32 block means,
+// Stage 1 of the method (ThriftAttention abstract): a cheap heuristic picks
+// the few query-key block pairs that matter most and marks them for FP16.
+// Reading used here: pooled scores from FP32 block means,
 // score(i,j) = fl32(sm_scale * fl32(mean_q(i) . mean_k(j))), and per
 // (batch, query head) the top k = ceil(rho * #valid - 1e-9) pairs, with the
 // diagonal pairs (i,i) and the key-block-0 pairs (i,0) ranked first and ties
@@ -15,6 +15,22 @@
 //   top-k    one CTA per head: radix select of the k-th largest 64-bit key
 //            (forced bit | order-preserving score bits | inverted index), so
 //            the selection is exactly k pairs, then the mask.
+//
+// A second selector, after HyQuant (abstract in the body of the page titled
+// "LampAttention: Look-Ahead Mixed-Precision FlashAttention for Dedicated
+// Accelerators"): there, the keys that many queries attend to (vertical lines
+// of the attention map) and a sliding window next to the diagonal keep full
+// precision, picked by a cheap attention-pattern signal.  Here the same idea
+// at block granularity and on the same budget k:
+//   column signal  per (batch, query head), from the same pooled scores: the
+//            softmax of each valid row of block scores, summed per key-block
+//            column (the attention mass a key block receives), in FP32 and in
+//            a fixed order; columns ranked by it (ties: lower column first);
+//   top-k    the same radix select on the key (window bit | inverted column
+//            rank | order-preserving score bits | inverted index): the pairs
+//            of the local window (i - W < j <= i, or |i - j| < W without the
+//            causal mask) first, then whole columns in rank order, each by
+//            descending score.
 #include <cuda_fp16.h>
 
 #include "common.h"
@@ -29,6 +45,7 @@ struct SelectWs {
   float* qm;      // [B*Hq][nb][D]
   float* km;      // [B*Hkv][nb][D]
   float* scores;  // [B*Hq][nb][nb]
+  int* rank;      // [B*Hq][nb] column ranks (vertical-line selector)
 };
 
 SelectWs carve(void* ws, const thrift_shape& s) {
@@ -40,6 +57,8 @@ SelectWs carve(void* ws, const thrift_shape& s) {
   w.km = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * static_cast<size_t>(s.B) * s.Hkv * nb * s.D);
   w.scores = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * static_cast<size_t>(s.B) * s.Hq * nb * nb);
+  w.rank = reinterpret_cast<int*>(p);
   return w;
 }
 
@@ -105,14 +124,84 @@ __device__ __forceinline__ uint64_t pair_key(float score, int i, int j, int nb) 
   return (forced << 63) | (static_cast<uint64_t>(u) << 31) | (0x7FFFFFFFull - idx);
 }
 
-// One CTA (1024 threads) per (batch, query head).
+// Key of the vertical-line / local-window selector: window bit (63), inverted
+// column rank (11 bits, 52..62), order-preserving score bits (20..51),
+// inverted query block (11 bits).  Ranks are a permutation of the columns, so
+// the rank fixes j and the key is unique; nb <= 2048.
+__device__ __forceinline__ uint64_t vw_key(float score, int i, int j, int causal, int window, int rank) {
+  if (score == 0.0f) score = 0.0f;
+  uint32_t u = __float_as_uint(score);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const bool in_window = causal ? (j <= i && j > i - window) : (abs(i - j) < window);
+  return (static_cast<uint64_t>(in_window) << 63) | (static_cast<uint64_t>(2047 - rank) << 52) |
+         (static_cast<uint64_t>(u) << 20) | static_cast<uint64_t>(2047 - i);
+}
+
+// Column signal and ranks of the vertical-line selector, one CTA (1024
+// threads) per (batch, query head); nb <= kMaxVWBlocks.  Deterministic: every
+// sum has a fixed order.
+__global__ void __launch_bounds__(1024) column_rank_kernel(const float* __restrict__ scores, int nb, int causal,
+                                                           int* __restrict__ rank_out) {
+  __shared__ float rmax[kMaxVWBlocks], rinv[kMaxVWBlocks], colv[kMaxVWBlocks];
+  const size_t bh = blockIdx.x;
+  const float* sc = scores + bh * nb * static_cast<size_t>(nb);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // row softmax of the valid block scores: maximum and 1 / sum of exponentials
+  for (int i = warp; i < nb; i += 32) {
+    const int jn = causal ? i + 1 : nb;
+    float m = -INFINITY;
+    for (int j = lane; j < jn; j += 32) m = fmaxf(m, sc[static_cast<size_t>(i) * nb + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float d = 0.f;
+    for (int j = lane; j < jn; j += 32) d += expf(sc[static_cast<size_t>(i) * nb + j] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (lane == 0) {
+      rmax[i] = m;
+      rinv[i] = 1.0f / d;
+    }
+  }
+  __syncthreads();
+  // attention mass each key-block column receives, summed over rows in order
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    float a = 0.f;
+    for (int i = causal ? j : 0; i < nb; ++i) a += expf(sc[static_cast<size_t>(i) * nb + j] - rmax[i]) * rinv[i];
+    colv[j] = a;
+  }
+  __syncthreads();
+  // rank: columns with a larger signal, or an equal one and a lower index
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const float vj = colv[j];
+    int rk = 0;
+    for (int jj = 0; jj < nb; ++jj) {
+      const float x = colv[jj];
+      rk += (x > vj || (x == vj && jj < j)) ? 1 : 0;
+    }
+    rank_out[bh * nb + j] = rk;
+  }
+}
+
+// One CTA (1024 threads) per (batch, query head).  VW = 0: the method's key;
+// VW = 1: the vertical-line / local-window key (column ranks in `rank`).
+template <int VW>
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int nb, int causal,
-                                                    long long k, uint8_t* __restrict__ mask) {
+                                                    long long k, uint8_t* __restrict__ mask,
+                                                    const int* __restrict__ rank, int window) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ long long s_remaining;
   __shared__ int s_done;
+  __shared__ int s_rank[VW ? kMaxVWBlocks : 1];
   const size_t bh = blockIdx.x;
+  if (VW) {
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) s_rank[j] = rank[bh * nb + j];
+    __syncthreads();
+  }
+  const auto key_of = [&](float score, int i, int j) -> uint64_t {
+    if (VW) return vw_key(score, i, j, causal, window, s_rank[j]);
+    return pair_key(score, i, j, nb);
+  };
   const float* sc = scores + bh * nb * static_cast<size_t>(nb);
   uint8_t* m = mask + bh * nb * static_cast<size_t>(nb);
   const size_t total = static_cast<size_t>(nb) * nb;
@@ -138,7 +227,7 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
       for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
         const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
         if (causal && j > i) continue;
-        const uint64_t key = pair_key(sc[idx], i, j, nb);
+        const uint64_t key = key_of(sc[idx], i, j);
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
@@ -166,7 +255,7 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
   for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
     const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
     uint8_t v = 0;
-    if (!(causal && j > i) && !select_none) v = pair_key(sc[idx], i, j, nb) >= threshold ? 1 : 0;
+    if (!(causal && j > i) && !select_none) v = key_of(sc[idx], i, j) >= threshold ? 1 : 0;
     m[idx] = v;
   }
 }
@@ -176,23 +265,45 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
 size_t select_workspace_bytes(const thrift_shape& s) {
   const size_t nb = s.N / s.blk;
   return align_up(sizeof(float) * s.B * s.Hq * nb * s.D) + align_up(sizeof(float) * s.B * s.Hkv * nb * s.D) +
-         align_up(sizeof(float) * s.B * s.Hq * nb * nb);
+         align_up(sizeof(float) * s.B * s.Hq * nb * nb) + align_up(sizeof(int) * s.B * s.Hq * nb);
+}
+
+namespace {
+long long budget_pairs(const thrift_shape& s, double rho) {
+  const int nb = s.N / s.blk;
+  const long long valid = s.causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
+  double kk = ceil(rho * static_cast<double>(valid) - 1e-9);
+  if (kk < 0) kk = 0;
+  if (kk > static_cast<double>(valid)) kk = static_cast<double>(valid);
+  return static_cast<long long>(kk);
+}
+
+void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s, const SelectWs& w, cudaStream_t st) {
+  const int nb = s.N / s.blk;
+  pool_kernel<<<dim3(nb, s.B * s.Hq), s.D / 2, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
+  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
+  const int tiles = (nb + 31) / 32;
+  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
+                                                               s.sm_scale, w.scores);
+}
+}  // namespace
+
+cudaError_t launch_select_vertical_window(const void* Q, const void* K, const thrift_shape& s, double rho, int window,
+                                          uint8_t* mask, void* ws, cudaStream_t st) {
+  const int nb = s.N / s.blk;
+  SelectWs w = carve(ws, s);
+  launch_pool_and_scores(Q, K, s, w, st);
+  column_rank_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, w.rank);
+  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), mask, w.rank, window);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st) {
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
-  pool_kernel<<<dim3(nb, s.B * s.Hq), s.D / 2, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
-  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
-  const int tiles = (nb + 31) / 32;
-  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
-                                                               s.sm_scale, w.scores);
-  const long long valid = s.causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
-  double kk = ceil(rho * static_cast<double>(valid) - 1e-9);
-  if (kk < 0) kk = 0;
-  if (kk > static_cast<double>(valid)) kk = static_cast<double>(valid);
-  topk_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, static_cast<long long>(kk), mask);
+  launch_pool_and_scores(Q, K, s, w, st);
+  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), mask, nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -104,17 +104,41 @@ THRIFT_API thrift_status thrift_quant_bytes(const thrift_shape* shape, thrift_op
 THRIFT_API thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
                                     void* scales, void* stream);
 
-/* Workspace bytes thrift_select_blocks needs (block means and pooled scores). */
+/* Workspace bytes thrift_select_blocks and thrift_select_blocks_vertical_window
+ * need (block means, pooled scores, column ranks). */
 THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape, size_t* bytes);
 
-/* Stage 1 ("a heuristic rapidly selects a small number of important
- * query-key block pairs", ThriftAttention abstract): writes
+/* Stage 1 (ThriftAttention abstract: a cheap heuristic picks the few
+ * query-key block pairs that matter most): writes
  * mask [B][Hq][nb][nb] (nb = N/blk) with 1 for pairs computed in FP16 and 0
  * for FP4 pairs and for invalid (causal, j > i) pairs.
  * rho in [0,1]; ws: device workspace of at least
  * thrift_select_workspace_bytes() bytes (contents need not be initialised). */
 THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
                                    uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
+
+/* An alternative stage 1 on the same FP16 budget, after HyQuant (abstract in
+ * the body of the page titled "LampAttention: Look-Ahead Mixed-Precision
+ * FlashAttention for Dedicated Accelerators"): HyQuant keeps full precision
+ * for the keys that many queries attend to (vertical lines of the attention
+ * map) and for a sliding window beside the diagonal, chosen by a cheap signal
+ * of the attention pattern.  At block granularity, per (batch, query head):
+ *   - pooled scores s(i,j) exactly as thrift_select_blocks computes them;
+ *   - column signal v_j = sum over valid rows i of softmax_j'(s(i,j'))[j], the
+ *     pooled attention mass key block j receives (FP32, fixed summation
+ *     order: per row the maximum, then the sum of exp(s - max); per column
+ *     the sum over i in increasing order); columns ranked by v descending,
+ *     ties to the lower j;
+ *   - the same budget k = ceil(rho * #valid_pairs - 1e-9); pairs ordered by
+ *     (in the window: i - window < j <= i causal, |i - j| < window otherwise)
+ *     first, then the column's rank, then s(i,j) descending, then lower i;
+ *     the first k are kept.
+ * window >= 0 in blocks (0: no window).  nb = N/blk must be <= 2048
+ * (THRIFT_ERR_UNSUPPORTED otherwise).  Workspace, mask layout and errors as
+ * for thrift_select_blocks; the workspace size is the same call. */
+THRIFT_API thrift_status thrift_select_blocks_vertical_window(const void* Q, const void* K, const thrift_shape* shape,
+                                                              double rho, int window, uint8_t* mask, void* ws,
+                                                              size_t ws_bytes, void* stream);
 
 /* thrift_select_blocks without a caller-supplied workspace.  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate
@@ -140,9 +164,8 @@ THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, cons
 THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* K, const thrift_shape* shape,
                                                      double rho, uint8_t* mask, void* stream);
 
-/* Stage 2 ("the selected blocks are computed in FP16 and the remaining blocks
- * in FP4, with both paths merged via online softmax into a single output",
- * ThriftAttention abstract): O [B][Hq][N][D] fp16.
+/* Stage 2 (ThriftAttention abstract: picked pairs in FP16, the others in
+ * FP4, one online softmax merging both): O [B][Hq][N][D] fp16.
  * mask: as written by thrift_select_blocks; q4/qs, k4/ks, v4/vs: the NVFP4
  * copies written by thrift_quantize_nvfp4 for Q, K and V. */
 THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,

@@ -59,6 +59,11 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert lib.thrift_select_blocks(fake, fake, sh, 1.5, fake, fake, 1 << 30, None) == 1
     assert lib.thrift_select_blocks(fake, fake, sh, 0.05, fake, None, 0, None) == 5
     assert lib.thrift_select_blocks(fake, fake, sh, 0.05, fake, fake, 16, None) == 5
+    vw = lib.thrift_select_blocks_vertical_window
+    assert vw(fake, fake, sh, 0.05, -1, fake, fake, 1 << 30, None) == 1      # negative window
+    assert vw(fake, None, sh, 0.05, 2, fake, fake, 1 << 30, None) == 1
+    assert vw(fake, fake, sh, -0.5, 2, fake, fake, 1 << 30, None) == 1
+    assert vw(fake, fake, sh, 0.05, 2, fake, fake, 16, None) == 5
     args = [fake] * 10
     assert lib.thrift_attention(None, *args[:9], sh, fake, None) == 1
     assert lib.thrift_attention_fused(fake, fake, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1
