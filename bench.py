@@ -491,6 +491,9 @@ def run_sweep(args):
          kv_el * (2 + 0.5625)),
         ("select (pool Q and K, score, top-k)", lambda: thrift.select_blocks(Qd, Kd, sh, w.rho, mask, sel_ws, stream),
          (q_el + kv_el) * 2),
+        ("select, vertical-line / window W=1 (pool, score, column rank, top-k)",
+         lambda: thrift.select_blocks_vertical_window(Qd, Kd, sh, w.rho, 1, mask, sel_ws, stream),
+         (q_el + kv_el) * 2),
     ]
     print(f"| stage ({w.name}) | ms | algorithmic GB | achieved GB/s |")
     print("|---|---:|---:|---:|")

@@ -7,7 +7,9 @@ looks at that shape through the proxy, on synthetic inputs.
 
 At every length the GPU's gap on sampled rows must agree with the oracle's
 within one point (the acceptance bar for the gap).  Run with -s to see the
-series: one line per length with the three relative errors and both gaps."""
+series: one line per length with the three relative errors and both gaps,
+and the gap of the vertical-line / local-window selector on the same budget
+(its parity with the oracle is in test_gpu_vertical_window)."""
 import numpy as np
 import pytest
 
@@ -44,6 +46,11 @@ def test_gap_recovered_by_sequence_length(N):
                                  ).astype(np.float64)
     g = oracle.gap_recovered(gpu[0.0], gpu[w.rho], gpu[1.0], ex)
     r = oracle.gap_recovered(ref[0.0], ref[w.rho], ref[1.0], ex)
+    # the vertical-line / local-window selector (window of one block) on the same budget
+    m_vw = thrift.select_blocks_vertical_window(Qd, Kd, sh, w.rho, 1)
+    o_vw = thrift.attention(Qd, Kd, Vd, m_vw, thrift.quantize_all(Qd, Kd, Vd, sh), sh).cpu().numpy()
+    assert thrift.last_device_error() == 0
+    g_vw = oracle.gap_recovered(gpu[0.0], o_vw[rows[:, 0], rows[:, 1], rows[:, 2]].astype(np.float64), gpu[1.0], ex)
     print(f"\ngap sweep N={N}: E(rho=0)={_rel_err(gpu[0.0], ex):.5f} E(rho={w.rho})={_rel_err(gpu[w.rho], ex):.5f} "
-          f"E(rho=1)={_rel_err(gpu[1.0], ex):.5f} gap_gpu={g:.2f} gap_oracle={r:.2f}")
+          f"E(rho=1)={_rel_err(gpu[1.0], ex):.5f} gap_gpu={g:.2f} gap_oracle={r:.2f} gap_vertical_window={g_vw:.2f}")
     assert abs(g - r) <= 1.0, (g, r)
