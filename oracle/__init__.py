@@ -3,9 +3,10 @@
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It is plain C
 (``oracle.c``, FP64 arithmetic, OpenMP over rows) loaded with ctypes, plus the
-numpy module ``vertical_window`` (the HyQuant-style selector), and it shares
-no code with the CUDA library.  See ``oracle.c`` and ``vertical_window.py``
-for what each function computes and which reading of the method it takes.
+numpy modules ``vertical_window`` (the HyQuant-style selector) and ``decode``
+(one decode step over the prefill's caches), and it shares no code with the
+CUDA library.  See ``oracle.c`` and the two modules for what each function
+computes and which reading of the method it takes.
 """
 from __future__ import annotations
 
