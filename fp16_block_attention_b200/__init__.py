@@ -78,6 +78,11 @@ def _load():
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_pool_keys": ([vp, psh, vp, vp], st),
+        "thrift_decode_select": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
+        "thrift_decode_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
+        "thrift_decode_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp, sz, vp], st),
+        "thrift_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_last_device_error": ([vp], st),
         "thrift_mma_rate_probe": ([st, st, vp], st),
         "thrift_strerror": ([st], ctypes.c_char_p),
@@ -95,7 +100,9 @@ _lib = _load()
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
            "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_attention",
            "thrift_fused_workspace_bytes",
-           "thrift_attention_fused", "thrift_last_device_error", "thrift_mma_rate_probe", "thrift_strerror")
+           "thrift_attention_fused", "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
+           "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error", "thrift_mma_rate_probe",
+           "thrift_strerror")
 
 
 def lib():
@@ -263,6 +270,70 @@ def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, str
 
 
 MMA_RATE_FLOP = {0: 2 * 128 * 256 * 64, 1: 2 * 128 * 256 * 16}  # per product: NVFP4, fp16
+
+
+# ---- decode ------------------------------------------------------------------
+def pool_keys(Kt: torch.Tensor, shape: Shape, km=None, stream=None):
+    """FP32 block means of K: [B, Hkv, nb, D]."""
+    _dev(Kt, "K", torch.float16)
+    if km is None:
+        km = torch.empty((shape.B, shape.Hkv, shape.nb, shape.D), dtype=torch.float32, device=Kt.device)
+    _check("thrift_pool_keys", _lib.thrift_pool_keys(_ptr(Kt), ctypes.byref(shape.c()), _ptr(km), _stream(stream)))
+    return km
+
+
+def decode_select(qt: torch.Tensor, km: torch.Tensor, shape: Shape, rho: float, mask=None, stream=None):
+    """Decode selection mask [B, Hq, nb] (u8, 1 = FP16 block) of q [B, Hq, D]."""
+    _dev(qt, "q", torch.float16)
+    _dev(km, "km", torch.float32)
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb), dtype=torch.uint8, device=qt.device)
+    _check("thrift_decode_select", _lib.thrift_decode_select(_ptr(qt), _ptr(km), ctypes.byref(shape.c()),
+                                                             float(rho), _ptr(mask), _stream(stream)))
+    return mask
+
+
+def decode_workspace_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check("thrift_decode_workspace_bytes", _lib.thrift_decode_workspace_bytes(ctypes.byref(shape.c()),
+                                                                               ctypes.byref(n)))
+    return n.value
+
+
+def decode_attention(qt, Kt, Vt, kq: "Quantised", mask, shape: Shape, out=None, ws=None, stream=None):
+    """Decode output [B, Hq, D] fp16 for the given block mask; kq holds the
+    NVFP4 copies of K and V (its q4 / qs fields are not read)."""
+    for t, n in ((qt, "q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    if out is None:
+        out = torch.empty((shape.B, shape.Hq, shape.D), dtype=torch.float16, device=qt.device)
+    if ws is None:
+        ws = torch.empty(decode_workspace_bytes(shape), dtype=torch.uint8, device=qt.device)
+    _check("thrift_decode_attention", _lib.thrift_decode_attention(
+        _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(mask),
+        ctypes.byref(shape.c()), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def decode_step(qt, Kt, Vt, kq: "Quantised", km, shape: Shape, rho: float, out=None, ws=None, stream=None):
+    """Selection and attention of one decode step: O [B, Hq, D] fp16."""
+    for t, n in ((qt, "q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    if out is None:
+        out = torch.empty((shape.B, shape.Hq, shape.D), dtype=torch.float16, device=qt.device)
+    if ws is None:
+        ws = torch.empty(decode_workspace_bytes(shape), dtype=torch.uint8, device=qt.device)
+    _check("thrift_decode_step", _lib.thrift_decode_step(
+        _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(km),
+        ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def quantize_kv(Kt, Vt, shape: Shape, stream=None) -> "Quantised":
+    """NVFP4 copies of K and V only (the decode cache); q4 / qs are None."""
+    k4, ks = quantize_nvfp4(Kt, K, shape, stream=stream)
+    v4, vs = quantize_nvfp4(Vt, V, shape, stream=stream)
+    return Quantised(None, None, k4, ks, v4, vs)
 
 
 def mma_rate_probe(kind: int, iters: int, stream=None):

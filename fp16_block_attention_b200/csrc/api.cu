@@ -216,6 +216,74 @@ thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V
   return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, err, cs));
 }
 
+namespace {
+// Decode supports D = 128, blk = 128 and up to 16 query heads per kv head.
+thrift_status check_decode_shape(const thrift_shape* shape) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (shape->D != 128 || shape->blk != 128 || shape->Hq / shape->Hkv > 16) return THRIFT_ERR_UNSUPPORTED;
+  return THRIFT_OK;
+}
+}  // namespace
+
+thrift_status thrift_pool_keys(const void* K, const thrift_shape* shape, float* km, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!K || !km || !aligned16(K) || !aligned16(km)) return THRIFT_ERR_INVALID_ARG;
+  return from_cuda(launch_pool_keys(K, *shape, km, static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_decode_select(const void* q, const float* km, const thrift_shape* shape, double rho,
+                                   uint8_t* mask, void* stream) {
+  thrift_status st = check_decode_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!q || !km || !mask || !(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(km)) return THRIFT_ERR_INVALID_ARG;
+  return from_cuda(launch_decode_select(q, km, *shape, rho, mask, static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_decode_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
+  thrift_status st = check_decode_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!bytes) return THRIFT_ERR_INVALID_ARG;
+  *bytes = decode_workspace_bytes(*shape);
+  return THRIFT_OK;
+}
+
+thrift_status thrift_decode_attention(const void* q, const void* K, const void* V, const void* k4, const void* ks,
+                                      const void* v4, const void* vs, const uint8_t* mask, const thrift_shape* shape,
+                                      void* O, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = check_decode_shape(shape);
+  if (st != THRIFT_OK) return st;
+  const void* ptrs[] = {q, K, V, k4, ks, v4, vs, O};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return THRIFT_ERR_INVALID_ARG;
+  if (!mask) return THRIFT_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < decode_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  return from_cuda(launch_decode_attention(q, K, V, k4, ks, v4, vs, mask, *shape, O, decode_carve(ws, *shape), err,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_decode_step(const void* q, const void* K, const void* V, const void* k4, const void* ks,
+                                 const void* v4, const void* vs, const float* km, const thrift_shape* shape,
+                                 double rho, void* O, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = check_decode_shape(shape);
+  if (st != THRIFT_OK) return st;
+  const void* ptrs[] = {q, K, V, k4, ks, v4, vs, km, O};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return THRIFT_ERR_INVALID_ARG;
+  if (!(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < decode_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const DecodeWs w = decode_carve(ws, *shape);
+  if (launch_decode_select(q, km, *shape, rho, w.mask, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  return from_cuda(launch_decode_attention(q, K, V, k4, ks, v4, vs, w.mask, *shape, O, w, err, cs));
+}
+
 thrift_status thrift_last_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return THRIFT_ERR_CUDA;
   uint32_t* err = device_error_word();

@@ -48,6 +48,28 @@ constexpr int kMaxVWBlocks = 2048;
 cudaError_t launch_select_vertical_window(const void* Q, const void* K, const thrift_shape& s, double rho, int window,
                                           uint8_t* mask, void* ws, cudaStream_t st);
 
+// ---- decode (decode.cu) -----------------------------------------------------
+// Block means of K for the decode selection: km [B][Hkv][nb][D] FP32 (select.cu).
+cudaError_t launch_pool_keys(const void* K, const thrift_shape& s, float* km, cudaStream_t st);
+struct DecodePlan {
+  int tiles_per_cta;  // key tiles of one CTA (<= 6)
+  int chunks;         // CTAs per (batch, kv head)
+};
+DecodePlan decode_plan(const thrift_shape& s);
+struct DecodeWs {
+  uint8_t* mask;  // [B][Hq][nb] (thrift_decode_step)
+  float* part_o;  // [B][Hq][chunks][D]
+  float* part_l;  // [B][Hq][chunks]
+  float* part_m;  // [B][Hq][chunks]
+};
+size_t decode_workspace_bytes(const thrift_shape& s);
+DecodeWs decode_carve(void* ws, const thrift_shape& s);
+cudaError_t launch_decode_select(const void* q, const float* km, const thrift_shape& s, double rho, uint8_t* mask,
+                                 cudaStream_t st);
+cudaError_t launch_decode_attention(const void* q, const void* K, const void* V, const void* k4, const void* ks,
+                                    const void* v4, const void* vs, const uint8_t* mask, const thrift_shape& s,
+                                    void* O, const DecodeWs& w, uint32_t* err, cudaStream_t st);
+
 // Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
 cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);
 

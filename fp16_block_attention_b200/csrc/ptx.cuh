@@ -148,6 +148,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) 
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with A MN-major as well (bit 15): A stored with M contiguous.
+__host__ __device__ constexpr uint32_t idesc_f16_mn(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_f16(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
 // Instruction descriptor, .kind::mxf4nvf4.block_scale.scale_vec::4X with E2M1
 // A/B and UE4M3 scales (one per 16 elements along K, K = 64 per instruction).
 //   bits 4-5 B scale-factor id, 7-9 A format (1 = E2M1), 10-11 B format

@@ -288,6 +288,12 @@ void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s,
 }
 }  // namespace
 
+cudaError_t launch_pool_keys(const void* K, const thrift_shape& s, float* km, cudaStream_t st) {
+  const int nb = s.N / s.blk;
+  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, km);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select_vertical_window(const void* Q, const void* K, const thrift_shape& s, double rho, int window,
                                           uint8_t* mask, void* ws, cudaStream_t st) {
   const int nb = s.N / s.blk;

@@ -181,6 +181,52 @@ THRIFT_API thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape,
 THRIFT_API thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V, const thrift_shape* shape,
                                      double rho, void* O, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- decode: one new query row per (batch, query head) ----------------------
+ * One decode step over the caches that prefill leaves behind: the fp16 K and
+ * V and their NVFP4 copies from thrift_quantize_nvfp4.  The ThriftAttention
+ * pages describe prefill only; re-using the block-scaled FP4 K/V of prefill
+ * as a decode cache follows TriAttention (abstract on the paper page of
+ * arXiv 2611.07256).  Reading: the query row is its own query block and sits
+ * after the N cached keys, seeing all of them.
+ *   - shape: B, Hq, Hkv, D, blk, sm_scale as for prefill, N = cache length;
+ *     causal is ignored.  Decode calls other than thrift_pool_keys need
+ *     D = 128, blk = 128 and Hq / Hkv <= 16 (THRIFT_ERR_UNSUPPORTED).
+ *   - q: [B][Hq][D] fp16; O: [B][Hq][D] fp16; K, V: [B][Hkv][N][D] fp16;
+ *     k4/ks, v4/vs: thrift_quantize_nvfp4(K, THRIFT_K) and (V, THRIFT_V)
+ *     for the same shape.
+ *   - selection: score_j = fl32(sm_scale * fl32(q . kmean_j)) over the nb =
+ *     N/blk key blocks, kmean_j the FP32 block means of thrift_pool_keys (the
+ *     means of the prefill heuristic); k = ceil(rho * nb - 1e-9) blocks, the
+ *     first (j = 0) and the last (j = nb - 1) first, then by score, ties to
+ *     the lower j.
+ *   - attention: selected blocks in FP16, the others in NVFP4 (q encoded
+ *     along D like a row of Q), the prefill's online softmax (integer
+ *     maximum, P pre-scaled by 2^11, l over the unquantised P). */
+
+/* FP32 block means of K: km [B][Hkv][nb][D] (exact FP64 sums of the fp16
+ * rows, divided by blk, rounded once).  Any supported prefill shape. */
+THRIFT_API thrift_status thrift_pool_keys(const void* K, const thrift_shape* shape, float* km, void* stream);
+
+/* Decode selection: mask [B][Hq][nb] (u8, 1 = FP16 block). */
+THRIFT_API thrift_status thrift_decode_select(const void* q, const float* km, const thrift_shape* shape, double rho,
+                                              uint8_t* mask, void* stream);
+
+/* Workspace bytes of thrift_decode_attention and thrift_decode_step (the
+ * mask of thrift_decode_step and per-chunk partial results). */
+THRIFT_API thrift_status thrift_decode_workspace_bytes(const thrift_shape* shape, size_t* bytes);
+
+/* Decode attention with a given mask [B][Hq][nb] (1 = FP16 block). */
+THRIFT_API thrift_status thrift_decode_attention(const void* q, const void* K, const void* V, const void* k4,
+                                                 const void* ks, const void* v4, const void* vs, const uint8_t* mask,
+                                                 const thrift_shape* shape, void* O, void* ws, size_t ws_bytes,
+                                                 void* stream);
+
+/* Selection and attention in one call (km from thrift_pool_keys). */
+THRIFT_API thrift_status thrift_decode_step(const void* q, const void* K, const void* V, const void* k4,
+                                            const void* ks, const void* v4, const void* vs, const float* km,
+                                            const thrift_shape* shape, double rho, void* O, void* ws,
+                                            size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read and clear the device error word of the current
  * device: THRIFT_OK, or THRIFT_ERR_TIMEOUT if a kernel gave up a bounded wait
  * since the last call, or THRIFT_ERR_CUDA if the synchronisation failed. */

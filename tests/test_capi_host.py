@@ -89,3 +89,29 @@ def test_strerror_names_every_status():
     lib = thrift.lib()
     names = {lib.thrift_strerror(i).decode() for i in range(6)}
     assert len(names) == 6 and "ok" in names
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0), (dict(D=64), 2), (dict(blk=64), 2), (dict(Hq=32, Hkv=1), 2), (dict(Hq=16, Hkv=1), 0),
+])
+def test_decode_shape_validation(kw, status):
+    n = ctypes.c_size_t()
+    assert thrift.lib().thrift_decode_workspace_bytes(ctypes.byref(_c(**kw)), ctypes.byref(n)) == status
+    if status == 0:
+        assert n.value > 0
+
+
+def test_decode_arguments_are_rejected_before_launch():
+    lib = thrift.lib()
+    sh = ctypes.byref(_c())
+    fake = ctypes.c_void_p(256)
+    assert lib.thrift_pool_keys(None, sh, fake, None) == 1
+    assert lib.thrift_pool_keys(fake, sh, ctypes.c_void_p(260), None) == 1          # misaligned
+    assert lib.thrift_decode_select(fake, fake, sh, 1.5, fake, None) == 1
+    assert lib.thrift_decode_select(fake, None, sh, 0.05, fake, None) == 1
+    assert lib.thrift_decode_select(fake, fake, ctypes.byref(_c(D=64)), 0.05, fake, None) == 2
+    args = [fake] * 7
+    assert lib.thrift_decode_attention(*args, None, sh, fake, fake, 1 << 30, None) == 1  # no mask
+    assert lib.thrift_decode_attention(*args, fake, sh, fake, fake, 16, None) == 5       # workspace too small
+    assert lib.thrift_decode_step(*args, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1
+    assert lib.thrift_decode_step(*args, fake, sh, 0.05, fake, None, 0, None) == 5
