@@ -546,6 +546,72 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def decode_bytes(w, mask_np):
+    """Algorithmic HBM bytes of one decode attention call: the NVFP4 K and V
+    caches (codes and scales, 0.5625 B per element each), the fp16 K and V of
+    every key tile that some query head of its kv group keeps in FP16, q and O.
+    mask_np: [B, Hq, nb] decode mask (blk = 128 = one key tile)."""
+    G = w.Hq // w.Hkv
+    per_kv = mask_np.reshape(w.B, w.Hkv, G, -1).any(axis=2)  # [B, Hkv, nb]
+    fp4 = 2 * w.B * w.Hkv * w.N * w.D * 0.5625
+    fp16 = 2 * int(per_kv.sum()) * w.blk * w.D * 2
+    return fp4 + fp16 + 2 * w.B * w.Hq * w.D * 2
+
+
+def run_decode_sweep(args, dev, peaks):
+    """Decode step (selection + attention + combine) and the attention kernel
+    alone, per workload at its rho: ms with the L2 flushed before every call
+    (a 256 MB write outside the timed region), and achieved HBM bandwidth over
+    the algorithmic bytes of decode_bytes."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    print("| decode workload | rho | step ms | attention ms | algorithmic MB | attention GB/s | of measured HBM |")
+    print("|---|---:|---:|---:|---:|---:|---:|")
+    for w in [synth.GQA_N32K, synth.BATCHED_GQA_N16K, synth.GQA_N128K]:
+        Q, K, V = synth.generate(w)
+        q = torch.from_numpy(np.ascontiguousarray(Q[:, :, -1])).to(dev)
+        del Q
+        Kd, Vd = (torch.from_numpy(a).to(dev) for a in (K, V))
+        del K, V
+        sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+        km = thrift.pool_keys(Kd, sh)
+        kq = thrift.quantize_kv(Kd, Vd, sh)
+        ws = torch.empty(thrift.decode_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
+        mask = thrift.decode_select(q, km, sh, w.rho)
+
+        def timed(fn, n):
+            total = 0.0
+            for i in range(args.warmup + n):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if i >= args.warmup:
+                    total += e0.elapsed_time(e1)
+            return total / n
+
+        n = max(3, min(args.steps, 20))
+        step_ms = timed(lambda: thrift.decode_step(q, Kd, Vd, kq, km, sh, w.rho, out, ws, stream), n)
+        attn_ms = timed(lambda: thrift.decode_attention(q, Kd, Vd, kq, mask, sh, out, ws, stream), n)
+        if thrift.last_device_error(stream) != 0:
+            raise RuntimeError(f"a kernel reported a bounded-wait timeout in decode on {w.name}")
+        nbytes = decode_bytes(w, mask.cpu().numpy())
+        gbs = nbytes / (attn_ms * 1e-3) / 1e9
+        print(f"| {w.name} | {w.rho:g} | {step_ms:.4f} | {attn_ms:.4f} | {nbytes / 1e6:.1f} | {gbs:.0f} | "
+              f"{gbs / peaks['hbm_gbs']:.3f} |", flush=True)
+        del q, Kd, Vd, km, kq, ws, out, mask
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -557,11 +623,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time the attention kernel on every workload and rho (markdown table), then exit")
+    ap.add_argument("--decode-sweep", action="store_true",
+                    help="time the decode step on the GQA and batched caches (markdown table), then exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.sweep:
         run_sweep(args)
+    elif args.decode_sweep:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_decode_sweep(args, dev, load_peaks()[0])
     elif args.impl == "reference":
         run_reference(args)
     else:

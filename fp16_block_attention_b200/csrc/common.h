@@ -52,8 +52,9 @@ cudaError_t launch_select_vertical_window(const void* Q, const void* K, const th
 // Block means of K for the decode selection: km [B][Hkv][nb][D] FP32 (select.cu).
 cudaError_t launch_pool_keys(const void* K, const thrift_shape& s, float* km, cudaStream_t st);
 struct DecodePlan {
-  int tiles_per_cta;  // key tiles of one CTA (<= 6)
-  int chunks;         // CTAs per (batch, kv head)
+  int tiles_per_cta;  // key tiles of one chunk (<= 8)
+  int chunks;         // chunks per (batch, kv head)
+  int grid;           // persistent CTAs (at most one per SM)
 };
 DecodePlan decode_plan(const thrift_shape& s);
 struct DecodeWs {

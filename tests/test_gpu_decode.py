@@ -25,7 +25,8 @@ SMALL = [
     synth.BATCHED_GQA_N16K.with_(N=2048, B=2, Hq=14, Hkv=2),        # 7 heads per kv head, batched
     synth.CAUSAL_MH_N8K.with_(N=1536, Hq=2, Hkv=2, blk=128),        # one head per kv head
     synth.GQA_N32K.with_(N=896, Hq=16, Hkv=1),                      # 16 heads per kv head (the most)
-    synth.GQA_N32K.with_(N=3712, B=2, Hq=32, Hkv=16),               # 3-tile chunks, the last one ragged
+    synth.GQA_N32K.with_(N=3712, B=2, Hq=32, Hkv=16),               # many units, the last chunk ragged
+    synth.GQA_N32K.with_(N=4864, B=2, Hq=128, Hkv=8),               # 16 heads per kv head, two chunks per CTA
 ]
 FULL = [synth.GQA_N32K, synth.BATCHED_GQA_N16K, synth.GQA_N128K]
 
