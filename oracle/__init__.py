@@ -3,10 +3,11 @@
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It is plain C
 (``oracle.c``, FP64 arithmetic, OpenMP over rows) loaded with ctypes, plus the
-numpy modules ``vertical_window`` (the HyQuant-style selector) and ``decode``
-(one decode step over the prefill's caches), and it shares no code with the
-CUDA library.  See ``oracle.c`` and the two modules for what each function
-computes and which reading of the method it takes.
+numpy modules ``vertical_window`` (the HyQuant-style selector), ``tiered``
+(FP16 / NVFP4 / skip selection) and ``decode`` (one decode step over the
+prefill's caches), and it shares no code with the CUDA library.  See
+``oracle.c`` and the modules for what each function computes and which
+reading of the method it takes.
 """
 from __future__ import annotations
 
@@ -172,6 +173,21 @@ def select(Q, K, blk, causal, sm_scale, rho):
     if _load().orc_select(Q.ctypes.data, K.ctypes.data, B, Hq, Hkv, N, D, blk, int(causal),
                           float(sm_scale), float(rho), mask.ctypes.data):
         raise ValueError("orc_select rejected the shape")
+    return mask
+
+
+def select_tiered(Q, K, blk, causal, sm_scale, rho, sigma):
+    """Mask [B,Hq,nb,nb] (u8: 1 FP16, 0 NVFP4, 2 skip) of the tiered selection
+    (``tiered``) on the pooled scores of every (batch, query head)."""
+    from . import tiered
+    B, Hq = Q.shape[:2]
+    group = Hq // K.shape[1]
+    nb = Q.shape[2] // blk
+    mask = np.zeros((B, Hq, nb, nb), np.uint8)
+    for b in range(B):
+        for h in range(Hq):
+            sc = pooled_scores(Q[b, h], K[b, h // group], blk, causal, sm_scale)
+            mask[b, h] = tiered.select_head(sc, causal, rho, sigma, budget)
     return mask
 
 

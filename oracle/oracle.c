@@ -29,6 +29,9 @@
  *   - Online softmax with an integer running maximum M = ceil(max t), t the
  *     log2-domain logit; rescales are exact powers of two.
  *   - l sums the unquantised P; quantisation only encodes the P.V operand.
+ *   - A mask value of 2 marks a skipped pair, absent from the softmax (the
+ *     skip precision of TriAttention's tile assignment, abstract on the paper
+ *     page of arXiv 2611.07256); 1 is FP16, 0 NVFP4.
  * All arithmetic is FP64 with FP32/FP16/FP4 rounding at the points the
  * readings name.
  */
@@ -375,7 +378,11 @@ static void attention_row(const orc_problem* p, const uint8_t* mask, int b, int 
     for (int oi = 0; oi < nb; ++oi) {
         int j = order ? order[oi] : oi;
         if (p->causal && j > qb) continue;
-        int fp16 = mask[(((long)b * p->Hq + h) * nb + qb) * nb + j] != 0;
+        /* mask: 1 = FP16 pair, 0 = NVFP4 pair, 2 = skipped pair (absent from
+         * the softmax: the skip precision of TriAttention's tile assignment) */
+        uint8_t cls = mask[(((long)b * p->Hq + h) * nb + qb) * nb + j];
+        if (cls == 2) continue;
+        int fp16 = cls == 1;
         float tmax = -INFINITY;
         for (int i = 0; i < blk; ++i) {
             int k = j * blk + i;
