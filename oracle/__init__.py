@@ -31,7 +31,7 @@ class Problem(ctypes.Structure):
         ("v4", ctypes.c_void_p), ("vs", ctypes.c_void_p),
         ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("N", ctypes.c_int),
         ("D", ctypes.c_int), ("blk", ctypes.c_int), ("causal", ctypes.c_int),
-        ("sm_scale", ctypes.c_float), ("p_log2", ctypes.c_int),
+        ("sm_scale", ctypes.c_float), ("p_log2", ctypes.c_int), ("p_jitter", ctypes.c_double),
     ]
 
 
@@ -216,7 +216,7 @@ class Quantised:
         self.v4, self.vs = quantize_v(V)
 
 
-def _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep):
+def _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep, p_jitter=0.0):
     Q, K, V = _bits16(Q), _bits16(K), _bits16(V)
     keep.extend([Q, K, V])
     B, Hq, N, D = Q.shape
@@ -227,17 +227,18 @@ def _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep):
         keep.extend(arrs)
         ptrs = [a.ctypes.data for a in arrs]
     return Problem(Q.ctypes.data, K.ctypes.data, V.ctypes.data, *ptrs, B, Hq, Hkv, N, D, blk,
-                   int(causal), float(sm_scale), int(p_log2))
+                   int(causal), float(sm_scale), int(p_log2), float(p_jitter))
 
 
 def attention_rows(Q, K, V, mask, rows, blk, causal, sm_scale, qz=None, order=None,
-                   p_log2=P_LOG2_DEFAULT):
+                   p_log2=P_LOG2_DEFAULT, p_jitter=0.0):
     """Mixed-precision attention output (float64, before fp16 rounding) for rows
-    [(b, h, r), ...] -> [nrows, D]."""
+    [(b, h, r), ...] -> [nrows, D].  p_jitter (tests only): encode P * (1 +
+    p_jitter) instead of P, to resolve E2M1 / fp16 rounding ties the other way."""
     keep = []
     if qz is None:
         qz = Quantised(Q, K, V)
-    p = _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep)
+    p = _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep, p_jitter)
     rows = _c(np.asarray(rows, np.int64).reshape(-1, 3))
     mask = _c(np.asarray(mask, np.uint8))
     out = np.empty((rows.shape[0], p.D), np.float64)

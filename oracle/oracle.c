@@ -312,6 +312,7 @@ typedef struct {
     int B, Hq, Hkv, N, D, blk, causal;
     float sm_scale;
     int p_log2;                                /* pre-scale exponent c of P */
+    double p_jitter;                           /* 0, or a relative change of the encoded P (below) */
 } orc_problem;
 
 /* log2-domain logit: t = fl32(fl32(S) * fl32(sm_scale * log2 e)). */
@@ -401,7 +402,16 @@ static void attention_row(const orc_problem* p, const uint8_t* mask, int b, int 
             P[i] = (t[i] == -INFINITY) ? 0.0 : (double)(float)exp2((double)t[i] - M);
             l += P[i];
         }
-        encode_p(P, blk, fp16, p->p_log2, Pt);
+        /* p_jitter (test use): the encoded P is taken as P * (1 + p_jitter),
+         * l keeps the exact P.  The pages fix no accuracy for exp2, so a P
+         * within a few ulps of an E2M1 or fp16 rounding boundary may be
+         * encoded either way; parity tests re-check a row that misses the
+         * bar against the oracle with P nudged both ways. */
+        if (p->p_jitter != 0.0)
+            for (int i = 0; i < blk; ++i) Pt[i] = P[i] * (1.0 + p->p_jitter);
+        else
+            memcpy(Pt, P, sizeof(double) * blk);
+        encode_p(Pt, blk, fp16, p->p_log2, Pt);
         for (int i = 0; i < blk; ++i) {
             if (Pt[i] == 0.0) continue;
             int k = j * blk + i;

@@ -413,3 +413,22 @@ def test_gap_recovered_closed_forms():
 def test_to_f16_matches_numpy():
     x = np.random.default_rng(12).standard_normal(1000) * 3
     assert np.array_equal(oracle.to_f16(x), x.astype(np.float16))
+
+
+def test_p_jitter_only_moves_rows_at_rounding_ties():
+    """The test-only nudge of the encoded P: zero leaves every output as it
+    was; 2^-19 (relative) only flips codes of P within that distance of an
+    E2M1 / fp16 rounding boundary, so outputs move by tiny amounts (fp16
+    boundaries are dense) and almost no row moves by more than 1e-3."""
+    w, Q, K, V = _small(synth.CAUSAL_MH_N8K, N=512, Hq=2, Hkv=2)
+    rows = oracle.all_rows(w.B, w.Hq, w.N)
+    mask = oracle.select(Q, K, w.blk, w.causal, w.sm_scale, 0.1)
+    qz = oracle.Quantised(Q, K, V)
+    base = oracle.attention_rows(Q, K, V, mask, rows, w.blk, w.causal, w.sm_scale, qz)
+    same = oracle.attention_rows(Q, K, V, mask, rows, w.blk, w.causal, w.sm_scale, qz, p_jitter=0.0)
+    assert np.array_equal(base, same)
+    for j in (2.0 ** -19, -(2.0 ** -19)):
+        nudged = oracle.attention_rows(Q, K, V, mask, rows, w.blk, w.causal, w.sm_scale, qz, p_jitter=j)
+        moved = np.abs(nudged - base).max(axis=1) > 1e-3
+        assert moved.mean() < 0.01
+        assert np.abs(nudged - base).mean() < 1e-5
