@@ -75,6 +75,7 @@ def _load():
         "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_select_blocks_static": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
         "thrift_select_blocks_vertical_window": ([vp, vp, psh, ctypes.c_double, st, vp, vp, sz, vp], st),
+        "thrift_select_blocks_tiered": ([vp, vp, psh, ctypes.c_double, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
@@ -98,7 +99,8 @@ _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
-           "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_attention",
+           "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_select_blocks_tiered",
+           "thrift_attention",
            "thrift_fused_workspace_bytes",
            "thrift_attention_fused", "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
            "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error", "thrift_mma_rate_probe",
@@ -178,6 +180,22 @@ def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, 
     _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
                                                              float(rho), _ptr(mask), _ptr(ws), ws.numel(),
                                                              _stream(stream)))
+    return mask
+
+
+def select_blocks_tiered(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, sigma: float, mask=None,
+                         ws=None, stream=None):
+    """Tiered selection mask [B, Hq, nb, nb] (u8): 1 FP16, 0 NVFP4, 2 skipped
+    (the lowest-ranked pairs, never forced or FP16 ones)."""
+    _dev(Qt, "Q", torch.float16)
+    _dev(Kt, "K", torch.float16)
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
+    if ws is None:
+        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_select_blocks_tiered", _lib.thrift_select_blocks_tiered(
+        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), float(sigma), _ptr(mask), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return mask
 
 

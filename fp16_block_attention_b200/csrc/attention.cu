@@ -100,7 +100,8 @@ struct Misc {
   volatile int abort;
   float red_max[2][kSplit][128];
   float red_l[kSplit][128];
-  uint8_t cls[1024];  // per key tile: bit (a*2 + c) = FP16 flag of block (query half a, key half c)
+  uint8_t cls[1024];  // per key tile: bit (a*2 + c) = FP16 flag, bit 4 + (a*2 + c) = skip flag of block
+                      // (query half a, key half c)
 };
 
 static_assert(sizeof(Misc) <= 8192, "barriers and exchange buffers must fit their shared-memory slice");
@@ -151,15 +152,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // precision class of every key tile of this query tile
   const uint8_t* mrow = p.mask + static_cast<size_t>(bh) * nb * nb;
+  // (mask 1 FP16, 0 NVFP4, 2 skipped: a skipped block is computed like an
+  // NVFP4 one and then masked out of the softmax)
   for (int kt = tid; kt < n_kt; kt += kThreads) {
     uint32_t c = 0;
     if (p.blk == 128) {
-      c = mrow[static_cast<size_t>(qt) * nb + kt] ? 0xFu : 0u;
+      const uint8_t mv = mrow[static_cast<size_t>(qt) * nb + kt];
+      c = (mv == 1 ? 0xFu : 0u) | (mv == 2 ? 0xF0u : 0u);
     } else {
       for (int a = 0; a < 2; ++a)
         for (int k = 0; k < 2; ++k) {
           const int i = 2 * qt + a, j = 2 * kt + k;
-          if (i < nb && j < nb && mrow[static_cast<size_t>(i) * nb + j]) c |= 1u << (a * 2 + k);
+          const uint8_t mv = (i < nb && j < nb) ? mrow[static_cast<size_t>(i) * nb + j] : 0;
+          if (mv == 1) c |= 1u << (a * 2 + k);
+          if (mv == 2) c |= 1u << (4 + a * 2 + k);
         }
     }
     ms.cls[kt] = static_cast<uint8_t>(c);
@@ -183,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 &ms.bar_q);
       int u4 = 0, u16 = 0, u16k_only = 0;
       for (int kt = 0; kt < n_kt && !ms.abort; ++kt) {
-        const uint32_t c = ms.cls[kt];
+        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
           if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t o_acc = 0;
       // issue S of tile kt (its loads are complete)
       auto issue_s = [&](int kt) {
-        const uint32_t c = ms.cls[kt];
+        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
         const uint32_t sfset = tm + kColSF + 24 * (kt & 1);
         if (c != 0u) {
           const uint32_t k16 = sbase + L::kSlot16;
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // wait for the loads of tile kt; records its FP4 slot
       auto wait_loads = [&](int kt) -> bool {
-        const uint32_t c = ms.cls[kt];
+        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
           if (!wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
@@ -292,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!wait_or_abort(&ms.bar_p_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) break;
         tc_fence_after();
-        const uint32_t c = ms.cls[kt];
+        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
         const uint32_t sfset = tm + kColSF + 24 * (kt & 1);
         const int slot4 = slot4_of[kt & 1];
         if (c != 0xFu) {
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float M = -INFINITY, l = 0.f;
     bool failed = false;  // this thread gave up a wait; the exit is taken jointly
     for (int kt = 0; kt < n_kt; ++kt) {
-      const uint32_t c = ms.cls[kt];
+      const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
       const bool fp16 = (c >> (a * 2 + kh)) & 1u;
       const bool need16 = c != 0u, need4 = c != 0xFu;
       if (!failed) failed = !wait_or_abort(&ms.bar_s_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
@@ -370,6 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < kKPT; ++j) s[j] = -INFINITY;
       }
 
+      // A skipped block leaves the softmax: all of this thread's keys.
+      if ((ms.cls[kt] >> (4 + a * 2 + kh)) & 1u) {
+#pragma unroll
+        for (int j = 0; j < kKPT; ++j) s[j] = -INFINITY;
+      }
       // Mask keys past N and, on the diagonal tile, keys after the query.
       const int key0 = kt * 128 + koff;
       if (kt * 128 + 128 > p.N || (p.causal && kt == qt)) {

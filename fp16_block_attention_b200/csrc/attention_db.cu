@@ -93,7 +93,8 @@ struct MiscDB {
   uint32_t tmem;
   volatile int abort;
   float lsum[2][128];  // partial row sums of the two halves, for the epilogue
-  uint8_t cls[1024];    // per key tile: 1 = FP16, 0 = NVFP4
+  uint16_t lst[1024];   // key tiles to process, in order: tile index, bit 15 set = FP16
+  int np;               // their number (skipped tiles are left out)
 };
 static_assert(sizeof(MiscDB) <= 4096, "barriers must fit their shared-memory slice");
 
@@ -142,14 +143,26 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     ms.abort = 0;
     fence_mbar_init();
   }
-  {
+  if (warp == 0) {
+    // Key tiles to process in increasing order: mask 1 FP16, 0 NVFP4, 2 skipped
+    // (left out of the list, so no role spends anything on them).
     const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
-    for (int kt = tid; kt < nk; kt += kDBThreads) ms.cls[kt] = m0[kt] ? 1 : 0;
+    int base = 0;
+    for (int k0 = 0; k0 < nk; k0 += 32) {
+      const int kt = k0 + lane;
+      const uint8_t mv = kt < nk ? m0[kt] : 2;
+      const uint32_t keep = __ballot_sync(0xffffffffu, mv != 2);
+      if (mv != 2)
+        ms.lst[base + __popc(keep & ((1u << lane) - 1u))] = static_cast<uint16_t>(kt | (mv == 1 ? 0x8000 : 0));
+      base += __popc(keep);
+    }
+    if (lane == 0) ms.np = base;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ms.tmem;
+  const int np = ms.np;
 
   if (warp == kDBProducer) {
     // ======================== producer ========================
@@ -163,8 +176,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       tma_load_3d(sm + L::kQ4, &mQ4, &ms.bar_q, 0, qt * 128, bh);
       bulk_load(sm + L::kQSF, p.qs + (static_cast<size_t>(bh) * p.NT + qt) * L::kQSFBytes, L::kQSFBytes, &ms.bar_q);
       int u4 = 0, u16 = 0;
-      for (int kt = 0; kt < nk && !ms.abort; ++kt) {
-        if (ms.cls[kt] == 0) {
+      for (int it = 0; it < np && !ms.abort; ++it) {
+        const int kt = ms.lst[it] & 0x3FF;
+        if (!(ms.lst[it] & 0x8000)) {
           const int slot = u4 % L::kNS, use = u4 / L::kNS;
           if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
@@ -215,9 +229,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         for (int c = 0; c < D / 64; ++c)
           tmem_cp_32x128b_x4(tm + kDColSFQ + 4 * c, make_sdesc(sbase + L::kQSF + 512 * c, 16, 128, LAYOUT_NONE));
       int u4 = 0, uk16 = 0;
-      for (int kt = 0; ok && kt < nk; ++kt) {
-        const int bb = kt & 1;
-        const bool fp16 = ms.cls[kt] != 0;
+      for (int it = 0; ok && it < np; ++it) {
+        const int bb = it & 1;
+        const bool fp16 = (ms.lst[it] & 0x8000) != 0;
         int slot = 0;
         if (!fp16) {
           slot = u4 % L::kNS;
@@ -235,11 +249,12 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         // Buffers bb were last used by key tile kt - 2: wait until its S was
         // loaded by the softmax threads, and until its P V product is done, so
         // that the softmax threads, once they see S(kt), may overwrite P buffer
-        // bb and its scales without waiting themselves.
-        if (kt >= 2) {
-          if (!(ok = wait_or_abort(&ms.bar_s_free[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
+        // bb and its scales without waiting themselves.  (Buffers and phases
+        // count processed tiles, it, not tile indices.)
+        if (it >= 2) {
+          if (!(ok = wait_or_abort(&ms.bar_s_free[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
             break;
-          if (!(ok = wait_or_abort(&ms.bar_o_done[bb], ((kt - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA)))
+          if (!(ok = wait_or_abort(&ms.bar_o_done[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA)))
             break;
           tc_fence_after();
         }
@@ -278,9 +293,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       bool ok = true;
       int u4 = 0, uv16 = 0;
       uint32_t acc = 0u;
-      for (int kt = 0; ok && kt < nk; ++kt) {
-        const int bb = kt & 1;
-        const bool fp16 = ms.cls[kt] != 0;
+      for (int it = 0; ok && it < np; ++it) {
+        const int bb = it & 1;
+        const bool fp16 = (ms.lst[it] & 0x8000) != 0;
         // The V operands (and the V4 scales, copied to tensor memory) do not
         // depend on P, so they are made ready before waiting for it.  The copy
         // follows the previous P V product in this thread's tcgen05 order, so
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uv16;
         }
-        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
         tc_fence_after();
         const uint32_t dO = tm + kDColO;
         if (!fp16) {
@@ -353,10 +368,11 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     const auto turn_in = [&] { named_bar_sync(2 + half, kDBSoftmax); };
     const auto turn_out = [&] { named_bar_arrive(3 - half, kDBSoftmax); };
     if (half == 1) named_bar_arrive(2, kDBSoftmax);  // half 0 goes first
-    for (int kt = 0; kt < nk; ++kt) {
-      const int bb = kt & 1;
-      const bool fp16 = ms.cls[kt] != 0;
-      if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (kt >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+    for (int it = 0; it < np; ++it) {
+      const int bb = it & 1;
+      const int kt = ms.lst[it] & 0x3FF;
+      const bool fp16 = (ms.lst[it] & 0x8000) != 0;
+      if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) {
         turn_in();
@@ -431,8 +447,8 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // product of key tile kt - 2 before issuing S(kt).  The fp16 P columns
       // are single-buffered, so an fp16 tile waits for the previous key tile's
       // product.
-      if (fp16 && kt >= 1) {
-        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (fp16 && it >= 1) {
+        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
         failed = __any_sync(0xffffffffu, failed);
         if (failed) {
           turn_in();
@@ -489,8 +505,8 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // Rescale this thread's half of O when the maximum grew (rows with alpha
       // = 1 are unchanged); O is stable once the previous key tile's P V
       // product is done.
-      if (kt > 0 && __any_sync(0xffffffffu, Mn > M)) {
-        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((kt - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (it > 0 && __any_sync(0xffffffffu, Mn > M)) {
+        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
         failed = __any_sync(0xffffffffu, failed);
         if (failed) continue;
         tc_fence_after();
@@ -520,9 +536,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     if (half == 0) turn_in();  // the turn half 1 passed after its last key tile
 
     // ---- epilogue: O / l -> fp16 (both carry the 2^11 pre-scale) ----
-    if (nk > 0) {
+    if (np > 0) {
       if (!failed)
-        failed = !wait_or_abort(&ms.bar_o_done[(nk - 1) & 1], ((nk - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = !wait_or_abort(&ms.bar_o_done[(np - 1) & 1], ((np - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       ms.lsum[half][r] = l;
       // every softmax thread takes the same exit decision (and sees lsum)
       failed = softmax_bar_or<kDBSoftmax>(failed);

@@ -184,9 +184,12 @@ __global__ void __launch_bounds__(1024) column_rank_kernel(const float* __restri
 
 // One CTA (1024 threads) per (batch, query head).  VW = 0: the method's key;
 // VW = 1: the vertical-line / local-window key (column ranks in `rank`).
+// The first k pairs by key are marked 1; with keep < #valid the pairs after
+// the first `keep` are marked 2 (skipped; the caller keeps them clear of
+// forced and FP16 pairs), the rest 0.
 template <int VW>
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int nb, int causal,
-                                                    long long k, uint8_t* __restrict__ mask,
+                                                    long long k, long long keep, uint8_t* __restrict__ mask,
                                                     const int* __restrict__ rank, int window) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
@@ -207,16 +210,13 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
   const size_t total = static_cast<size_t>(nb) * nb;
   const long long valid = causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(total);
 
-  uint64_t threshold;  // select keys >= threshold
-  bool select_none = (k <= 0);
-  if (k >= valid) {
-    threshold = 0;  // every valid pair
-  } else if (select_none) {
-    threshold = ~0ull;
-  } else {
+  // Key of the kk-th largest valid pair (1 <= kk < valid) by an 8-bit radix
+  // select: the first kk pairs are exactly those with key >= the result.
+  const auto kth_largest = [&](long long kk) -> uint64_t {
+    __syncthreads();  // every thread has read the previous result
     if (threadIdx.x == 0) {
       s_prefix = 0;
-      s_remaining = k;
+      s_remaining = kk;
       s_done = 0;
     }
     uint64_t pmask = 0;
@@ -250,12 +250,23 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
       pmask |= 255ull << shift;
       if (s_done) break;
     }
-    threshold = s_prefix;
-  }
+    return s_prefix;
+  };
+
+  const bool select_none = k <= 0, select_all = k >= valid;
+  const uint64_t threshold = (select_none || select_all) ? 0ull : kth_largest(k);  // FP16: key >= threshold
+  const bool skip_any = keep < valid;
+  const uint64_t keep_from = (skip_any && keep > 0) ? kth_largest(keep) : 0ull;  // skipped: key < keep_from
   for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
     const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
     uint8_t v = 0;
-    if (!(causal && j > i) && !select_none) v = key_of(sc[idx], i, j) >= threshold ? 1 : 0;
+    if (!(causal && j > i)) {
+      const uint64_t key = key_of(sc[idx], i, j);
+      if (!select_none && (select_all || key >= threshold))
+        v = 1;
+      else if (skip_any && (keep <= 0 || key < keep_from))
+        v = 2;
+    }
     m[idx] = v;
   }
 }
@@ -269,9 +280,13 @@ size_t select_workspace_bytes(const thrift_shape& s) {
 }
 
 namespace {
+long long valid_pairs(const thrift_shape& s) {
+  const long long nb = s.N / s.blk;
+  return s.causal ? nb * (nb + 1) / 2 : nb * nb;
+}
+
 long long budget_pairs(const thrift_shape& s, double rho) {
-  const int nb = s.N / s.blk;
-  const long long valid = s.causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
+  const long long valid = valid_pairs(s);
   double kk = ceil(rho * static_cast<double>(valid) - 1e-9);
   if (kk < 0) kk = 0;
   if (kk > static_cast<double>(valid)) kk = static_cast<double>(valid);
@@ -300,7 +315,8 @@ cudaError_t launch_select_vertical_window(const void* Q, const void* K, const th
   SelectWs w = carve(ws, s);
   launch_pool_and_scores(Q, K, s, w, st);
   column_rank_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, w.rank);
-  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), mask, w.rank, window);
+  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), valid_pairs(s), mask,
+                                               w.rank, window);
   return cudaGetLastError();
 }
 
@@ -309,7 +325,24 @@ cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, d
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
   launch_pool_and_scores(Q, K, s, w, st);
-  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), mask, nullptr, 0);
+  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), valid_pairs(s), mask,
+                                               nullptr, 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double sigma,
+                                 uint8_t* mask, void* ws, cudaStream_t st) {
+  const int nb = s.N / s.blk;
+  SelectWs w = carve(ws, s);
+  launch_pool_and_scores(Q, K, s, w, st);
+  // skipped pairs: the last ks of the ranking, clear of the forced and FP16 pairs
+  const long long n = valid_pairs(s), k16 = budget_pairs(s, rho);
+  const long long forced = 2LL * nb - 1;  // the diagonal and key block 0, (0, 0) once
+  long long ks = budget_pairs(s, sigma);
+  const long long cap = n - (k16 > forced ? k16 : forced);
+  if (ks > cap) ks = cap;
+  if (ks < 0) ks = 0;
+  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k16, n - ks, mask, nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -117,6 +117,23 @@ THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape
 THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
                                    uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
 
+/* Stage 1 with a third class, skipped pairs, after TriAttention's tile
+ * precisions (abstract on the paper page of arXiv 2611.07256: interactions
+ * that matter least are skipped, the precision of the rest lowered).  The
+ * method's ranking (as thrift_select_blocks) is cut in three per (batch,
+ * query head):
+ *   the first k16 = ceil(rho * #valid - 1e-9) pairs          -> 1 (FP16)
+ *   the last  ks  = min(ceil(sigma * #valid - 1e-9),
+ *                       #valid - max(k16, 2 nb - 1)) pairs   -> 2 (skipped)
+ *   the others                                               -> 0 (NVFP4)
+ * so the forced pairs (diagonal and key block 0, 2 nb - 1 of them) and the
+ * FP16 pairs are never skipped; sigma = 0 gives thrift_select_blocks' mask.
+ * thrift_attention treats a skipped pair as absent from the softmax.
+ * Workspace, layout and errors as for thrift_select_blocks. */
+THRIFT_API thrift_status thrift_select_blocks_tiered(const void* Q, const void* K, const thrift_shape* shape,
+                                                     double rho, double sigma, uint8_t* mask, void* ws,
+                                                     size_t ws_bytes, void* stream);
+
 /* An alternative stage 1 on the same FP16 budget, after HyQuant (abstract in
  * the body of the page titled "LampAttention: Look-Ahead Mixed-Precision
  * FlashAttention for Dedicated Accelerators"): HyQuant keeps full precision
@@ -166,7 +183,9 @@ THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* 
 
 /* Stage 2 (ThriftAttention abstract: picked pairs in FP16, the others in
  * FP4, one online softmax merging both): O [B][Hq][N][D] fp16.
- * mask: as written by thrift_select_blocks; q4/qs, k4/ks, v4/vs: the NVFP4
+ * mask: as written by thrift_select_blocks (1 FP16, 0 NVFP4), or by
+ * thrift_select_blocks_tiered (2: skipped, absent from the softmax; every
+ * query block must keep at least one pair); q4/qs, k4/ks, v4/vs: the NVFP4
  * copies written by thrift_quantize_nvfp4 for Q, K and V. */
 THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,

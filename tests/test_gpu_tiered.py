@@ -1,0 +1,91 @@
+"""Parity of the tiered selection (FP16 / NVFP4 / skip) and of attention with
+skipped pairs on the GPU (through the C ABI) with the oracle.
+
+Selection: exactly k16 FP16 pairs and ks skipped pairs per head; the masks
+agree except for pairs whose pooled score lies within 1e-5 (relative) of one
+of the two cuts (the lowest FP16 score of a non-forced pair, the highest
+skipped score), where FP32 summation order may swap neighbours.  Attention:
+the oracle's mask given to the GPU, outputs within max-abs 2e-2 and mean-abs
+1e-3 of the oracle's (the prefill bars), where a row that misses the bar is
+re-checked against the oracle with its encoded P nudged by 2^-19 both ways
+(rounding ties of P, which skipping makes visible by concentrating a row's
+weight on few NVFP4 keys; at most one row in a thousand); blk 128 leaves
+skipped tiles out of every role's work, blk 64 masks skipped blocks inside a
+128-key tile.
+"""
+import numpy as np
+import pytest
+
+import fp16_block_attention_b200 as thrift
+import oracle
+import synth
+from gpu_helpers import ATOL_MAX, ATOL_MEAN, compare_o_with_ties, shape_of, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    synth.TINY_NONCAUSAL_D64,                                         # blk 64, non-causal
+    synth.CAUSAL_MH_N8K.with_(N=1536, Hq=2, Hkv=2),                   # blk 64, causal
+    synth.GQA_N32K.with_(N=2048, Hq=4, Hkv=2),                        # blk 128, GQA
+    synth.BATCHED_GQA_N16K.with_(N=1280, B=2, Hq=4, Hkv=2),           # blk 128, batched, ragged tail
+]
+IDS = [f"{w.name}-N{w.N}-B{w.B}-H{w.Hq}x{w.Hkv}-blk{w.blk}" for w in CASES]
+
+
+def _valid(nb, causal):
+    return np.tril(np.ones((nb, nb), bool)) if causal else np.ones((nb, nb), bool)
+
+
+@pytest.mark.parametrize("rho,sigma", [(0.05, 0.25), (0.0, 0.6), (0.3, 0.5), (0.05, 1.0)])
+@pytest.mark.parametrize("w", CASES, ids=IDS)
+def test_tiered_select_matches_oracle(w, rho, sigma):
+    Q, K, _ = synth.generate(w)
+    Qd, Kd = to_dev(Q, K)
+    m = thrift.select_blocks_tiered(Qd, Kd, shape_of(w), rho, sigma).cpu().numpy()
+    ref = oracle.select_tiered(Q, K, w.blk, w.causal, w.sm_scale, rho, sigma)
+    nb = w.N // w.blk
+    valid = _valid(nb, w.causal)
+    forced = np.zeros((nb, nb), bool)
+    forced[np.arange(nb), np.arange(nb)] = True
+    forced[:, 0] = True
+    G = w.Hq // w.Hkv
+    for b in range(w.B):
+        for h in range(w.Hq):
+            mg, mo = m[b, h], ref[b, h]
+            assert (mg == 1).sum() == (mo == 1).sum() and (mg == 2).sum() == (mo == 2).sum()
+            assert not np.any((mg == 2) & forced) and not np.any((mg != 0) & ~valid)
+            diff = mg != mo
+            if not diff.any():
+                continue
+            sc = oracle.pooled_scores(Q[b, h], K[b, h // G], w.blk, w.causal, w.sm_scale)
+            cuts = []
+            if np.any((mo == 1) & ~forced):
+                cuts.append(sc[(mo == 1) & ~forced].min())
+            if np.any(mo == 2):
+                cuts.append(sc[mo == 2].max())
+            near = np.zeros_like(diff)
+            for c in cuts:
+                near |= np.abs(sc - c) <= 1e-5 * max(abs(c), 1e-30)
+            assert np.all(near[diff]), (b, h)
+
+
+@pytest.mark.parametrize("rho,sigma", [(0.05, 0.25), (0.0, 0.6), (0.3, 0.9)])
+@pytest.mark.parametrize("w", CASES, ids=IDS)
+def test_attention_with_skipped_pairs_matches_oracle(w, rho, sigma):
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    sh = shape_of(w)
+    m = oracle.select_tiered(Q, K, w.blk, w.causal, w.sm_scale, rho, sigma)
+    assert (m == 2).any()
+    md, = to_dev(m)
+    qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+    o = thrift.attention(Qd, Kd, Vd, md, qz, sh)
+    assert thrift.last_device_error() == 0
+    o = o.cpu().numpy()
+    rows = oracle.all_rows(w.B, w.Hq, w.N)
+    if rows.shape[0] > 8192:
+        rows = rows[np.random.default_rng(2).choice(rows.shape[0], 8192, replace=False)]
+    mx, mean, resolved = compare_o_with_ties(o[rows[:, 0], rows[:, 1], rows[:, 2]], Q, K, V, m, rows, w.blk,
+                                             w.causal, w.sm_scale)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
+    assert resolved <= max(1, rows.shape[0] // 1000), resolved  # ties are rare
