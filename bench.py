@@ -155,7 +155,8 @@ class ClockSampler:
 
 def flop_split(w, mask_np):
     """Effective FLOPs of the FP16 and FP4 block pairs (diagonal pairs count their
-    causal triangle), from the selection mask [B, Hq, nb, nb]."""
+    causal triangle), from the selection mask [B, Hq, nb, nb] (1 FP16, 0 NVFP4,
+    2 skipped: not computed, counted in neither)."""
     nb = w.N // w.blk
     full = 4.0 * w.blk * w.blk * w.D
     diag = 4.0 * w.D * w.blk * (w.blk + 1) / 2 if w.causal else full
@@ -163,8 +164,8 @@ def flop_split(w, mask_np):
     valid = np.tril(np.ones((nb, nb), bool)) if w.causal else np.ones((nb, nb), bool)
     weight = np.where(eye, diag, full) * valid
     f16 = float((weight[None, None] * (mask_np == 1)).sum())
-    total = float(weight.sum()) * w.B * w.Hq
-    return f16, total - f16
+    f4 = float((weight[None, None] * (mask_np == 0)).sum())
+    return f16, f4
 
 
 MUFU_PER_CLK_PER_SM = 16  # ex2 / lg2 throughput of compute capability 10.0 (16 per clock per SM)
@@ -544,6 +545,54 @@ def run_sweep(args):
               f"{t_bound * 1e3 / ms:.4f} | {mufu['frac']:.4f} |", flush=True)
         del Qd, Kd, Vd, Od, qz, mask
         torch.cuda.empty_cache()
+    print()
+    run_skip_sweep(args, dev, peaks, n_sm)
+
+
+def run_skip_sweep(args, dev, peaks, n_sm):
+    """Skipped block pairs (tiered selection) on the 32k GQA workload at rho =
+    5%: attention ms, dense-equivalent TFLOP/s (the full causal FLOPs over the
+    time), the TFLOP/s of the pairs computed, and the blended roofline and
+    MUFU fractions over the computed pairs."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    p16 = peaks["bf16_tflops"] * 1e12
+    p4 = FP4_OVER_BF16 * p16
+    w = synth.GQA_N32K
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+    sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+    qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+    Od = torch.empty_like(Qd)
+    stream = torch.cuda.current_stream(dev)
+    print(f"| skipped share sigma ({w.name}, rho {w.rho:g}) | attention ms | dense-equivalent TFLOP/s | "
+          "computed TFLOP/s | roofline frac (computed) | MUFU frac |")
+    print("|---:|---:|---:|---:|---:|---:|")
+    for sigma in (0.0, 0.25, 0.5, 0.75):
+        mask = thrift.select_blocks_tiered(Qd, Kd, sh, w.rho, sigma)
+        for _ in range(args.warmup):
+            thrift.attention_tiered(Qd, Kd, Vd, mask, qz, sh, Od, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(2, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n):
+            thrift.attention_tiered(Qd, Kd, Vd, mask, qz, sh, Od, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if thrift.last_device_error(stream) != 0:
+            raise RuntimeError("a kernel reported a bounded-wait timeout in the skip sweep")
+        ms = e0.elapsed_time(e1) / n
+        m = mask.cpu().numpy()
+        f16, f4 = flop_split(w, m)
+        t_bound = max(f16 / p16 + f4 / p4, attention_bytes(w, m) / (peaks["hbm_gbs"] * 1e9))
+        mufu = mufu_ceiling(w, m, ms, 1965.0, n_sm)
+        print(f"| {sigma:g} | {ms:.4f} | {w.flops() / (ms * 1e-3) / 1e12:.1f} | "
+              f"{(f16 + f4) / (ms * 1e-3) / 1e12:.1f} | {t_bound * 1e3 / ms:.4f} | {mufu['frac']:.4f} |", flush=True)
+    del Qd, Kd, Vd, Od, qz
+    torch.cuda.empty_cache()
 
 
 def decode_bytes(w, mask_np):

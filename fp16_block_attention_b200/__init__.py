@@ -77,6 +77,7 @@ def _load():
         "thrift_select_blocks_vertical_window": ([vp, vp, psh, ctypes.c_double, st, vp, vp, sz, vp], st),
         "thrift_select_blocks_tiered": ([vp, vp, psh, ctypes.c_double, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
+        "thrift_attention_tiered": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_pool_keys": ([vp, psh, vp, vp], st),
@@ -100,7 +101,7 @@ _lib = _load()
 # C-ABI symbols the header declares (checked by the tests).
 EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
            "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_select_blocks_tiered",
-           "thrift_attention",
+           "thrift_attention", "thrift_attention_tiered",
            "thrift_fused_workspace_bytes",
            "thrift_attention_fused", "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
            "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error", "thrift_mma_rate_probe",
@@ -261,6 +262,20 @@ def attention(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=No
     if out is None:
         out = torch.empty_like(Qt)
     _check("thrift_attention", _lib.thrift_attention(
+        _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
+        _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
+    return out
+
+
+def attention_tiered(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None):
+    """attention() for masks that may hold 2 (skipped pairs, absent from the
+    softmax), as from select_blocks_tiered."""
+    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    _dev(mask, "mask", torch.uint8)
+    if out is None:
+        out = torch.empty_like(Qt)
+    _check("thrift_attention_tiered", _lib.thrift_attention_tiered(
         _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
         _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
     return out

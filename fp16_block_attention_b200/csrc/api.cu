@@ -181,9 +181,10 @@ thrift_status thrift_select_blocks_static(const void* Q, const void* K, const th
   return from_cuda(launch_select_static(Q, K, *shape, rho, mask, static_cast<cudaStream_t>(stream)));
 }
 
-thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
-                               const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                               const thrift_shape* shape, void* O, void* stream) {
+namespace {
+thrift_status attention_entry(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
+                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
+                              const thrift_shape* shape, void* O, bool skip, void* stream) {
   thrift_status st = check_shape(shape);
   if (st != THRIFT_OK) return st;
   const void* ptrs[] = {Q, K, V, q4, qs, k4, ks, v4, vs, O};
@@ -192,8 +193,21 @@ thrift_status thrift_attention(const void* Q, const void* K, const void* V, cons
   if (!mask) return THRIFT_ERR_INVALID_ARG;
   uint32_t* err = device_error_word();
   if (!err) return THRIFT_ERR_CUDA;
-  return from_cuda(
-      launch_attention(Q, K, V, mask, q4, qs, k4, ks, v4, vs, *shape, O, err, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_attention(Q, K, V, mask, q4, qs, k4, ks, v4, vs, *shape, O, skip, err,
+                                    static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
+                               const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
+                               const thrift_shape* shape, void* O, void* stream) {
+  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, false, stream);
+}
+
+thrift_status thrift_attention_tiered(const void* Q, const void* K, const void* V, const uint8_t* mask,
+                                      const void* q4, const void* qs, const void* k4, const void* ks, const void* v4,
+                                      const void* vs, const thrift_shape* shape, void* O, void* stream) {
+  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, true, stream);
 }
 
 thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
@@ -224,7 +238,7 @@ thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V
   if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   if (launch_select(Q, K, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
-  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, err, cs));
+  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, false, err, cs));
 }
 
 namespace {

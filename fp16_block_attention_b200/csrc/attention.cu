@@ -100,13 +100,17 @@ struct Misc {
   volatile int abort;
   float red_max[2][kSplit][128];
   float red_l[kSplit][128];
-  uint8_t cls[1024];  // per key tile: bit (a*2 + c) = FP16 flag, bit 4 + (a*2 + c) = skip flag of block
-                      // (query half a, key half c)
+  uint8_t cls[1024];  // per key tile: bit (a*2 + c) = FP16 flag of block (query half a, key half c);
+                      // SKIP: bit 4 + (a*2 + c) = skip flag
 };
 
 static_assert(sizeof(Misc) <= 8192, "barriers and exchange buffers must fit their shared-memory slice");
 
-template <int D>
+// SKIP = false: masks of 0 / 1 (the method).  SKIP = true: masks may hold 2
+// (skipped pairs); a skipped block is computed like an NVFP4 one and its keys
+// are then masked out of the softmax.  Separate instantiations, so the first
+// keeps its own code.
+template <int D, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1)
     thrift_attention_kernel(const __grid_constant__ CUtensorMap mQ16, const __grid_constant__ CUtensorMap mK16,
                             const __grid_constant__ CUtensorMap mV16, const __grid_constant__ CUtensorMap mQ4,
@@ -152,20 +156,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // precision class of every key tile of this query tile
   const uint8_t* mrow = p.mask + static_cast<size_t>(bh) * nb * nb;
-  // (mask 1 FP16, 0 NVFP4, 2 skipped: a skipped block is computed like an
-  // NVFP4 one and then masked out of the softmax)
   for (int kt = tid; kt < n_kt; kt += kThreads) {
     uint32_t c = 0;
     if (p.blk == 128) {
       const uint8_t mv = mrow[static_cast<size_t>(qt) * nb + kt];
-      c = (mv == 1 ? 0xFu : 0u) | (mv == 2 ? 0xF0u : 0u);
+      c = SKIP ? ((mv == 1 ? 0xFu : 0u) | (mv == 2 ? 0xF0u : 0u)) : (mv ? 0xFu : 0u);
     } else {
       for (int a = 0; a < 2; ++a)
         for (int k = 0; k < 2; ++k) {
           const int i = 2 * qt + a, j = 2 * kt + k;
           const uint8_t mv = (i < nb && j < nb) ? mrow[static_cast<size_t>(i) * nb + j] : 0;
-          if (mv == 1) c |= 1u << (a * 2 + k);
-          if (mv == 2) c |= 1u << (4 + a * 2 + k);
+          if (SKIP ? mv == 1 : mv != 0) c |= 1u << (a * 2 + k);
+          if (SKIP && mv == 2) c |= 1u << (4 + a * 2 + k);
         }
     }
     ms.cls[kt] = static_cast<uint8_t>(c);
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 &ms.bar_q);
       int u4 = 0, u16 = 0, u16k_only = 0;
       for (int kt = 0; kt < n_kt && !ms.abort; ++kt) {
-        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
+        const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
           if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t o_acc = 0;
       // issue S of tile kt (its loads are complete)
       auto issue_s = [&](int kt) {
-        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
+        const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         const uint32_t sfset = tm + kColSF + 24 * (kt & 1);
         if (c != 0u) {
           const uint32_t k16 = sbase + L::kSlot16;
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // wait for the loads of tile kt; records its FP4 slot
       auto wait_loads = [&](int kt) -> bool {
-        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
+        const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
           if (!wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!wait_or_abort(&ms.bar_p_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) break;
         tc_fence_after();
-        const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
+        const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         const uint32_t sfset = tm + kColSF + 24 * (kt & 1);
         const int slot4 = slot4_of[kt & 1];
         if (c != 0xFu) {
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float M = -INFINITY, l = 0.f;
     bool failed = false;  // this thread gave up a wait; the exit is taken jointly
     for (int kt = 0; kt < n_kt; ++kt) {
-      const uint32_t c = ms.cls[kt] & 0xFu;  // FP16 flags
+      const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
       const bool fp16 = (c >> (a * 2 + kh)) & 1u;
       const bool need16 = c != 0u, need4 = c != 0xFu;
       if (!failed) failed = !wait_or_abort(&ms.bar_s_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
@@ -376,15 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < kKPT; ++j) s[j] = -INFINITY;
       }
 
-      // A skipped block leaves the softmax: all of this thread's keys.
-      if ((ms.cls[kt] >> (4 + a * 2 + kh)) & 1u) {
-#pragma unroll
-        for (int j = 0; j < kKPT; ++j) s[j] = -INFINITY;
-      }
-      // Mask keys past N and, on the diagonal tile, keys after the query.
+      // Mask keys past N, on the diagonal tile keys after the query, and (SKIP)
+      // all of this thread's keys when its block is skipped.
       const int key0 = kt * 128 + koff;
-      if (kt * 128 + 128 > p.N || (p.causal && kt == qt)) {
-        const int lim = p.causal ? min(qrow + 1, p.N) : p.N;  // keys < lim are valid
+      const bool skipped = SKIP && ((ms.cls[kt] >> (4 + a * 2 + kh)) & 1u);
+      if (kt * 128 + 128 > p.N || (p.causal && kt == qt) || skipped) {
+        const int lim = skipped ? key0 : (p.causal ? min(qrow + 1, p.N) : p.N);  // keys < lim are valid
 #pragma unroll
         for (int j = 0; j < kKPT; ++j)
           if (key0 + j >= lim) s[j] = -INFINITY;
@@ -560,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4, const void* qs,
                      const void* k4, const void* ks, const void* v4, const void* vs, const thrift_shape& s, void* O,
-                     uint32_t* err, cudaStream_t st) {
+                     bool skip, uint32_t* err, cudaStream_t st) {
   CUtensorMap mQ16, mK16, mV16, mQ4, mK4, mV4;
   const uint64_t BHq = static_cast<uint64_t>(s.B) * s.Hq, BHk = static_cast<uint64_t>(s.B) * s.Hkv;
   const CUtensorMapSwizzle sw4 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -587,13 +586,14 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.causal = s.causal;
   prm.NT = num_tiles(s.N);
   prm.scale_log2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
+  prm.skip = skip ? 1 : 0;
   if (s.blk == 128) return launch_attention_db<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
   const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   const size_t smem = Smem<D>::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(thrift_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const auto kern = skip ? thrift_attention_kernel<D, true> : thrift_attention_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  thrift_attention_kernel<D><<<grid, kThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
+  kern<<<grid, kThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
   return cudaGetLastError();
 }
 
@@ -601,9 +601,9 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
 
 cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                             const thrift_shape& s, void* O, uint32_t* err, cudaStream_t st) {
-  if (s.D == 128) return launch_d<128>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, err, st);
-  return launch_d<64>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, err, st);
+                             const thrift_shape& s, void* O, bool skip, uint32_t* err, cudaStream_t st) {
+  if (s.D == 128) return launch_d<128>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, err, st);
+  return launch_d<64>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, err, st);
 }
 
 }  // namespace thrift

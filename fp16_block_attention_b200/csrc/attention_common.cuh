@@ -20,6 +20,7 @@ struct Params {
   uint32_t* err;
   int B, Hq, Hkv, N, blk, causal, NT;
   float scale_log2;
+  int skip;  // the mask may hold 2 (skipped pairs): the kernels' skip-aware instantiations
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,

@@ -93,12 +93,19 @@ struct MiscDB {
   uint32_t tmem;
   volatile int abort;
   float lsum[2][128];  // partial row sums of the two halves, for the epilogue
-  uint16_t lst[1024];   // key tiles to process, in order: tile index, bit 15 set = FP16
-  int np;               // their number (skipped tiles are left out)
+  union {
+    uint8_t cls[1024];   // SKIP = false: per key tile, 1 = FP16, 0 = NVFP4
+    uint16_t lst[1024];  // SKIP = true: key tiles to process in order, tile index | 0x8000 for FP16
+  };
+  int np;                // key tiles processed
 };
 static_assert(sizeof(MiscDB) <= 4096, "barriers must fit their shared-memory slice");
 
-template <int D>
+// SKIP = false: masks of 0 / 1 (the method); every key tile of the query
+// tile is processed.  SKIP = true: masks may hold 2 (skipped pairs); the
+// skipped tiles are left out of an ordered list that every role walks.  The
+// two are separate instantiations so the first keeps its own code.
+template <int D, bool SKIP>
 __global__ void __launch_bounds__(kDBThreads, 1)
     thrift_attention_db_kernel(const __grid_constant__ CUtensorMap mQ16, const __grid_constant__ CUtensorMap mK16,
                                const __grid_constant__ CUtensorMap mV16, const __grid_constant__ CUtensorMap mQ4,
@@ -143,26 +150,38 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     ms.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    // Key tiles to process in increasing order: mask 1 FP16, 0 NVFP4, 2 skipped
-    // (left out of the list, so no role spends anything on them).
-    const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
-    int base = 0;
-    for (int k0 = 0; k0 < nk; k0 += 32) {
-      const int kt = k0 + lane;
-      const uint8_t mv = kt < nk ? m0[kt] : 2;
-      const uint32_t keep = __ballot_sync(0xffffffffu, mv != 2);
-      if (mv != 2)
-        ms.lst[base + __popc(keep & ((1u << lane) - 1u))] = static_cast<uint16_t>(kt | (mv == 1 ? 0x8000 : 0));
-      base += __popc(keep);
+  if constexpr (SKIP) {
+    if (warp == 0) {
+      // Key tiles to process in increasing order: mask 1 FP16, 0 NVFP4, 2
+      // skipped (left out).  All of the row's mask bytes are loaded at once
+      // (nk <= 1024 = 32 x 32), then compacted in order from registers.
+      const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
+      uint8_t mv[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) mv[q] = (q * 32 + lane < nk) ? m0[q * 32 + lane] : 2;
+      int base = 0;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const uint32_t keep = __ballot_sync(0xffffffffu, mv[q] != 2);
+        if (mv[q] != 2)
+          ms.lst[base + __popc(keep & ((1u << lane) - 1u))] =
+              static_cast<uint16_t>((q * 32 + lane) | (mv[q] == 1 ? 0x8000 : 0));
+        base += __popc(keep);
+      }
+      if (lane == 0) ms.np = base;
     }
-    if (lane == 0) ms.np = base;
+  } else {
+    const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
+    for (int kt = tid; kt < nk; kt += kDBThreads) ms.cls[kt] = m0[kt] ? 1 : 0;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ms.tmem;
-  const int np = ms.np;
+  const int np = SKIP ? ms.np : nk;
+  // the it-th processed key tile and its precision
+  const auto tile_of = [&](int it) -> int { return SKIP ? (ms.lst[it] & 0x3FF) : it; };
+  const auto fp16_of = [&](int it) -> bool { return SKIP ? (ms.lst[it] & 0x8000) != 0 : ms.cls[it] != 0; };
 
   if (warp == kDBProducer) {
     // ======================== producer ========================
@@ -177,8 +196,8 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       bulk_load(sm + L::kQSF, p.qs + (static_cast<size_t>(bh) * p.NT + qt) * L::kQSFBytes, L::kQSFBytes, &ms.bar_q);
       int u4 = 0, u16 = 0;
       for (int it = 0; it < np && !ms.abort; ++it) {
-        const int kt = ms.lst[it] & 0x3FF;
-        if (!(ms.lst[it] & 0x8000)) {
+        const int kt = tile_of(it);
+        if (!fp16_of(it)) {
           const int slot = u4 % L::kNS, use = u4 / L::kNS;
           if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
@@ -231,7 +250,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       int u4 = 0, uk16 = 0;
       for (int it = 0; ok && it < np; ++it) {
         const int bb = it & 1;
-        const bool fp16 = (ms.lst[it] & 0x8000) != 0;
+        const bool fp16 = fp16_of(it);
         int slot = 0;
         if (!fp16) {
           slot = u4 % L::kNS;
@@ -295,7 +314,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       uint32_t acc = 0u;
       for (int it = 0; ok && it < np; ++it) {
         const int bb = it & 1;
-        const bool fp16 = (ms.lst[it] & 0x8000) != 0;
+        const bool fp16 = fp16_of(it);
         // The V operands (and the V4 scales, copied to tensor memory) do not
         // depend on P, so they are made ready before waiting for it.  The copy
         // follows the previous P V product in this thread's tcgen05 order, so
@@ -370,8 +389,8 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     if (half == 1) named_bar_arrive(2, kDBSoftmax);  // half 0 goes first
     for (int it = 0; it < np; ++it) {
       const int bb = it & 1;
-      const int kt = ms.lst[it] & 0x3FF;
-      const bool fp16 = (ms.lst[it] & 0x8000) != 0;
+      const int kt = tile_of(it);
+      const bool fp16 = fp16_of(it);
       if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) {
@@ -578,17 +597,25 @@ __global__ void __launch_bounds__(kDBThreads, 1)
 
 }  // namespace
 
+template <int D, bool SKIP>
+static cudaError_t launch_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
+                             const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                             const attn::Params& prm, cudaStream_t st) {
+  const size_t smem = SmemDB<D>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(thrift_attention_db_kernel<D, SKIP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(prm.B * prm.Hq * prm.NT);
+  thrift_attention_db_kernel<D, SKIP><<<grid, kDBThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_attention_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
                                 const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
                                 const attn::Params& prm, cudaStream_t st) {
-  const size_t smem = SmemDB<D>::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(thrift_attention_db_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(prm.B * prm.Hq * prm.NT);
-  thrift_attention_db_kernel<D><<<grid, kDBThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
-  return cudaGetLastError();
+  if (prm.skip) return launch_db<D, true>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
+  return launch_db<D, false>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
 }
 
 template cudaError_t launch_attention_db<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

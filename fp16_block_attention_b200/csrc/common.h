@@ -77,8 +77,9 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
 // Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
 cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);
 
+// skip: the mask may hold 2 (skipped pairs); selects the kernels' skip-aware instantiations.
 cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                             const thrift_shape& s, void* O, uint32_t* err, cudaStream_t st);
+                             const thrift_shape& s, void* O, bool skip, uint32_t* err, cudaStream_t st);
 
 }  // namespace thrift

@@ -128,7 +128,7 @@ THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, cons
  *   the others                                               -> 0 (NVFP4)
  * so the forced pairs (diagonal and key block 0, 2 nb - 1 of them) and the
  * FP16 pairs are never skipped; sigma = 0 gives thrift_select_blocks' mask.
- * thrift_attention treats a skipped pair as absent from the softmax.
+ * thrift_attention_tiered treats a skipped pair as absent from the softmax.
  * Workspace, layout and errors as for thrift_select_blocks. */
 THRIFT_API thrift_status thrift_select_blocks_tiered(const void* Q, const void* K, const thrift_shape* shape,
                                                      double rho, double sigma, uint8_t* mask, void* ws,
@@ -183,13 +183,23 @@ THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* 
 
 /* Stage 2 (ThriftAttention abstract: picked pairs in FP16, the others in
  * FP4, one online softmax merging both): O [B][Hq][N][D] fp16.
- * mask: as written by thrift_select_blocks (1 FP16, 0 NVFP4), or by
- * thrift_select_blocks_tiered (2: skipped, absent from the softmax; every
- * query block must keep at least one pair); q4/qs, k4/ks, v4/vs: the NVFP4
+ * mask: as written by thrift_select_blocks (1 FP16, 0 NVFP4; any nonzero
+ * byte counts as FP16); q4/qs, k4/ks, v4/vs: the NVFP4
  * copies written by thrift_quantize_nvfp4 for Q, K and V. */
 THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
                                const thrift_shape* shape, void* O, void* stream);
+
+/* thrift_attention for masks that may also hold 2, as written by
+ * thrift_select_blocks_tiered: a skipped pair is absent from the softmax
+ * (every query row must keep at least one key; the tiered selection never
+ * skips the diagonal).  With blk = 128 the skipped key tiles are left out of
+ * the kernel's work; with blk = 64 a skipped block inside a 128-key tile is
+ * computed and masked.  Arguments and errors as for thrift_attention. */
+THRIFT_API thrift_status thrift_attention_tiered(const void* Q, const void* K, const void* V, const uint8_t* mask,
+                                                 const void* q4, const void* qs, const void* k4, const void* ks,
+                                                 const void* v4, const void* vs, const thrift_shape* shape, void* O,
+                                                 void* stream);
 
 /* Workspace bytes of thrift_attention_fused (NVFP4 copies, mask and the
  * selection workspace, each 256-byte aligned). */

@@ -79,7 +79,7 @@ def test_attention_with_skipped_pairs_matches_oracle(w, rho, sigma):
     assert (m == 2).any()
     md, = to_dev(m)
     qz = thrift.quantize_all(Qd, Kd, Vd, sh)
-    o = thrift.attention(Qd, Kd, Vd, md, qz, sh)
+    o = thrift.attention_tiered(Qd, Kd, Vd, md, qz, sh)
     assert thrift.last_device_error() == 0
     o = o.cpu().numpy()
     rows = oracle.all_rows(w.B, w.Hq, w.N)
@@ -89,3 +89,36 @@ def test_attention_with_skipped_pairs_matches_oracle(w, rho, sigma):
                                              w.causal, w.sm_scale)
     assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
     assert resolved <= max(1, rows.shape[0] // 1000), resolved  # ties are rare
+
+
+@pytest.mark.parametrize("sigma", [0.0, 0.25, 0.5, 0.75])
+def test_quality_cost_of_skipping(sigma):
+    """The relative error of the output against exact attention on sampled
+    rows of the causal GQA generator (N = 8192) at rho = 5% as the skipped
+    share grows, GPU beside the oracle (within one point of the FP4-to-FP16
+    gap).  Run with -s for the series."""
+    w = synth.GQA_N32K.with_(N=8192)
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    sh = shape_of(w)
+    rows = synth.sample_rows(w, 48, per_block=8)
+    ex = oracle.exact_rows(Q, K, V, rows, w.causal, w.sm_scale)
+    qd = thrift.quantize_all(Qd, Kd, Vd, sh)
+    qz = oracle.Quantised(Q, K, V)
+
+    def gpu(mask_d):
+        o = thrift.attention_tiered(Qd, Kd, Vd, mask_d, qd, sh).cpu().numpy()
+        assert thrift.last_device_error() == 0
+        return o[rows[:, 0], rows[:, 1], rows[:, 2]].astype(np.float64)
+
+    err = lambda o: float(np.linalg.norm(o - ex) / np.linalg.norm(ex))
+    e4 = err(gpu(thrift.select_blocks(Qd, Kd, sh, 0.0)))
+    e16 = err(gpu(thrift.select_blocks(Qd, Kd, sh, 1.0)))
+    m = thrift.select_blocks_tiered(Qd, Kd, sh, w.rho, sigma)
+    eg = err(gpu(m))
+    er = err(oracle.to_f16(oracle.attention_rows(Q, K, V, m.cpu().numpy(), rows, w.blk, w.causal, w.sm_scale, qz)))
+    skipped = float((m.cpu().numpy() == 2).mean() / (0.5 + 0.5 / (w.N // w.blk)))
+    gap = lambda e: 100.0 * (e4 - e) / (e4 - e16)
+    print(f"\nskip sigma={sigma}: skipped share {skipped:.3f} E(gpu)={eg:.5f} E(oracle)={er:.5f} "
+          f"E(rho=0)={e4:.5f} E(rho=1)={e16:.5f} gap_gpu={gap(eg):.2f} gap_oracle={gap(er):.2f}")
+    assert abs(gap(eg) - gap(er)) <= 1.0
