@@ -29,6 +29,8 @@ class Problem(ctypes.Structure):
         ("Q", ctypes.c_void_p), ("K", ctypes.c_void_p), ("V", ctypes.c_void_p),
         ("q4", ctypes.c_void_p), ("qs", ctypes.c_void_p), ("k4", ctypes.c_void_p), ("ks", ctypes.c_void_p),
         ("v4", ctypes.c_void_p), ("vs", ctypes.c_void_p),
+        ("q8", ctypes.c_void_p), ("qs8", ctypes.c_void_p), ("k8", ctypes.c_void_p), ("ks8", ctypes.c_void_p),
+        ("v8", ctypes.c_void_p), ("vs8", ctypes.c_void_p),
         ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("N", ctypes.c_int),
         ("D", ctypes.c_int), ("blk", ctypes.c_int), ("causal", ctypes.c_int),
         ("sm_scale", ctypes.c_float), ("p_log2", ctypes.c_int), ("p_jitter", ctypes.c_double),
@@ -58,7 +60,11 @@ def _load():
         "orc_e2m1_encode": ([f64], ctypes.c_uint8),
         "orc_e4m3_value": ([ctypes.c_uint8], f64),
         "orc_e4m3_encode": ([f64], ctypes.c_uint8),
+        "orc_e4m3_encode_direct": ([f64], ctypes.c_uint8),
+        "orc_e8m0_value": ([ctypes.c_uint8], f64),
         "orc_quantize_rows": ([vp, i64, i32, vp, vp], i32),
+        "orc_quantize_rows_mx8": ([vp, i64, i32, vp, vp], i32),
+        "orc_quantize_v_mx8": ([vp, i64, i32, i32, vp, vp], i32),
         "orc_quantize_v": ([vp, i64, i32, i32, vp, vp], i32),
         "orc_budget": ([f64, i64], i64),
         "orc_pooled_scores": ([vp, vp, i32, i32, i32, i32, ctypes.c_float, vp], i32),
@@ -139,6 +145,46 @@ def quantize_v(V):
     return codes, scales
 
 
+def e4m3_encode_direct(v: float) -> int:
+    return int(_load().orc_e4m3_encode_direct(float(v)))
+
+
+def e8m0_value(code: int) -> float:
+    return float(_load().orc_e8m0_value(int(code)))
+
+
+def quantize_rows_mx8(x):
+    """MXFP8 along the last axis: codes [..., L] (E4M3 bytes) and scales
+    [..., L/32] (E8M0 bytes)."""
+    x = _bits16(x)
+    L = x.shape[-1]
+    rows = x.size // L
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty(x.shape[:-1] + (L // 32,), np.uint8)
+    if _load().orc_quantize_rows_mx8(x.ctypes.data, rows, L, codes.ctypes.data, scales.ctypes.data):
+        raise ValueError("orc_quantize_rows_mx8: length must be a multiple of 32")
+    return codes, scales
+
+
+def quantize_v_mx8(V):
+    """MXFP8 of V [B,H,N,D] along keys: codes [B,H,D,N], scales [B,H,D,N/32]."""
+    V = _bits16(V)
+    B, H, N, D = V.shape
+    codes = np.empty((B, H, D, N), np.uint8)
+    scales = np.empty((B, H, D, N // 32), np.uint8)
+    if _load().orc_quantize_v_mx8(V.ctypes.data, B * H, N, D, codes.ctypes.data, scales.ctypes.data):
+        raise ValueError("orc_quantize_v_mx8: N must be a multiple of 32")
+    return codes, scales
+
+
+def dequantize_mx8(codes, scales):
+    """Decode MXFP8 codes / scales along the last axis into float64 (test helper)."""
+    codes = np.asarray(codes, np.uint8)
+    vals = np.array([e4m3_value(c) for c in range(256)])[codes]
+    sc = np.array([e8m0_value(e) for e in range(256)])[np.asarray(scales, np.uint8)]
+    return vals * np.repeat(sc, 32, axis=-1)
+
+
 def dequantize(codes, scales):
     """Decode NVFP4 codes/scales along the last axis into float64 (test helper)."""
     lut = np.array([e2m1_value(c) for c in range(16)])
@@ -176,9 +222,9 @@ def select(Q, K, blk, causal, sm_scale, rho):
     return mask
 
 
-def select_tiered(Q, K, blk, causal, sm_scale, rho, sigma):
-    """Mask [B,Hq,nb,nb] (u8: 1 FP16, 0 NVFP4, 2 skip) of the tiered selection
-    (``tiered``) on the pooled scores of every (batch, query head)."""
+def select_tiered(Q, K, blk, causal, sm_scale, rho, sigma, rho8=0.0):
+    """Mask [B,Hq,nb,nb] (u8: 1 FP16, 3 MXFP8, 0 NVFP4, 2 skip) of the tiered
+    selection (``tiered``) on the pooled scores of every (batch, query head)."""
     from . import tiered
     B, Hq = Q.shape[:2]
     group = Hq // K.shape[1]
@@ -187,7 +233,7 @@ def select_tiered(Q, K, blk, causal, sm_scale, rho, sigma):
     for b in range(B):
         for h in range(Hq):
             sc = pooled_scores(Q[b, h], K[b, h // group], blk, causal, sm_scale)
-            mask[b, h] = tiered.select_head(sc, causal, rho, sigma, budget)
+            mask[b, h] = tiered.select_head(sc, causal, rho, sigma, budget, rho8)
     return mask
 
 
@@ -208,12 +254,18 @@ def select_vertical_window(Q, K, blk, causal, sm_scale, rho, window):
 
 # ---- attention -------------------------------------------------------------------
 class Quantised:
-    """Oracle NVFP4 copies of Q, K (along D) and V (along keys)."""
+    """Oracle NVFP4 copies of Q, K (along D) and V (along keys); with mx8, also
+    the MXFP8 copies that 8-bit pairs (mask value 3) read."""
 
-    def __init__(self, Q, K, V):
+    def __init__(self, Q, K, V, mx8=False):
         self.q4, self.qs = quantize_rows(Q)
         self.k4, self.ks = quantize_rows(K)
         self.v4, self.vs = quantize_v(V)
+        self.q8 = self.qs8 = self.k8 = self.ks8 = self.v8 = self.vs8 = None
+        if mx8:
+            self.q8, self.qs8 = quantize_rows_mx8(Q)
+            self.k8, self.ks8 = quantize_rows_mx8(K)
+            self.v8, self.vs8 = quantize_v_mx8(V)
 
 
 def _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep, p_jitter=0.0):
@@ -226,7 +278,12 @@ def _problem(Q, K, V, qz, blk, causal, sm_scale, p_log2, keep, p_jitter=0.0):
         arrs = [_c(qz.q4), _c(qz.qs), _c(qz.k4), _c(qz.ks), _c(qz.v4), _c(qz.vs)]
         keep.extend(arrs)
         ptrs = [a.ctypes.data for a in arrs]
-    return Problem(Q.ctypes.data, K.ctypes.data, V.ctypes.data, *ptrs, B, Hq, Hkv, N, D, blk,
+    ptrs8 = [None] * 6
+    if qz is not None and getattr(qz, "q8", None) is not None:
+        arrs = [_c(qz.q8), _c(qz.qs8), _c(qz.k8), _c(qz.ks8), _c(qz.v8), _c(qz.vs8)]
+        keep.extend(arrs)
+        ptrs8 = [a.ctypes.data for a in arrs]
+    return Problem(Q.ctypes.data, K.ctypes.data, V.ctypes.data, *ptrs, *ptrs8, B, Hq, Hkv, N, D, blk,
                    int(causal), float(sm_scale), int(p_log2), float(p_jitter))
 
 
@@ -245,8 +302,11 @@ def attention_rows(Q, K, V, mask, rows, blk, causal, sm_scale, qz=None, order=No
     order_arr = None
     if order is not None:
         order_arr = _c(np.asarray(order, np.int32))
-    if _load().orc_attention_rows(ctypes.byref(p), mask.ctypes.data, rows.ctypes.data, rows.shape[0],
-                                  None if order_arr is None else order_arr.ctypes.data, out.ctypes.data):
+    rc = _load().orc_attention_rows(ctypes.byref(p), mask.ctypes.data, rows.ctypes.data, rows.shape[0],
+                                    None if order_arr is None else order_arr.ctypes.data, out.ctypes.data)
+    if rc == 2:
+        raise ValueError("8-bit pairs (mask 3) need Quantised(..., mx8=True)")
+    if rc:
         raise ValueError("orc_attention_rows rejected the shape")
     return out
 

@@ -31,7 +31,10 @@
  *   - l sums the unquantised P; quantisation only encodes the P.V operand.
  *   - A mask value of 2 marks a skipped pair, absent from the softmax (the
  *     skip precision of TriAttention's tile assignment, abstract on the paper
- *     page of arXiv 2611.07256); 1 is FP16, 0 NVFP4.
+ *     page of arXiv 2611.07256); 3 marks an 8-bit pair (the same page's 8-bit
+ *     precision), computed in MXFP8: the OCP microscaling format with E4M3
+ *     elements and one E8M0 power-of-two scale per 32 elements (Q, K along D,
+ *     V along keys, P per 32 keys); 1 is FP16, 0 NVFP4.
  * All arithmetic is FP64 with FP32/FP16/FP4 rounding at the points the
  * readings name.
  */
@@ -206,6 +209,83 @@ static double deq(const uint8_t* codes, const uint8_t* scales, long row, int len
 }
 
 /* ------------------------------------------------------------------------ */
+/* MXFP8 group quantisation (8-bit pairs)                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Nearest E4M3 to v by its binary expansion, ties to even, saturating at 448:
+ * the same result as orc_e4m3_encode's search (a pin checks the two agree),
+ * fast enough for whole tensors. */
+uint8_t orc_e4m3_encode_direct(double v) {
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs(v);
+    if (a >= 464.0) return sign | 0x7E;            /* 464 = 448 + half a step: saturate */
+    if (a < ldexp(1.0, -6)) {                        /* subnormal: m * 2^-9, m = 0..8 */
+        double m = nearbyint(ldexp(a, 9));           /* FE_TONEAREST: ties to even */
+        return sign | (uint8_t)m;                    /* m = 8 is the smallest normal, code 8 */
+    }
+    int ex;
+    double fr = frexp(a, &ex);                       /* a = fr * 2^ex, fr in [0.5, 1) */
+    int e = ex - 1;                                  /* a = (2 fr) * 2^e, 2 fr in [1, 2) */
+    double m = nearbyint((2.0 * fr - 1.0) * 8.0);   /* mantissa steps of 1/8 */
+    if (m == 8.0) { m = 0.0; ++e; }
+    if (e > 8 || (e == 8 && m > 6.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | (int)m);
+}
+
+double orc_e8m0_value(uint8_t e) { return ldexp(1.0, (int)e - 127); }
+
+/* One MXFP8 group of 32 values: X = 2^(floor(log2 amax) - 8) (8 = the exponent
+ * of E4M3's largest normal, 448 = 1.75 * 2^8), stored as the E8M0 byte
+ * floor(log2 amax) - 8 + 127 (clamped to 0..254); codes E4M3(v / X), nearest
+ * even, saturating at 448; an all-zero group takes byte 0 and zero codes. */
+static void quant_group32_mx8(const double* x, uint8_t* codes, uint8_t* scale) {
+    double amax = 0;
+    for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(x[i]));
+    int e = 0;
+    if (amax > 0) {
+        int ex;
+        frexp(amax, &ex);
+        e = (ex - 1) - 8 + 127;
+        if (e < 0) e = 0;
+        if (e > 254) e = 254;
+    }
+    *scale = (uint8_t)e;
+    double X = orc_e8m0_value((uint8_t)e);
+    for (int i = 0; i < 32; ++i) codes[i] = amax > 0 ? orc_e4m3_encode_direct(x[i] / X) : 0;
+}
+
+/* MXFP8 along rows: codes [rows][len] (E4M3 bytes), scales [rows][len/32]. */
+int orc_quantize_rows_mx8(const uint16_t* x, long rows, int len, uint8_t* codes, uint8_t* scales) {
+    if (len <= 0 || len % 32) return 1;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r)
+        for (int g = 0; g < len / 32; ++g) {
+            double v[32];
+            for (int i = 0; i < 32; ++i) v[i] = orc_f16_value(x[r * len + g * 32 + i]);
+            quant_group32_mx8(v, codes + r * len + g * 32, &scales[r * (len / 32) + g]);
+        }
+    return 0;
+}
+
+/* MXFP8 of V along keys: V [BH][N][D] -> codes [BH][D][N], scales [BH][D][N/32]. */
+int orc_quantize_v_mx8(const uint16_t* V, long BH, int N, int D, uint8_t* codes, uint8_t* scales) {
+    if (N <= 0 || N % 32 || D <= 0) return 1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (long bh = 0; bh < BH; ++bh)
+        for (int d = 0; d < D; ++d)
+            for (int g = 0; g < N / 32; ++g) {
+                double v[32];
+                for (int i = 0; i < 32; ++i) v[i] = orc_f16_value(V[(bh * N + g * 32 + i) * (long)D + d]);
+                quant_group32_mx8(v, codes + (bh * D + d) * (long)N + g * 32, &scales[(bh * D + d) * (long)(N / 32) + g]);
+            }
+    return 0;
+}
+
+static double deq8(const uint8_t* codes, const uint8_t* scales, long row, int len, int i) {
+    return E4M3_TABLE[codes[row * len + i]] * orc_e8m0_value(scales[row * (len / 32) + i / 32]);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Stage 1: block-pair selection                                             */
 /* ------------------------------------------------------------------------ */
 
@@ -309,6 +389,8 @@ typedef struct {
     const uint16_t *Q, *K, *V;                 /* fp16 [B,H,N,D] */
     const uint8_t *q4, *qs, *k4, *ks;          /* NVFP4 along D: [B,H,N,D/2], [B,H,N,D/16] */
     const uint8_t *v4, *vs;                    /* NVFP4 along keys: [B,Hkv,D,N/2], [B,Hkv,D,N/16] */
+    const uint8_t *q8, *qs8, *k8, *ks8;        /* MXFP8 along D: [B,H,N,D], [B,H,N,D/32] (or NULL) */
+    const uint8_t *v8, *vs8;                   /* MXFP8 along keys: [B,Hkv,D,N], [B,Hkv,D,N/32] (or NULL) */
     int B, Hq, Hkv, N, D, blk, causal;
     float sm_scale;
     int p_log2;                                /* pre-scale exponent c of P */
@@ -321,35 +403,51 @@ static float logit_log2(double S, float sm_scale) {
     return (float)((double)(float)S * (double)c);
 }
 
+/* Precision of a pair: the mask byte (0 NVFP4, 1 FP16, 3 MXFP8). */
+enum { PREC_FP4 = 0, PREC_FP16 = 1, PREC_FP8 = 3 };
+
 /* Raw score S of (query row r of head h, key k of key head hk) in the given
- * precision: FP16 operands, or dequantised NVFP4 operands.  FP64 sum. */
-static double score(const orc_problem* p, int b, int h, int hk, int r, int k, int fp16) {
+ * precision: FP16 operands, or dequantised NVFP4 / MXFP8 operands.  FP64 sum. */
+static double score(const orc_problem* p, int b, int h, int hk, int r, int k, int prec) {
     const int D = p->D;
     long qrow = ((long)b * p->Hq + h) * p->N + r;
     long krow = ((long)b * p->Hkv + hk) * p->N + k;
     double s = 0;
     for (int d = 0; d < D; ++d) {
-        double qv = fp16 ? F16_TABLE[p->Q[qrow * D + d]] : deq(p->q4, p->qs, qrow, D, d);
-        double kv = fp16 ? F16_TABLE[p->K[krow * D + d]] : deq(p->k4, p->ks, krow, D, d);
+        double qv = prec == PREC_FP16 ? F16_TABLE[p->Q[qrow * D + d]]
+                  : prec == PREC_FP8  ? deq8(p->q8, p->qs8, qrow, D, d) : deq(p->q4, p->qs, qrow, D, d);
+        double kv = prec == PREC_FP16 ? F16_TABLE[p->K[krow * D + d]]
+                  : prec == PREC_FP8  ? deq8(p->k8, p->ks8, krow, D, d) : deq(p->k4, p->ks, krow, D, d);
         s += qv * kv;
     }
     return s;
 }
 
 /* V element (key k, channel d) in the given precision. */
-static double v_elem(const orc_problem* p, int b, int hk, int k, int d, int fp16) {
-    if (fp16) return F16_TABLE[p->V[(((long)b * p->Hkv + hk) * p->N + k) * p->D + d]];
+static double v_elem(const orc_problem* p, int b, int hk, int k, int d, int prec) {
+    if (prec == PREC_FP16) return F16_TABLE[p->V[(((long)b * p->Hkv + hk) * p->N + k) * p->D + d]];
     long vrow = ((long)b * p->Hkv + hk) * p->D + d;
+    if (prec == PREC_FP8) return deq8(p->v8, p->vs8, vrow, p->N, k);
     return deq(p->v4, p->vs, vrow, p->N, k);
 }
 
-/* Encode the P of one key block: FP16 (nearest fp16 of P*2^c) or NVFP4 per
- * aligned group of 16 keys of P*2^c; returns the decoded values times 2^-c.
- * Masked keys carry P = 0. */
-static void encode_p(const double* P, int n, int fp16, int p_log2, double* out) {
+/* Encode the P of one key block: FP16 (nearest fp16 of P*2^c), MXFP8 per
+ * aligned group of 32 keys, or NVFP4 per aligned group of 16 keys of P*2^c;
+ * returns the decoded values times 2^-c.  Masked keys carry P = 0. */
+static void encode_p(const double* P, int n, int prec, int p_log2, double* out) {
     double pre = ldexp(1.0, p_log2), post = ldexp(1.0, -p_log2);
-    if (fp16) {
+    if (prec == PREC_FP16) {
         for (int i = 0; i < n; ++i) out[i] = orc_f16_value(orc_f16_encode(P[i] * pre)) * post;
+        return;
+    }
+    if (prec == PREC_FP8) {
+        for (int g = 0; g < n; g += 32) {
+            double x[32];
+            uint8_t c[32], sc;
+            for (int i = 0; i < 32; ++i) x[i] = P[g + i] * pre;
+            quant_group32_mx8(x, c, &sc);
+            for (int i = 0; i < 32; ++i) out[g + i] = E4M3_TABLE[c[i]] * orc_e8m0_value(sc) * post;
+        }
         return;
     }
     for (int g = 0; g < n; g += 16) {
@@ -383,12 +481,12 @@ static void attention_row(const orc_problem* p, const uint8_t* mask, int b, int 
          * the softmax: the skip precision of TriAttention's tile assignment) */
         uint8_t cls = mask[(((long)b * p->Hq + h) * nb + qb) * nb + j];
         if (cls == 2) continue;
-        int fp16 = cls == 1;
+        int prec = cls == 1 ? PREC_FP16 : cls == 3 ? PREC_FP8 : PREC_FP4;
         float tmax = -INFINITY;
         for (int i = 0; i < blk; ++i) {
             int k = j * blk + i;
             if (p->causal && k > r) { t[i] = -INFINITY; continue; }
-            t[i] = logit_log2(score(p, b, h, hk, r, k, fp16), p->sm_scale);
+            t[i] = logit_log2(score(p, b, h, hk, r, k, prec), p->sm_scale);
             if (t[i] > tmax) tmax = t[i];
         }
         double Mn = fmax(M, ceil((double)tmax));
@@ -411,11 +509,11 @@ static void attention_row(const orc_problem* p, const uint8_t* mask, int b, int 
             for (int i = 0; i < blk; ++i) Pt[i] = P[i] * (1.0 + p->p_jitter);
         else
             memcpy(Pt, P, sizeof(double) * blk);
-        encode_p(Pt, blk, fp16, p->p_log2, Pt);
+        encode_p(Pt, blk, prec, p->p_log2, Pt);
         for (int i = 0; i < blk; ++i) {
             if (Pt[i] == 0.0) continue;
             int k = j * blk + i;
-            for (int d = 0; d < D; ++d) acc[d] += Pt[i] * v_elem(p, b, hk, k, d, fp16);
+            for (int d = 0; d < D; ++d) acc[d] += Pt[i] * v_elem(p, b, hk, k, d, prec);
         }
     }
     for (int d = 0; d < D; ++d) out[d] = acc[d] / l;
@@ -434,6 +532,11 @@ static int check_problem(const orc_problem* p) {
 int orc_attention_rows(const orc_problem* p, const uint8_t* mask, const int64_t* rows, long nrows,
                        const int* order, double* out) {
     if (check_problem(p)) return 1;
+    if (!p->q8 || !p->k8 || !p->v8) {  /* 8-bit pairs need the MXFP8 copies */
+        long nb = p->N / p->blk, n = (long)p->B * p->Hq * nb * nb;
+        for (long i = 0; i < n; ++i)
+            if (mask[i] == 3) return 2;
+    }
     #pragma omp parallel for schedule(dynamic, 4)
     for (long i = 0; i < nrows; ++i)
         attention_row(p, mask, (int)rows[3 * i], (int)rows[3 * i + 1], (int)rows[3 * i + 2], order,

@@ -10,21 +10,23 @@ then the pooled score descending, then the lower linear index) and cuts it
 in three:
 
   the first k16 = ceil(rho * #valid - 1e-9) pairs      FP16   (mask 1)
+  the next  k8  = min(ceil(rho8 * #valid - 1e-9),
+                      #valid - k16) pairs               MXFP8  (mask 3)
   the last  ks  = min(ceil(sigma * #valid - 1e-9),
-                      #valid - max(k16, #forced))       skip   (mask 2)
+                      #valid - max(k16 + k8, #forced))  skip   (mask 2)
   the rest                                              NVFP4  (mask 0)
 
-so forced pairs and FP16 pairs are never skipped, and sigma = 0 gives the
-method's two-class mask.  A skipped pair is absent from the softmax (the
-row oracle's mask value 2).
+so precision falls with rank, forced, FP16 and 8-bit pairs are never
+skipped, and rho8 = sigma = 0 gives the method's two-class mask.  A skipped
+pair is absent from the softmax (the row oracle's mask value 2).
 """
 from __future__ import annotations
 
 import numpy as np
 
 
-def select_head(scores: np.ndarray, causal: bool, rho: float, sigma: float, budget) -> np.ndarray:
-    """Mask [nb, nb] (u8: 1 FP16, 0 NVFP4, 2 skip) of one head from its pooled scores."""
+def select_head(scores: np.ndarray, causal: bool, rho: float, sigma: float, budget, rho8: float = 0.0) -> np.ndarray:
+    """Mask [nb, nb] (u8: 1 FP16, 3 MXFP8, 0 NVFP4, 2 skip) of one head from its pooled scores."""
     nb = scores.shape[0]
     ii, jj = np.meshgrid(np.arange(nb), np.arange(nb), indexing="ij")
     valid = (jj <= ii) if causal else np.ones((nb, nb), bool)
@@ -35,9 +37,11 @@ def select_head(scores: np.ndarray, causal: bool, rho: float, sigma: float, budg
     order = np.lexsort((i * nb + j, -sc, ~forced))
     n = int(valid.sum())
     k16 = budget(rho, n)
-    ks = min(budget(sigma, n), n - max(k16, int(forced.sum())))
+    k8 = min(budget(rho8, n), n - k16)
+    ks = min(budget(sigma, n), n - max(k16 + k8, int(forced.sum())))
     mask = np.zeros((nb, nb), np.uint8)
     mask[i[order[:k16]], j[order[:k16]]] = 1
+    mask[i[order[k16:k16 + k8]], j[order[k16:k16 + k8]]] = 3
     if ks > 0:
         mask[i[order[n - ks:]], j[order[n - ks:]]] = 2
     return mask

@@ -104,3 +104,28 @@ def test_a_skipped_pair_is_absent_from_the_softmax():
         p = np.exp(s - s.max())
         ex[t] = p @ V[0, 0, keys].astype(np.float64) / p.sum()
     assert np.linalg.norm(o - ex) / np.linalg.norm(ex) < 1e-3
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_eight_bit_pairs_come_next_in_rank(causal):
+    """With an 8-bit budget: the FP16 pairs are unchanged, the 8-bit pairs are
+    the next ones of the ranking (every 8-bit pair's score between the FP16
+    cut and the NVFP4 pairs' scores), and skipping spares them."""
+    w, Q, K, V = _case(N=1024, Hq=2, Hkv=1, causal=causal)
+    nb = w.N // w.blk
+    n = int(_valid(nb, causal).sum())
+    for rho, rho8, sigma in [(0.05, 0.1, 0.0), (0.05, 0.2, 0.5), (0.0, 0.3, 0.9)]:
+        m = oracle.select_tiered(Q, K, w.blk, causal, w.sm_scale, rho, sigma, rho8)
+        base = oracle.select_tiered(Q, K, w.blk, causal, w.sm_scale, rho, 0.0)
+        assert np.array_equal(m == 1, base == 1)
+        for h in range(w.Hq):
+            mh = m[0, h]
+            assert (mh == 3).sum() == oracle.budget(rho8, n)
+            sc = oracle.pooled_scores(Q[0, h], K[0, h // 2], w.blk, causal, w.sm_scale)
+            forced = np.zeros((nb, nb), bool)
+            forced[np.arange(nb), np.arange(nb)] = True
+            forced[:, 0] = True
+            free4 = (mh == 0) & ~forced & _valid(nb, causal)
+            free8 = (mh == 3) & ~forced
+            if free8.any() and free4.any():
+                assert sc[free8].min() >= sc[free4].max()
