@@ -71,6 +71,8 @@ def _load():
     sig = {
         "thrift_quant_bytes": ([psh, st, ctypes.POINTER(sz), ctypes.POINTER(sz)], st),
         "thrift_quantize_nvfp4": ([vp, st, psh, vp, vp, vp], st),
+        "thrift_quant8_bytes": ([psh, st, ctypes.POINTER(sz), ctypes.POINTER(sz)], st),
+        "thrift_quantize_mxfp8": ([vp, st, psh, vp, vp, vp], st),
         "thrift_select_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_select_blocks_static": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
@@ -99,7 +101,8 @@ def _load():
 _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
-EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_select_workspace_bytes", "thrift_select_blocks",
+EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quant8_bytes", "thrift_quantize_mxfp8",
+           "thrift_select_workspace_bytes", "thrift_select_blocks",
            "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_select_blocks_tiered",
            "thrift_attention", "thrift_attention_tiered",
            "thrift_fused_workspace_bytes",
@@ -161,6 +164,36 @@ def quantize_nvfp4(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=No
     _check("thrift_quantize_nvfp4", _lib.thrift_quantize_nvfp4(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
                                                                _ptr(scales), _stream(stream)))
     return codes, scales
+
+
+def quant8_bytes(shape: Shape, op: int):
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("thrift_quant8_bytes", _lib.thrift_quant8_bytes(ctypes.byref(shape.c()), op, ctypes.byref(c),
+                                                           ctypes.byref(s)))
+    return c.value, s.value
+
+
+def quantize_mxfp8(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=None, stream=None):
+    """MXFP8 copy of Q/K (along D) or V (along keys): (codes u8, scales u8)."""
+    _dev(x, "x", torch.float16)
+    nc, ns = quant8_bytes(shape, op)
+    if codes is None:
+        codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
+    _check("thrift_quantize_mxfp8", _lib.thrift_quantize_mxfp8(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
+                                                               _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def mx8_qk_scale_index(bh, n, g, NT):
+    """Byte of the MXFP8 scale of (row n, group g = d / 32) of Q or K."""
+    return (bh * NT + n // 128) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + g
+
+
+def mx8_v_scale_index(bh, d, n, NT):
+    """Byte of the MXFP8 scale of (channel d, key n) of V."""
+    return (bh * NT + n // 128) * 512 + (d % 32) * 16 + (d // 32) * 4 + (n % 128) // 32
 
 
 def select_workspace_bytes(shape: Shape) -> int:

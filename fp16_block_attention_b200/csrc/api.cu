@@ -129,6 +129,27 @@ thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thri
   return from_cuda(launch_quantize_qk(x, BH * s.N, s.N, s.D, codes, scales, cs));
 }
 
+thrift_status thrift_quant8_bytes(const thrift_shape* shape, thrift_operand op, size_t* codes_bytes,
+                                  size_t* scales_bytes) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (op != THRIFT_Q && op != THRIFT_K && op != THRIFT_V) return THRIFT_ERR_INVALID_ARG;
+  if (!codes_bytes || !scales_bytes) return THRIFT_ERR_INVALID_ARG;
+  *codes_bytes = mx8_codes_bytes(*shape, op);
+  *scales_bytes = mx8_scales_bytes(*shape, op);
+  return THRIFT_OK;
+}
+
+thrift_status thrift_quantize_mxfp8(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
+                                    void* scales, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (op != THRIFT_Q && op != THRIFT_K && op != THRIFT_V) return THRIFT_ERR_INVALID_ARG;
+  if (!x || !codes || !scales) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return THRIFT_ERR_INVALID_ARG;
+  return from_cuda(launch_quantize_mx8(x, op, *shape, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
 thrift_status thrift_select_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
   thrift_status st = check_shape(shape);
   if (st != THRIFT_OK) return st;

@@ -36,6 +36,12 @@ cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* c
                                cudaStream_t st);
 cudaError_t launch_quantize_v(const void* v, size_t bh, int N, int D, void* codes, void* scales, cudaStream_t st);
 
+// MXFP8 copies (quantize8.cu).
+size_t mx8_codes_bytes(const thrift_shape& s, thrift_operand op);
+size_t mx8_scales_bytes(const thrift_shape& s, thrift_operand op);
+cudaError_t launch_quantize_mx8(const void* x, thrift_operand op, const thrift_shape& s, void* codes, void* scales,
+                                cudaStream_t st);
+
 size_t select_workspace_bytes(const thrift_shape& s);
 // Size of the library's static selection scratch (thrift_select_blocks_static).
 constexpr size_t kSelectStaticBytes = size_t(16) << 20;

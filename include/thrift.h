@@ -104,6 +104,22 @@ THRIFT_API thrift_status thrift_quant_bytes(const thrift_shape* shape, thrift_op
 THRIFT_API thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
                                     void* scales, void* stream);
 
+/* MXFP8 copies for 8-bit block pairs (mask value 3 of the tiered selection),
+ * after TriAttention's 8-bit precision (abstract on the paper page of arXiv
+ * 2611.07256): the OCP microscaling format with E4M3 elements and one E8M0
+ * scale per 32 consecutive elements, X = 2^(floor(log2 amax) - 8); element =
+ * E4M3(v / X), nearest even, saturating at 448; an all-zero group has scale
+ * byte 0 and zero codes.  Q, K along D, V along keys.
+ * Codes: Q/K [B][H][N][D] bytes; V [B][Hkv][D][N] bytes (keys contiguous).
+ * Scales, NT = ceil(N/128), one 512-byte chunk per 128-row tile:
+ *   Q/K: byte (bh*NT + n/128)*512 + (n%32)*16 + ((n%128)/32)*4 + d/32;
+ *   V:   byte (bh*NT + n/128)*512 + (d%32)*16 + (d/32)*4 + (n%128)/32.
+ * Bytes no element maps to are 0.  Errors as for thrift_quantize_nvfp4. */
+THRIFT_API thrift_status thrift_quant8_bytes(const thrift_shape* shape, thrift_operand op, size_t* codes_bytes,
+                                             size_t* scales_bytes);
+THRIFT_API thrift_status thrift_quantize_mxfp8(const void* x, thrift_operand op, const thrift_shape* shape,
+                                               void* codes, void* scales, void* stream);
+
 /* Workspace bytes thrift_select_blocks and thrift_select_blocks_vertical_window
  * need (block means, pooled scores, column ranks). */
 THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape, size_t* bytes);
