@@ -77,7 +77,8 @@ def _load():
         "thrift_select_blocks": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_select_blocks_static": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
         "thrift_select_blocks_vertical_window": ([vp, vp, psh, ctypes.c_double, st, vp, vp, sz, vp], st),
-        "thrift_select_blocks_tiered": ([vp, vp, psh, ctypes.c_double, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_select_blocks_tiered": ([vp, vp, psh, ctypes.c_double, ctypes.c_double, ctypes.c_double, vp, vp, sz,
+                                         vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_attention_tiered": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
@@ -218,9 +219,10 @@ def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, 
 
 
 def select_blocks_tiered(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, sigma: float, mask=None,
-                         ws=None, stream=None):
-    """Tiered selection mask [B, Hq, nb, nb] (u8): 1 FP16, 0 NVFP4, 2 skipped
-    (the lowest-ranked pairs, never forced or FP16 ones)."""
+                         ws=None, stream=None, rho8: float = 0.0):
+    """Tiered selection mask [B, Hq, nb, nb] (u8): 1 FP16, 3 MXFP8 (the next
+    rho8 of the ranking), 0 NVFP4, 2 skipped (the lowest-ranked pairs, never
+    forced, FP16 or 8-bit ones)."""
     _dev(Qt, "Q", torch.float16)
     _dev(Kt, "K", torch.float16)
     if mask is None:
@@ -228,7 +230,7 @@ def select_blocks_tiered(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: 
     if ws is None:
         ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
     _check("thrift_select_blocks_tiered", _lib.thrift_select_blocks_tiered(
-        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), float(sigma), _ptr(mask), _ptr(ws), ws.numel(),
+        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(mask), _ptr(ws), ws.numel(),
         _stream(stream)))
     return mask
 

@@ -169,14 +169,17 @@ thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_sh
 }
 
 thrift_status thrift_select_blocks_tiered(const void* Q, const void* K, const thrift_shape* shape, double rho,
-                                          double sigma, uint8_t* mask, void* ws, size_t ws_bytes, void* stream) {
+                                          double rho8, double sigma, uint8_t* mask, void* ws, size_t ws_bytes,
+                                          void* stream) {
   thrift_status st = check_shape(shape);
   if (st != THRIFT_OK) return st;
-  if (!Q || !K || !mask || !(rho >= 0.0 && rho <= 1.0) || !(sigma >= 0.0 && sigma <= 1.0))
+  if (!Q || !K || !mask || !(rho >= 0.0 && rho <= 1.0) || !(rho8 >= 0.0 && rho8 <= 1.0) ||
+      !(sigma >= 0.0 && sigma <= 1.0))
     return THRIFT_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return THRIFT_ERR_INVALID_ARG;
   if (!ws || ws_bytes < select_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
-  return from_cuda(launch_select_tiered(Q, K, *shape, rho, sigma, mask, ws, static_cast<cudaStream_t>(stream)));
+  return from_cuda(
+      launch_select_tiered(Q, K, *shape, rho, rho8, sigma, mask, ws, static_cast<cudaStream_t>(stream)));
 }
 
 thrift_status thrift_select_blocks_vertical_window(const void* Q, const void* K, const thrift_shape* shape, double rho,

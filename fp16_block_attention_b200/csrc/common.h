@@ -49,9 +49,9 @@ cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shap
                                  cudaStream_t st);
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st);
-// Tiered selection (select.cu): mask 1 FP16, 0 NVFP4, 2 skipped.
-cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double sigma,
-                                 uint8_t* mask, void* ws, cudaStream_t st);
+// Tiered selection (select.cu): mask 1 FP16, 3 MXFP8, 0 NVFP4, 2 skipped.
+cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
+                                 double sigma, uint8_t* mask, void* ws, cudaStream_t st);
 // Vertical-line / local-window selector (select.cu); nb = N / blk <= kMaxVWBlocks.
 constexpr int kMaxVWBlocks = 2048;
 cudaError_t launch_select_vertical_window(const void* Q, const void* K, const thrift_shape& s, double rho, int window,

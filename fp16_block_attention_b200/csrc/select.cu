@@ -184,12 +184,14 @@ __global__ void __launch_bounds__(1024) column_rank_kernel(const float* __restri
 
 // One CTA (1024 threads) per (batch, query head).  VW = 0: the method's key;
 // VW = 1: the vertical-line / local-window key (column ranks in `rank`).
-// The first k pairs by key are marked 1; with keep < #valid the pairs after
-// the first `keep` are marked 2 (skipped; the caller keeps them clear of
-// forced and FP16 pairs), the rest 0.
+// The first k pairs by key are marked 1, the next ones up to the k8end-th 3
+// (8-bit); with keep < #valid the pairs after the first `keep` are marked 2
+// (skipped; the caller keeps them clear of forced, FP16 and 8-bit pairs), the
+// rest 0.
 template <int VW>
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int nb, int causal,
-                                                    long long k, long long keep, uint8_t* __restrict__ mask,
+                                                    long long k, long long k8end, long long keep,
+                                                    uint8_t* __restrict__ mask,
                                                     const int* __restrict__ rank, int window) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
@@ -255,6 +257,8 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
 
   const bool select_none = k <= 0, select_all = k >= valid;
   const uint64_t threshold = (select_none || select_all) ? 0ull : kth_largest(k);  // FP16: key >= threshold
+  const bool eight_any = k8end > k && k8end > 0 && k < valid, eight_all = k8end >= valid;
+  const uint64_t eight_from = (eight_any && !eight_all) ? kth_largest(k8end) : 0ull;  // 8-bit: key >= eight_from
   const bool skip_any = keep < valid;
   const uint64_t keep_from = (skip_any && keep > 0) ? kth_largest(keep) : 0ull;  // skipped: key < keep_from
   for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
@@ -264,6 +268,8 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
       const uint64_t key = key_of(sc[idx], i, j);
       if (!select_none && (select_all || key >= threshold))
         v = 1;
+      else if (eight_any && (eight_all || key >= eight_from))
+        v = 3;
       else if (skip_any && (keep <= 0 || key < keep_from))
         v = 2;
     }
@@ -315,8 +321,8 @@ cudaError_t launch_select_vertical_window(const void* Q, const void* K, const th
   SelectWs w = carve(ws, s);
   launch_pool_and_scores(Q, K, s, w, st);
   column_rank_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, w.rank);
-  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), valid_pairs(s), mask,
-                                               w.rank, window);
+  const long long k = budget_pairs(s, rho);
+  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, w.rank, window);
   return cudaGetLastError();
 }
 
@@ -325,24 +331,27 @@ cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, d
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
   launch_pool_and_scores(Q, K, s, w, st);
-  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, budget_pairs(s, rho), valid_pairs(s), mask,
-                                               nullptr, 0);
+  const long long k = budget_pairs(s, rho);
+  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, nullptr, 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double sigma,
-                                 uint8_t* mask, void* ws, cudaStream_t st) {
+cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
+                                 double sigma, uint8_t* mask, void* ws, cudaStream_t st) {
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
   launch_pool_and_scores(Q, K, s, w, st);
-  // skipped pairs: the last ks of the ranking, clear of the forced and FP16 pairs
+  // 8-bit pairs: the k8 after the FP16 ones; skipped pairs: the last ks of the
+  // ranking, clear of the forced, FP16 and 8-bit pairs
   const long long n = valid_pairs(s), k16 = budget_pairs(s, rho);
+  long long k8 = budget_pairs(s, rho8);
+  if (k8 > n - k16) k8 = n - k16;
   const long long forced = 2LL * nb - 1;  // the diagonal and key block 0, (0, 0) once
   long long ks = budget_pairs(s, sigma);
-  const long long cap = n - (k16 > forced ? k16 : forced);
+  const long long cap = n - (k16 + k8 > forced ? k16 + k8 : forced);
   if (ks > cap) ks = cap;
   if (ks < 0) ks = 0;
-  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k16, n - ks, mask, nullptr, 0);
+  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k16, k16 + k8, n - ks, mask, nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -133,21 +133,24 @@ THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape
 THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
                                    uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
 
-/* Stage 1 with a third class, skipped pairs, after TriAttention's tile
- * precisions (abstract on the paper page of arXiv 2611.07256: interactions
- * that matter least are skipped, the precision of the rest lowered).  The
- * method's ranking (as thrift_select_blocks) is cut in three per (batch,
- * query head):
+/* Stage 1 with two more classes, 8-bit and skipped pairs, after
+ * TriAttention's tile precisions (abstract on the paper page of arXiv
+ * 2611.07256: interactions that matter least are skipped, the precision of
+ * the rest lowered, 8-bit among the precisions).  The method's ranking (as
+ * thrift_select_blocks) is cut in four per (batch, query head):
  *   the first k16 = ceil(rho * #valid - 1e-9) pairs          -> 1 (FP16)
+ *   the next  k8  = min(ceil(rho8 * #valid - 1e-9),
+ *                       #valid - k16) pairs                  -> 3 (MXFP8)
  *   the last  ks  = min(ceil(sigma * #valid - 1e-9),
- *                       #valid - max(k16, 2 nb - 1)) pairs   -> 2 (skipped)
+ *                       #valid - max(k16 + k8, 2 nb - 1))    -> 2 (skipped)
  *   the others                                               -> 0 (NVFP4)
- * so the forced pairs (diagonal and key block 0, 2 nb - 1 of them) and the
- * FP16 pairs are never skipped; sigma = 0 gives thrift_select_blocks' mask.
- * thrift_attention_tiered treats a skipped pair as absent from the softmax.
- * Workspace, layout and errors as for thrift_select_blocks. */
+ * so the forced pairs (diagonal and key block 0, 2 nb - 1 of them), the FP16
+ * and the 8-bit pairs are never skipped; rho8 = sigma = 0 gives
+ * thrift_select_blocks' mask.  thrift_attention_tiered treats a skipped pair
+ * as absent from the softmax.  rho, rho8, sigma in [0, 1]; workspace, layout
+ * and errors as for thrift_select_blocks. */
 THRIFT_API thrift_status thrift_select_blocks_tiered(const void* Q, const void* K, const thrift_shape* shape,
-                                                     double rho, double sigma, uint8_t* mask, void* ws,
+                                                     double rho, double rho8, double sigma, uint8_t* mask, void* ws,
                                                      size_t ws_bytes, void* stream);
 
 /* An alternative stage 1 on the same FP16 budget, after HyQuant (abstract in

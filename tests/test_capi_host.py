@@ -64,6 +64,13 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert vw(fake, None, sh, 0.05, 2, fake, fake, 1 << 30, None) == 1
     assert vw(fake, fake, sh, -0.5, 2, fake, fake, 1 << 30, None) == 1
     assert vw(fake, fake, sh, 0.05, 2, fake, fake, 16, None) == 5
+    tr = lib.thrift_select_blocks_tiered
+    assert tr(fake, fake, sh, 0.05, 1.5, 0.1, fake, fake, 1 << 30, None) == 1    # rho8 out of range
+    assert tr(fake, fake, sh, 0.05, 0.1, -0.1, fake, fake, 1 << 30, None) == 1   # sigma out of range
+    assert tr(fake, fake, sh, 0.05, 0.1, 0.1, None, fake, 1 << 30, None) == 1
+    assert tr(fake, fake, sh, 0.05, 0.1, 0.1, fake, fake, 16, None) == 5
+    assert lib.thrift_quantize_mxfp8(fake, 3, sh, fake, fake, None) == 1
+    assert lib.thrift_quantize_mxfp8(fake, 0, sh, None, fake, None) == 1
     args = [fake] * 10
     assert lib.thrift_attention(None, *args[:9], sh, fake, None) == 1
     assert lib.thrift_attention_fused(fake, fake, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1

@@ -1,10 +1,10 @@
-"""Parity of the tiered selection (FP16 / NVFP4 / skip) and of attention with
+"""Parity of the tiered selection (FP16 / MXFP8 / NVFP4 / skip) and of attention with
 skipped pairs on the GPU (through the C ABI) with the oracle.
 
-Selection: exactly k16 FP16 pairs and ks skipped pairs per head; the masks
-agree except for pairs whose pooled score lies within 1e-5 (relative) of one
-of the two cuts (the lowest FP16 score of a non-forced pair, the highest
-skipped score), where FP32 summation order may swap neighbours.  Attention:
+Selection: exactly k16 FP16, k8 8-bit and ks skipped pairs per head; the
+masks agree except for pairs whose pooled score lies within 1e-5 (relative)
+of a score beside one of the three cuts of the ranking, where FP32 summation
+order may swap neighbours.  Attention:
 the oracle's mask given to the GPU, outputs within max-abs 2e-2 and mean-abs
 1e-3 of the oracle's (the prefill bars), where a row that misses the bar is
 re-checked against the oracle with its encoded P nudged by 2^-19 both ways
@@ -36,15 +36,28 @@ def _valid(nb, causal):
     return np.tril(np.ones((nb, nb), bool)) if causal else np.ones((nb, nb), bool)
 
 
-@pytest.mark.parametrize("rho,sigma", [(0.05, 0.25), (0.0, 0.6), (0.3, 0.5), (0.05, 1.0)])
+def _cut_scores(sc, nb, causal, cuts):
+    """Pooled scores on both sides of each cut position of the ranking (forced
+    pairs first, then score descending, then the lower linear index)."""
+    ii, jj = np.meshgrid(np.arange(nb), np.arange(nb), indexing="ij")
+    valid = _valid(nb, causal)
+    i, j, v = ii[valid], jj[valid], sc[valid]
+    order = np.lexsort((i * nb + j, -v, ~((i == j) | (j == 0))))
+    n = len(order)
+    return [v[order[k + d]] for k in cuts if 0 < k < n for d in (-1, 0)]
+
+
+@pytest.mark.parametrize("rho,rho8,sigma", [(0.05, 0.0, 0.25), (0.0, 0.0, 0.6), (0.3, 0.0, 0.5), (0.05, 0.0, 1.0),
+                                            (0.05, 0.1, 0.0), (0.05, 0.2, 0.5), (0.0, 0.3, 0.9), (0.02, 1.0, 0.0)])
 @pytest.mark.parametrize("w", CASES, ids=IDS)
-def test_tiered_select_matches_oracle(w, rho, sigma):
+def test_tiered_select_matches_oracle(w, rho, rho8, sigma):
     Q, K, _ = synth.generate(w)
     Qd, Kd = to_dev(Q, K)
-    m = thrift.select_blocks_tiered(Qd, Kd, shape_of(w), rho, sigma).cpu().numpy()
-    ref = oracle.select_tiered(Q, K, w.blk, w.causal, w.sm_scale, rho, sigma)
+    m = thrift.select_blocks_tiered(Qd, Kd, shape_of(w), rho, sigma, rho8=rho8).cpu().numpy()
+    ref = oracle.select_tiered(Q, K, w.blk, w.causal, w.sm_scale, rho, sigma, rho8)
     nb = w.N // w.blk
     valid = _valid(nb, w.causal)
+    n = int(valid.sum())
     forced = np.zeros((nb, nb), bool)
     forced[np.arange(nb), np.arange(nb)] = True
     forced[:, 0] = True
@@ -52,19 +65,16 @@ def test_tiered_select_matches_oracle(w, rho, sigma):
     for b in range(w.B):
         for h in range(w.Hq):
             mg, mo = m[b, h], ref[b, h]
-            assert (mg == 1).sum() == (mo == 1).sum() and (mg == 2).sum() == (mo == 2).sum()
+            for c in (1, 2, 3):
+                assert (mg == c).sum() == (mo == c).sum(), (b, h, c)
             assert not np.any((mg == 2) & forced) and not np.any((mg != 0) & ~valid)
             diff = mg != mo
             if not diff.any():
                 continue
             sc = oracle.pooled_scores(Q[b, h], K[b, h // G], w.blk, w.causal, w.sm_scale)
-            cuts = []
-            if np.any((mo == 1) & ~forced):
-                cuts.append(sc[(mo == 1) & ~forced].min())
-            if np.any(mo == 2):
-                cuts.append(sc[mo == 2].max())
+            k16, k8, ks = (int((mo == c).sum()) for c in (1, 3, 2))
             near = np.zeros_like(diff)
-            for c in cuts:
+            for c in _cut_scores(sc, nb, w.causal, (k16, k16 + k8, n - ks)):
                 near |= np.abs(sc - c) <= 1e-5 * max(abs(c), 1e-30)
             assert np.all(near[diff]), (b, h)
 
