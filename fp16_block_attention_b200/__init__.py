@@ -80,7 +80,7 @@ def _load():
         "thrift_select_blocks_tiered": ([vp, vp, psh, ctypes.c_double, ctypes.c_double, ctypes.c_double, vp, vp, sz,
                                          vp], st),
         "thrift_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
-        "thrift_attention_tiered": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp], st),
+        "thrift_attention_tiered": ([vp] * 16 + [psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_pool_keys": ([vp, psh, vp, vp], st),
@@ -302,17 +302,37 @@ def attention(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=No
     return out
 
 
-def attention_tiered(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None):
+@dataclasses.dataclass
+class Quantised8:
+    """MXFP8 copies of Q, K, V (codes and scales) for 8-bit pairs."""
+    q8: torch.Tensor
+    qs8: torch.Tensor
+    k8: torch.Tensor
+    ks8: torch.Tensor
+    v8: torch.Tensor
+    vs8: torch.Tensor
+
+
+def quantize_all_mxfp8(Qt, Kt, Vt, shape: Shape, stream=None) -> Quantised8:
+    q8, qs8 = quantize_mxfp8(Qt, Q, shape, stream=stream)
+    k8, ks8 = quantize_mxfp8(Kt, K, shape, stream=stream)
+    v8, vs8 = quantize_mxfp8(Vt, V, shape, stream=stream)
+    return Quantised8(q8, qs8, k8, ks8, v8, vs8)
+
+
+def attention_tiered(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None, q8: Quantised8 = None):
     """attention() for masks that may hold 2 (skipped pairs, absent from the
-    softmax), as from select_blocks_tiered."""
+    softmax) and, given the MXFP8 copies q8, 3 (8-bit pairs), as from
+    select_blocks_tiered."""
     for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
         _dev(t, n, torch.float16)
     _dev(mask, "mask", torch.uint8)
     if out is None:
         out = torch.empty_like(Qt)
+    p8 = [None] * 6 if q8 is None else [_ptr(t) for t in (q8.q8, q8.qs8, q8.k8, q8.ks8, q8.v8, q8.vs8)]
     _check("thrift_attention_tiered", _lib.thrift_attention_tiered(
         _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
-        _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
+        _ptr(qz.v4), _ptr(qz.vs), *p8, ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
     return out
 
 
@@ -411,7 +431,8 @@ def mma_rate_probe(kind: int, iters: int, stream=None):
 
 
 def last_device_error(stream=None) -> int:
-    """Synchronise and read/clear the device error word (0 = none, 4 = a bounded wait timed out)."""
+    """Synchronise and read/clear the device error word (0 = none, 4 = a bounded wait timed out,
+    1 = a kernel met a mask byte it cannot compute)."""
     return int(_lib.thrift_last_device_error(_stream(stream)))
 
 

@@ -5,6 +5,7 @@
 #include <cstdint>
 
 #include "common.h"
+#include "ptx.cuh"
 
 namespace thrift {
 
@@ -208,16 +209,22 @@ thrift_status thrift_select_blocks_static(const void* Q, const void* K, const th
 namespace {
 thrift_status attention_entry(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                               const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                              const thrift_shape* shape, void* O, bool skip, void* stream) {
+                              const thrift_shape* shape, void* O, bool skip, const Mx8Copies* eight, void* stream) {
   thrift_status st = check_shape(shape);
   if (st != THRIFT_OK) return st;
   const void* ptrs[] = {Q, K, V, q4, qs, k4, ks, v4, vs, O};
   for (const void* ptr : ptrs)
     if (!ptr || !aligned16(ptr)) return THRIFT_ERR_INVALID_ARG;
   if (!mask) return THRIFT_ERR_INVALID_ARG;
+  if (eight) {
+    const void* p8[] = {eight->q8, eight->qs8, eight->k8, eight->ks8, eight->v8, eight->vs8};
+    for (const void* ptr : p8)
+      if (!ptr || !aligned16(ptr)) return THRIFT_ERR_INVALID_ARG;
+    if (shape->blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  }
   uint32_t* err = device_error_word();
   if (!err) return THRIFT_ERR_CUDA;
-  return from_cuda(launch_attention(Q, K, V, mask, q4, qs, k4, ks, v4, vs, *shape, O, skip, err,
+  return from_cuda(launch_attention(Q, K, V, mask, q4, qs, k4, ks, v4, vs, *shape, O, skip, eight, err,
                                     static_cast<cudaStream_t>(stream)));
 }
 }  // namespace
@@ -225,13 +232,17 @@ thrift_status attention_entry(const void* Q, const void* K, const void* V, const
 thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
                                const thrift_shape* shape, void* O, void* stream) {
-  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, false, stream);
+  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, false, nullptr, stream);
 }
 
 thrift_status thrift_attention_tiered(const void* Q, const void* K, const void* V, const uint8_t* mask,
                                       const void* q4, const void* qs, const void* k4, const void* ks, const void* v4,
-                                      const void* vs, const thrift_shape* shape, void* O, void* stream) {
-  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, true, stream);
+                                      const void* vs, const void* q8, const void* qs8, const void* k8,
+                                      const void* ks8, const void* v8, const void* vs8, const thrift_shape* shape,
+                                      void* O, void* stream) {
+  const bool none = !q8 && !qs8 && !k8 && !ks8 && !v8 && !vs8;
+  const Mx8Copies eight = {q8, qs8, k8, ks8, v8, vs8};
+  return attention_entry(Q, K, V, mask, q4, qs, k4, ks, v4, vs, shape, O, true, none ? nullptr : &eight, stream);
 }
 
 thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape, size_t* bytes) {
@@ -262,7 +273,7 @@ thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V
   if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   if (launch_select(Q, K, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
-  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, false, err, cs));
+  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, false, nullptr, err, cs));
 }
 
 namespace {
@@ -342,7 +353,7 @@ thrift_status thrift_last_device_error(void* stream) {
   if (v != 0) {
     const uint32_t zero = 0;
     if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return THRIFT_ERR_CUDA;
-    return THRIFT_ERR_TIMEOUT;
+    return v == DEV_BAD_ARG ? THRIFT_ERR_INVALID_ARG : THRIFT_ERR_TIMEOUT;
   }
   return THRIFT_OK;
 }

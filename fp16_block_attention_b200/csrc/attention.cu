@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.blk == 128) {
       const uint8_t mv = mrow[static_cast<size_t>(qt) * nb + kt];
       c = SKIP ? ((mv == 1 ? 0xFu : 0u) | (mv == 2 ? 0xF0u : 0u)) : (mv ? 0xFu : 0u);
+      if (SKIP && mv > 2) record_error(p.err, DEV_BAD_ARG);  // 8-bit pairs need the 128-block kernel
     } else {
       for (int a = 0; a < 2; ++a)
         for (int k = 0; k < 2; ++k) {
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t mv = (i < nb && j < nb) ? mrow[static_cast<size_t>(i) * nb + j] : 0;
           if (SKIP ? mv == 1 : mv != 0) c |= 1u << (a * 2 + k);
           if (SKIP && mv == 2) c |= 1u << (4 + a * 2 + k);
+          if (SKIP && mv > 2) record_error(p.err, DEV_BAD_ARG);
         }
     }
     ms.cls[kt] = static_cast<uint8_t>(c);
@@ -559,8 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4, const void* qs,
                      const void* k4, const void* ks, const void* v4, const void* vs, const thrift_shape& s, void* O,
-                     bool skip, uint32_t* err, cudaStream_t st) {
+                     bool skip, const Mx8Copies* eight, uint32_t* err, cudaStream_t st) {
   CUtensorMap mQ16, mK16, mV16, mQ4, mK4, mV4;
+  CUtensorMap mQ8 = {}, mK8 = {}, mV8 = {};  // read only by the 8-bit instantiation
   const uint64_t BHq = static_cast<uint64_t>(s.B) * s.Hq, BHk = static_cast<uint64_t>(s.B) * s.Hkv;
   const CUtensorMapSwizzle sw4 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   bool ok = true;
@@ -570,6 +573,14 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   ok &= make_tmap_3d(&mQ4, q4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, s.N, BHq, D / 2, 128, sw4);
   ok &= make_tmap_3d(&mK4, k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D / 2, s.N, BHk, D / 2, 128, sw4);
   ok &= make_tmap_3d(&mV4, v4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.N / 2, D, BHk, 64, D, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (eight) {
+    // MXFP8 codes: Q / K rows of D bytes, V rows of N bytes (keys contiguous)
+    const CUtensorMapSwizzle sw8 = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    ok &= make_tmap_3d(&mQ8, eight->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, s.N, BHq, D, 128, sw8);
+    ok &= make_tmap_3d(&mK8, eight->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, s.N, BHk, D, 128, sw8);
+    ok &= make_tmap_3d(&mV8, eight->v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.N, D, BHk, 128, D,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  }
   if (!ok) return cudaErrorInvalidValue;
   Params prm;
   prm.mask = mask;
@@ -587,7 +598,12 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.NT = num_tiles(s.N);
   prm.scale_log2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
   prm.skip = skip ? 1 : 0;
-  if (s.blk == 128) return launch_attention_db<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
+  prm.qs8 = eight ? static_cast<const uint8_t*>(eight->qs8) : nullptr;
+  prm.ks8 = eight ? static_cast<const uint8_t*>(eight->ks8) : nullptr;
+  prm.vs8 = eight ? static_cast<const uint8_t*>(eight->vs8) : nullptr;
+  prm.eight = eight ? 1 : 0;
+  if (s.blk == 128) return launch_attention_db<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm, st);
+  if (eight) return cudaErrorInvalidValue;  // the entry point rejects this shape first
   const unsigned grid = static_cast<unsigned>(BHq * prm.NT);
   const size_t smem = Smem<D>::kBytes + 1024;
   const auto kern = skip ? thrift_attention_kernel<D, true> : thrift_attention_kernel<D, false>;
@@ -601,9 +617,10 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
 
 cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                             const thrift_shape& s, void* O, bool skip, uint32_t* err, cudaStream_t st) {
-  if (s.D == 128) return launch_d<128>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, err, st);
-  return launch_d<64>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, err, st);
+                             const thrift_shape& s, void* O, bool skip, const Mx8Copies* eight, uint32_t* err,
+                             cudaStream_t st) {
+  if (s.D == 128) return launch_d<128>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, eight, err, st);
+  return launch_d<64>(Q, K, V, mask, q4, qs, k4, ks, v4, vs, s, O, skip, eight, err, st);
 }
 
 }  // namespace thrift

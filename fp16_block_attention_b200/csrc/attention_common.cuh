@@ -21,6 +21,11 @@ struct Params {
   int B, Hq, Hkv, N, blk, causal, NT;
   float scale_log2;
   int skip;  // the mask may hold 2 (skipped pairs): the kernels' skip-aware instantiations
+  // MXFP8 scales of Q, K, V for 8-bit pairs (mask 3; blk = 128 only), or null
+  const uint8_t* qs8;
+  const uint8_t* ks8;
+  const uint8_t* vs8;
+  int eight;  // the MXFP8 copies are present: the 8-bit instantiation
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
@@ -126,10 +131,11 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }  // namespace attn
 
 // Kernel with double-buffered S and P for 128 x 128 selection blocks
-// (attention_db.cu).
+// (attention_db.cu).  The MXFP8 maps are read only when prm.eight is set.
 template <int D>
 cudaError_t launch_attention_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
                                 const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                                const CUtensorMap& mQ8, const CUtensorMap& mK8, const CUtensorMap& mV8,
                                 const attn::Params& prm, cudaStream_t st);
 
 }  // namespace thrift

@@ -27,6 +27,14 @@
 // sums meet once, in the epilogue.  Warp 8 is the TMA producer, 9 issues the
 // S products (and owns tensor memory), 10 issues the P V products.  The two
 // issuing threads and the softmax threads meet only through mbarriers.
+//
+// A third instantiation adds 8-bit pairs (mask 3, the MXFP8 copies of Q, K
+// and V): S from .kind::mxf8f6f4 products with E8M0 scales in tensor memory,
+// and P * 2^11 encoded per 32 keys as MXFP8 (E8M0 scale from the group's
+// maximum, E4M3 codes) into a 128-byte-swizzled shared-memory P buffer.  Its
+// K / V tiles share the fp16 tiles' slots and barriers; it keeps three NVFP4
+// ring slots instead of four to make room for the Q copy and the wider P
+// buffers.
 #include <cuda_fp16.h>
 
 #include "attention_common.cuh"
@@ -52,8 +60,12 @@ constexpr uint32_t kDColSFQ = 448;  // Q4 scales, 4 columns per 64-wide chunk of
 constexpr uint32_t kDColSFK = 456;  // K4 scales of the key tile being multiplied
 constexpr uint32_t kDColSFV = 464;  // V4 scales of the key tile being multiplied
 constexpr uint32_t kDColSFP = 472;  // P4 scales of P buffer b at 8 b: chunk c of row r at 4 c + r / 32
+                                    // (P8: keys 64 h .. 64 h + 63 of row r at 4 h + r / 32, one byte per 32 keys)
+constexpr uint32_t kDColSFQ8 = 488;  // Q8 scales (byte g: channels 32 g ..)
+constexpr uint32_t kDColSFK8 = 492;  // K8 scales of the key tile being multiplied
+constexpr uint32_t kDColSFV8 = 496;  // V8 scales (byte g: keys 32 g ..)
 
-template <int D>
+template <int D, bool EIGHT>
 struct SmemDB {
   static constexpr uint32_t kQ16Bytes = 128 * D * 2;
   static constexpr uint32_t kQ16 = 0;
@@ -61,24 +73,36 @@ struct SmemDB {
   static constexpr uint32_t kQ4 = kQ16 + kQ16Bytes;
   static constexpr uint32_t kQSFBytes = (D / 64) * 512;
   static constexpr uint32_t kQSF = kQ4 + kQ4Bytes;
-  static constexpr uint32_t kP4Bytes = 8192;  // 128 rows x 128 keys of E2M1, 64B-swizzled
+  // P buffer: 128 rows x 128 keys of E2M1 (64B-swizzled) or, with 8-bit
+  // pairs, of E4M3 (128B-swizzled)
+  static constexpr uint32_t kPBufBytes = EIGHT ? 16384 : 8192;
   static constexpr uint32_t kP4 = (kQSF + kQSFBytes + 1023) / 1024 * 1024;  // two buffers
+  static constexpr uint32_t kQ8Bytes = EIGHT ? 128 * D : 0;                 // Q8 tile, then its scales
+  static constexpr uint32_t kQ8 = kP4 + 2 * kPBufBytes;
+  static constexpr uint32_t kQS8Bytes = EIGHT ? 512 : 0;
+  static constexpr uint32_t kQS8 = kQ8 + kQ8Bytes;
   static constexpr uint32_t kK4Bytes = 128 * D / 2;
   static constexpr uint32_t kV4Bytes = D * 64;
   static constexpr uint32_t kKSFBytes = (D / 64) * 512;
   static constexpr uint32_t kVSFBytes = 1024;
   static constexpr uint32_t kSlot4Bytes = (kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes + 1023) / 1024 * 1024;
-  static constexpr uint32_t kSlot4 = kP4 + 2 * kP4Bytes;
-  static constexpr int kNS = 4;  // NVFP4 K/V ring slots
+  static constexpr uint32_t kSlot4 = (kQS8 + kQS8Bytes + 1023) / 1024 * 1024;
+  static constexpr int kNS = EIGHT ? 3 : 4;  // NVFP4 K/V ring slots
   static constexpr uint32_t kK16Bytes = 128 * D * 2;
   static constexpr uint32_t kSlot16 = kSlot4 + kNS * kSlot4Bytes;  // K16 then V16
   static constexpr uint32_t kMisc = kSlot16 + 2 * kK16Bytes;
   static constexpr uint32_t kBytes = kMisc + 4096;
   static constexpr uint32_t kTx4 = kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes;
   static constexpr uint32_t kTx16 = kK16Bytes;
-  static constexpr uint32_t kTxQ = kQ16Bytes + kQ4Bytes + kQSFBytes;
+  static constexpr uint32_t kTxQ = kQ16Bytes + kQ4Bytes + kQSFBytes + kQ8Bytes + kQS8Bytes;
+  // 8-bit K / V tiles in the fp16 slots, each followed by its 512 scale bytes
+  static constexpr uint32_t kK8Bytes = 128 * D;  // 128 keys x D channels
+  static constexpr uint32_t kV8Bytes = D * 128;  // D channels x 128 keys
+  static constexpr uint32_t kTx8 = kK8Bytes + 512;
+  static_assert(kK8Bytes + 512 <= kK16Bytes && kV8Bytes + 512 <= kK16Bytes, "8-bit tiles must fit the fp16 slots");
   static_assert(kBytes + 1024 <= 232448, "shared memory above the 227 KB per-CTA limit");
-  static_assert(kQ4 % 1024 == 0 && kSlot4 % 1024 == 0 && kSlot16 % 1024 == 0, "TMA tiles need 1 KB alignment");
+  static_assert(kQ4 % 1024 == 0 && kSlot4 % 1024 == 0 && kSlot16 % 1024 == 0 && kQ8 % 1024 == 0,
+                "TMA tiles need 1 KB alignment");
 };
 
 struct MiscDB {
@@ -95,7 +119,7 @@ struct MiscDB {
   float lsum[2][128];  // partial row sums of the two halves, for the epilogue
   union {
     uint8_t cls[1024];   // SKIP = false: per key tile, 1 = FP16, 0 = NVFP4
-    uint16_t lst[1024];  // SKIP = true: key tiles to process in order, tile index | 0x8000 for FP16
+    uint16_t lst[1024];  // SKIP = true: key tiles to process in order, tile index | 0x8000 FP16 | 0x4000 8-bit
   };
   int np;                // key tiles processed
 };
@@ -103,15 +127,20 @@ static_assert(sizeof(MiscDB) <= 4096, "barriers must fit their shared-memory sli
 
 // SKIP = false: masks of 0 / 1 (the method); every key tile of the query
 // tile is processed.  SKIP = true: masks may hold 2 (skipped pairs); the
-// skipped tiles are left out of an ordered list that every role walks.  The
-// two are separate instantiations so the first keeps its own code.
-template <int D, bool SKIP>
+// skipped tiles are left out of an ordered list that every role walks.
+// EIGHT = true (with SKIP): masks may also hold 3, 8-bit pairs.  They are
+// separate instantiations so the method's keeps its own code.  A mask byte
+// the instantiation does not know records DEV_BAD_ARG (the tile is then
+// computed in NVFP4).
+template <int D, bool SKIP, bool EIGHT>
 __global__ void __launch_bounds__(kDBThreads, 1)
     thrift_attention_db_kernel(const __grid_constant__ CUtensorMap mQ16, const __grid_constant__ CUtensorMap mK16,
                                const __grid_constant__ CUtensorMap mV16, const __grid_constant__ CUtensorMap mQ4,
                                const __grid_constant__ CUtensorMap mK4, const __grid_constant__ CUtensorMap mV4,
-                               const Params p) {
-  using L = SmemDB<D>;
+                               const __grid_constant__ CUtensorMap mQ8, const __grid_constant__ CUtensorMap mK8,
+                               const __grid_constant__ CUtensorMap mV8, const Params p) {
+  static_assert(SKIP || !EIGHT, "8-bit pairs come with the skip-aware list");
+  using L = SmemDB<D, EIGHT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   MiscDB& ms = *reinterpret_cast<MiscDB*>(sm + L::kMisc);
@@ -152,22 +181,25 @@ __global__ void __launch_bounds__(kDBThreads, 1)
   }
   if constexpr (SKIP) {
     if (warp == 0) {
-      // Key tiles to process in increasing order: mask 1 FP16, 0 NVFP4, 2
-      // skipped (left out).  All of the row's mask bytes are loaded at once
-      // (nk <= 1024 = 32 x 32), then compacted in order from registers.
+      // Key tiles to process in increasing order: mask 1 FP16, 3 8-bit, 0
+      // NVFP4, 2 skipped (left out).  All of the row's mask bytes are loaded
+      // at once (nk <= 1024 = 32 x 32), then compacted in order from registers.
       const uint8_t* m0 = p.mask + static_cast<size_t>(bh) * nb * nb + static_cast<size_t>(qt) * nb;
       uint8_t mv[32];
 #pragma unroll
       for (int q = 0; q < 32; ++q) mv[q] = (q * 32 + lane < nk) ? m0[q * 32 + lane] : 2;
       int base = 0;
+      bool bad = false;
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
         const uint32_t keep = __ballot_sync(0xffffffffu, mv[q] != 2);
+        bad |= mv[q] > (EIGHT ? 3 : 2);
         if (mv[q] != 2)
-          ms.lst[base + __popc(keep & ((1u << lane) - 1u))] =
-              static_cast<uint16_t>((q * 32 + lane) | (mv[q] == 1 ? 0x8000 : 0));
+          ms.lst[base + __popc(keep & ((1u << lane) - 1u))] = static_cast<uint16_t>(
+              (q * 32 + lane) | (mv[q] == 1 ? 0x8000 : 0) | ((EIGHT && mv[q] == 3) ? 0x4000 : 0));
         base += __popc(keep);
       }
+      if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(p.err, DEV_BAD_ARG);
       if (lane == 0) ms.np = base;
     }
   } else {
@@ -182,6 +214,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
   // the it-th processed key tile and its precision
   const auto tile_of = [&](int it) -> int { return SKIP ? (ms.lst[it] & 0x3FF) : it; };
   const auto fp16_of = [&](int it) -> bool { return SKIP ? (ms.lst[it] & 0x8000) != 0 : ms.cls[it] != 0; };
+  const auto eight_of = [&](int it) -> bool { return EIGHT && (ms.lst[it] & 0x4000) != 0; };
 
   if (warp == kDBProducer) {
     // ======================== producer ========================
@@ -189,15 +222,23 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       prefetch_tensormap(&mQ16);
       prefetch_tensormap(&mK4);
       prefetch_tensormap(&mV4);
+      if constexpr (EIGHT) {
+        prefetch_tensormap(&mK8);
+        prefetch_tensormap(&mV8);
+      }
       mbar_arrive_expect_tx(&ms.bar_q, L::kTxQ);
       for (int pnl = 0; pnl < D / 64; ++pnl)
         tma_load_3d(sm + L::kQ16 + pnl * 16384, &mQ16, &ms.bar_q, pnl * 64, qt * 128, bh);
       tma_load_3d(sm + L::kQ4, &mQ4, &ms.bar_q, 0, qt * 128, bh);
       bulk_load(sm + L::kQSF, p.qs + (static_cast<size_t>(bh) * p.NT + qt) * L::kQSFBytes, L::kQSFBytes, &ms.bar_q);
+      if constexpr (EIGHT) {
+        tma_load_3d(sm + L::kQ8, &mQ8, &ms.bar_q, 0, qt * 128, bh);
+        bulk_load(sm + L::kQS8, p.qs8 + (static_cast<size_t>(bh) * p.NT + qt) * 512, 512, &ms.bar_q);
+      }
       int u4 = 0, u16 = 0;
       for (int it = 0; it < np && !ms.abort; ++it) {
         const int kt = tile_of(it);
-        if (!fp16_of(it)) {
+        if (!fp16_of(it) && !eight_of(it)) {
           const int slot = u4 % L::kNS, use = u4 / L::kNS;
           if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
@@ -211,19 +252,34 @@ __global__ void __launch_bounds__(kDBThreads, 1)
                     p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * kt) * 512, L::kVSFBytes, &ms.bar_full4[slot]);
           ++u4;
         } else {
+          // fp16 or 8-bit tile: the same two slots and barriers
+          const bool eight = eight_of(it);
           uint8_t* st = sm + L::kSlot16;
           if (u16 > 0 && !wait_or_abort(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
-          mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
-          for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
+          if (EIGHT && eight) {
+            mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx8);
+            tma_load_3d(st, &mK8, &ms.bar_full_k16, 0, kt * 128, bhk);
+            bulk_load(st + L::kK8Bytes, p.ks8 + (static_cast<size_t>(bhk) * p.NT + kt) * 512, 512, &ms.bar_full_k16);
+          } else {
+            mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
+            for (int pnl = 0; pnl < D / 64; ++pnl)
+              tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
+          }
           if (u16 > 0 && !wait_or_abort(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
-            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K16 copy of this tile is in flight
+            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K copy of this tile is in flight
             break;
           }
-          mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
-          for (int pnl = 0; pnl < D / 64; ++pnl)
-            tma_load_3d(st + L::kK16Bytes + pnl * 16384, &mV16, &ms.bar_full_v16, pnl * 64, kt * 128, bhk);
+          if (EIGHT && eight) {
+            mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx8);
+            tma_load_3d(st + L::kK16Bytes, &mV8, &ms.bar_full_v16, kt * 128, 0, bhk);
+            bulk_load(st + L::kK16Bytes + L::kV8Bytes, p.vs8 + (static_cast<size_t>(bhk) * p.NT + kt) * 512, 512,
+                      &ms.bar_full_v16);
+          } else {
+            mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
+            for (int pnl = 0; pnl < D / 64; ++pnl)
+              tma_load_3d(st + L::kK16Bytes + pnl * 16384, &mV16, &ms.bar_full_v16, pnl * 64, kt * 128, bhk);
+          }
           ++u16;
         }
       }
@@ -244,15 +300,17 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
       bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
       tc_fence_after();
-      if (ok)
+      if (ok) {
         for (int c = 0; c < D / 64; ++c)
           tmem_cp_32x128b_x4(tm + kDColSFQ + 4 * c, make_sdesc(sbase + L::kQSF + 512 * c, 16, 128, LAYOUT_NONE));
+        if constexpr (EIGHT) tmem_cp_32x128b_x4(tm + kDColSFQ8, make_sdesc(sbase + L::kQS8, 16, 128, LAYOUT_NONE));
+      }
       int u4 = 0, uk16 = 0;
       for (int it = 0; ok && it < np; ++it) {
         const int bb = it & 1;
-        const bool fp16 = fp16_of(it);
+        const bool fp16 = fp16_of(it), eight = eight_of(it);
         int slot = 0;
-        if (!fp16) {
+        if (!fp16 && !eight) {
           slot = u4 % L::kNS;
           if (!(ok = wait_or_abort(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++u4;
@@ -264,6 +322,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           if (!(ok = wait_or_abort(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uk16;
           tc_fence_after();
+          if (EIGHT && eight)
+            tmem_cp_32x128b_x4(tm + kDColSFK8,
+                               make_sdesc(sbase + L::kSlot16 + L::kK8Bytes, 16, 128, LAYOUT_NONE));
         }
         // Buffers bb were last used by key tile kt - 2: wait until its S was
         // loaded by the softmax threads, and until its P V product is done, so
@@ -278,7 +339,16 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           tc_fence_after();
         }
         const uint32_t dS = tm + kDColS + 128 * bb;
-        if (!fp16) {
+        if (EIGHT && eight) {
+          // MXFP8 along D: K = 32 per product, scale byte kk of each row's column
+          constexpr uint32_t sbo8 = (D == 128) ? 1024u : 512u;
+          constexpr uint32_t sw8 = (D == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
+          const uint32_t q8 = sbase + L::kQ8, k8 = sbase + L::kSlot16;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_mxf8(dS, make_sdesc(q8 + 32 * kk, 16, sbo8, sw8), make_sdesc(k8 + 32 * kk, 16, sbo8, sw8),
+                     idesc_mxf8(128, 128, kk, kk), tm + kDColSFQ8, tm + kDColSFK8, kk > 0);
+        } else if (!fp16) {
           const uint32_t q4 = sbase + L::kQ4;
           const uint32_t k4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
 #pragma unroll
@@ -296,7 +366,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
         mma_commit(&ms.bar_s_full[bb]);
         // the K operands of this key tile are no longer needed (V: the P V issuer)
-        if (!fp16)
+        if (!fp16 && !eight)
           mma_commit(&ms.bar_empty4[slot]);
         else
           mma_commit(&ms.bar_empty_k16);
@@ -314,14 +384,14 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       uint32_t acc = 0u;
       for (int it = 0; ok && it < np; ++it) {
         const int bb = it & 1;
-        const bool fp16 = fp16_of(it);
+        const bool fp16 = fp16_of(it), eight = eight_of(it);
         // The V operands (and the V4 scales, copied to tensor memory) do not
         // depend on P, so they are made ready before waiting for it.  The copy
         // follows the previous P V product in this thread's tcgen05 order, so
         // it cannot overwrite scales that product still reads.
         int slot = 0;
         uint32_t v4 = 0;
-        if (!fp16) {
+        if (!fp16 && !eight) {
           slot = u4 % L::kNS;
           const int use = u4 / L::kNS;
           ++u4;
@@ -338,12 +408,30 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         } else {
           if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uv16;
+          if (EIGHT && eight) {
+            tc_fence_after();
+            tmem_cp_32x128b_x4(tm + kDColSFV8, make_sdesc(sbase + L::kSlot16 + L::kK16Bytes + L::kV8Bytes, 16, 128,
+                                                          LAYOUT_NONE));
+          }
         }
         if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
         tc_fence_after();
         const uint32_t dO = tm + kDColO;
-        if (!fp16) {
-          const uint32_t p4s = sbase + L::kP4 + bb * L::kP4Bytes;
+        if (EIGHT && eight) {
+          // P8 (128 x 128 keys, 128B-swizzled) times V8 (D x 128 keys): K = 32
+          // per product; P's scale for keys 32 kk .. is byte kk % 2 of column
+          // 4 (kk / 2) + r / 32, V's byte kk of column d / 32
+          const uint32_t p8s = sbase + L::kP4 + bb * L::kPBufBytes;
+          const uint32_t v8 = sbase + L::kSlot16 + L::kK16Bytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_mxf8(dO, make_sdesc(p8s + 32 * kk, 16, 1024, LAYOUT_SW128),
+                     make_sdesc(v8 + 32 * kk, 16, 1024, LAYOUT_SW128), idesc_mxf8(128, D, kk & 1, kk),
+                     tm + kDColSFP + 8 * bb + 4 * (kk >> 1), tm + kDColSFV8, acc);
+            acc = 1;
+          }
+        } else if (!fp16) {
+          const uint32_t p4s = sbase + L::kP4 + bb * L::kPBufBytes;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             mma_nvf4(dO, make_sdesc(p4s + 32 * c, 16, 512, LAYOUT_SW64), make_sdesc(v4 + 32 * c, 16, 512, LAYOUT_SW64),
@@ -360,7 +448,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           }
         }
         mma_commit(&ms.bar_o_done[bb]);
-        if (!fp16)
+        if (!fp16 && !eight)
           mma_commit(&ms.bar_empty4[slot]);
         else
           mma_commit(&ms.bar_empty_v16);
@@ -390,7 +478,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     for (int it = 0; it < np; ++it) {
       const int bb = it & 1;
       const int kt = tile_of(it);
-      const bool fp16 = fp16_of(it);
+      const bool fp16 = fp16_of(it), eight = eight_of(it);
       if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) {
@@ -450,7 +538,22 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // (independent chains, ahead of the exponentials).
       float sce[4], bias[4];
       uint32_t sfw = 0u;
-      if (!fp16) {
+      if (EIGHT && eight) {
+        // MXFP8 group scales of this half's two 32-key groups: X = 2^(floor(
+        // log2 amax) - 8) from the exponent field of amax = max of P * 2^11,
+        // E8M0 byte = that exponent - 8 (biased), clamped at 0.  A group whose
+        // byte would be 0 (amax below 2^-118, P below 2^-129) is encoded as
+        // zeros; the codes are E4M3(P * 2^11 / X) with -log2 X in the bias.
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float amax = ex2(fmaf(fmaxf(gh[2 * c], gh[2 * c + 1]), c2, base));
+          const int eb = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+          const bool live = eb > 8;
+          sce[c] = live ? __uint_as_float(static_cast<uint32_t>(eb - 8) << 23) : 0.f;  // X
+          bias[c] = live ? base + static_cast<float>(135 - eb) : -INFINITY;
+          sfw |= static_cast<uint32_t>(live ? eb - 8 : 0) << (8 * c);
+        }
+      } else if (!fp16) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const float amax = ex2(fmaf(gh[g], c2, base));                         // max of P * 2^11
@@ -494,8 +597,33 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
         rs = (sum16(&s[0]) + sum16(&s[16])) + (sum16(&s[32]) + sum16(&s[48]));
         tmem_st32(lane_base + kDColP16 + 32 * half, w);
+      } else if (EIGHT && eight) {
+        uint8_t* d8 = sm + L::kP4 + bb * L::kPBufBytes;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float2 bv = make_float2(bias[c], bias[c]);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float2 pp = ex2_fma2(s[32 * c + i], s[32 * c + i + 1], c2v, bv);
+            s[32 * c + i] = pp.x;
+            s[32 * c + i + 1] = pp.y;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) rs = fmaf(sum16(&s[32 * c]) + sum16(&s[32 * c + 16]), sce[c], rs);
+        // 16 keys per 16-byte chunk; this half's keys are chunks 4 h .. 4 h + 3
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w[i] = (cvt_e4m3x2(s[16 * q + 4 * i], s[16 * q + 4 * i + 1]) & 0xFFFFu) |
+                   (cvt_e4m3x2(s[16 * q + 4 * i + 2], s[16 * q + 4 * i + 3]) << 16);
+          *reinterpret_cast<uint4*>(d8 + sw128_off(r, 4 * half + q)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        tmem_st1(lane_base + kDColSFP + 8 * bb + 4 * half + quad, sfw);
       } else {
-        uint8_t* d4 = sm + L::kP4 + bb * L::kP4Bytes;
+        uint8_t* d4 = sm + L::kP4 + bb * L::kPBufBytes;
         // exponentials with 1/scale folded in, then sums and codes
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -597,32 +725,38 @@ __global__ void __launch_bounds__(kDBThreads, 1)
 
 }  // namespace
 
-template <int D, bool SKIP>
+template <int D, bool SKIP, bool EIGHT>
 static cudaError_t launch_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
                              const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                             const CUtensorMap& mQ8, const CUtensorMap& mK8, const CUtensorMap& mV8,
                              const attn::Params& prm, cudaStream_t st) {
-  const size_t smem = SmemDB<D>::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(thrift_attention_db_kernel<D, SKIP>,
+  const size_t smem = SmemDB<D, EIGHT>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(thrift_attention_db_kernel<D, SKIP, EIGHT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(prm.B * prm.Hq * prm.NT);
-  thrift_attention_db_kernel<D, SKIP><<<grid, kDBThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm);
+  thrift_attention_db_kernel<D, SKIP, EIGHT>
+      <<<grid, kDBThreads, smem, st>>>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_attention_db(const CUtensorMap& mQ16, const CUtensorMap& mK16, const CUtensorMap& mV16,
                                 const CUtensorMap& mQ4, const CUtensorMap& mK4, const CUtensorMap& mV4,
+                                const CUtensorMap& mQ8, const CUtensorMap& mK8, const CUtensorMap& mV8,
                                 const attn::Params& prm, cudaStream_t st) {
-  if (prm.skip) return launch_db<D, true>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
-  return launch_db<D, false>(mQ16, mK16, mV16, mQ4, mK4, mV4, prm, st);
+  if (prm.eight) return launch_db<D, true, true>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm, st);
+  if (prm.skip) return launch_db<D, true, false>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm, st);
+  return launch_db<D, false, false>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm, st);
 }
 
-template cudaError_t launch_attention_db<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                             const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                             const attn::Params&, cudaStream_t);
-template cudaError_t launch_attention_db<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                              const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+#define THRIFT_DB_INSTANCE(D)                                                                                        \
+  template cudaError_t launch_attention_db<D>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,          \
+                                              const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,          \
+                                              const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,          \
                                               const attn::Params&, cudaStream_t);
+THRIFT_DB_INSTANCE(64)
+THRIFT_DB_INSTANCE(128)
+#undef THRIFT_DB_INSTANCE
 
 }  // namespace thrift

@@ -83,9 +83,17 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
 // Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
 cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);
 
-// skip: the mask may hold 2 (skipped pairs); selects the kernels' skip-aware instantiations.
+// MXFP8 copies of Q, K, V (codes and scales, as launch_quantize_mx8 writes them).
+struct Mx8Copies {
+  const void *q8, *qs8, *k8, *ks8, *v8, *vs8;
+};
+
+// skip: the mask may hold 2 (skipped pairs); selects the kernels' skip-aware
+// instantiations.  eight: null, or the MXFP8 copies for masks that may hold 3
+// (8-bit pairs; blk = 128 only).
 cudaError_t launch_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                              const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
-                             const thrift_shape& s, void* O, bool skip, uint32_t* err, cudaStream_t st);
+                             const thrift_shape& s, void* O, bool skip, const Mx8Copies* eight, uint32_t* err,
+                             cudaStream_t st);
 
 }  // namespace thrift

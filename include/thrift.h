@@ -209,16 +209,29 @@ THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const vo
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
                                const thrift_shape* shape, void* O, void* stream);
 
-/* thrift_attention for masks that may also hold 2, as written by
- * thrift_select_blocks_tiered: a skipped pair is absent from the softmax
+/* thrift_attention for masks that may also hold 2 and 3, as written by
+ * thrift_select_blocks_tiered.  A skipped pair (2) is absent from the softmax
  * (every query row must keep at least one key; the tiered selection never
  * skips the diagonal).  With blk = 128 the skipped key tiles are left out of
  * the kernel's work; with blk = 64 a skipped block inside a 128-key tile is
- * computed and masked.  Arguments and errors as for thrift_attention. */
+ * computed and masked.  An 8-bit pair (3) takes S from the MXFP8 copies of Q
+ * and K, encodes P * 2^11 as MXFP8 per aligned group of 32 keys (E8M0 scale
+ * 2^(floor(log2 amax) - 8) of the group's maximum, E4M3 codes; a group whose
+ * scale byte would be 0 is encoded as zeros) and multiplies it with the
+ * MXFP8 copy of V.
+ *   q8, qs8, k8, ks8, v8, vs8: the MXFP8 copies from thrift_quantize_mxfp8
+ *     (Q with THRIFT_Q, K with THRIFT_K, V with THRIFT_V), all six or none
+ *     (THRIFT_ERR_INVALID_ARG otherwise); with them blk must be 128
+ *     (THRIFT_ERR_UNSUPPORTED otherwise).
+ * A mask byte the call cannot compute (3 without the copies, above 3) makes
+ * thrift_last_device_error() return THRIFT_ERR_INVALID_ARG; that tile is
+ * then computed in NVFP4.  Other arguments and errors as for
+ * thrift_attention. */
 THRIFT_API thrift_status thrift_attention_tiered(const void* Q, const void* K, const void* V, const uint8_t* mask,
                                                  const void* q4, const void* qs, const void* k4, const void* ks,
-                                                 const void* v4, const void* vs, const thrift_shape* shape, void* O,
-                                                 void* stream);
+                                                 const void* v4, const void* vs, const void* q8, const void* qs8,
+                                                 const void* k8, const void* ks8, const void* v8, const void* vs8,
+                                                 const thrift_shape* shape, void* O, void* stream);
 
 /* Workspace bytes of thrift_attention_fused (NVFP4 copies, mask and the
  * selection workspace, each 256-byte aligned). */
@@ -276,8 +289,10 @@ THRIFT_API thrift_status thrift_decode_step(const void* q, const void* K, const 
                                             size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read and clear the device error word of the current
- * device: THRIFT_OK, or THRIFT_ERR_TIMEOUT if a kernel gave up a bounded wait
- * since the last call, or THRIFT_ERR_CUDA if the synchronisation failed. */
+ * device: THRIFT_OK; THRIFT_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call; THRIFT_ERR_INVALID_ARG if a kernel met a mask byte it
+ * cannot compute; THRIFT_ERR_CUDA if the synchronisation failed.  The word
+ * keeps the first error recorded. */
 THRIFT_API thrift_status thrift_last_device_error(void* stream);
 
 /* Measurement helper, not part of the method (the pages have no counterpart):

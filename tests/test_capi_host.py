@@ -71,6 +71,10 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert tr(fake, fake, sh, 0.05, 0.1, 0.1, fake, fake, 16, None) == 5
     assert lib.thrift_quantize_mxfp8(fake, 3, sh, fake, fake, None) == 1
     assert lib.thrift_quantize_mxfp8(fake, 0, sh, None, fake, None) == 1
+    at = lib.thrift_attention_tiered
+    assert at(*[fake] * 10, fake, None, fake, fake, fake, fake, sh, fake, None) == 1        # some copies missing
+    assert at(*[fake] * 10, fake, ctypes.c_void_p(264), fake, fake, fake, fake, sh, fake, None) == 1  # misaligned
+    assert at(*[fake] * 16, ctypes.byref(_c(blk=64)), fake, None) == 2                      # 8-bit needs blk 128
     args = [fake] * 10
     assert lib.thrift_attention(None, *args[:9], sh, fake, None) == 1
     assert lib.thrift_attention_fused(fake, fake, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1
