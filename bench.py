@@ -39,6 +39,7 @@ WORKLOAD = synth.GQA_N32K
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
+FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 PF / 2.25 PF)
 PROFILE_FILE = os.path.join(ROOT, "profiles", "attention_gqa_n32k_traffic.json")
 KERNEL_SOURCES = ["attention.cu", "attention_db.cu", "attention_common.cuh", "ptx.cuh", "tmap.h"]
 LAUNCHES_PER_STEP = 8        # quantize Q, K, V; pool Q, K; scores; top-k; attention
@@ -153,31 +154,36 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def flop_split(w, mask_np):
-    """Effective FLOPs of the FP16 and FP4 block pairs (diagonal pairs count their
-    causal triangle), from the selection mask [B, Hq, nb, nb] (1 FP16, 0 NVFP4,
-    2 skipped: not computed, counted in neither)."""
+def pair_flops(w, mask_np, cls):
+    """Effective FLOPs of the block pairs of one class of the selection mask
+    [B, Hq, nb, nb] (1 FP16, 3 MXFP8, 0 NVFP4, 2 skipped: not computed);
+    diagonal pairs count their causal triangle."""
     nb = w.N // w.blk
     full = 4.0 * w.blk * w.blk * w.D
     diag = 4.0 * w.D * w.blk * (w.blk + 1) / 2 if w.causal else full
     eye = np.eye(nb, dtype=bool)
     valid = np.tril(np.ones((nb, nb), bool)) if w.causal else np.ones((nb, nb), bool)
     weight = np.where(eye, diag, full) * valid
-    f16 = float((weight[None, None] * (mask_np == 1)).sum())
-    f4 = float((weight[None, None] * (mask_np == 0)).sum())
-    return f16, f4
+    return float((weight[None, None] * (mask_np == cls)).sum())
+
+
+def flop_split(w, mask_np):
+    """Effective FLOPs of the FP16 and the NVFP4 block pairs."""
+    return pair_flops(w, mask_np, 1), pair_flops(w, mask_np, 0)
 
 
 MUFU_PER_CLK_PER_SM = 16  # ex2 / lg2 throughput of compute capability 10.0 (16 per clock per SM)
 
 
 def mufu_ops(w, mask_np):
-    """MUFU operations the method needs at least: one exponential per valid
-    (query, key) pair, and per 16-key NVFP4 group of P one exponential (the
-    group maximum) and one logarithm (its scale)."""
+    """MUFU operations the method needs at least: one exponential per computed
+    (query, key) pair, per 16-key NVFP4 group of P one exponential (the group
+    maximum) and one logarithm (its scale), per 32-key MXFP8 group of P one
+    exponential (the group maximum)."""
     f16, f4 = flop_split(w, mask_np)
+    f8 = pair_flops(w, mask_np, 3)
     per_elem = 4.0 * w.D
-    return (f16 + f4) / per_elem + (f4 / per_elem) * 2.0 / 16.0
+    return (f16 + f4 + f8) / per_elem + (f4 / per_elem) * 2.0 / 16.0 + (f8 / per_elem) / 32.0
 
 
 def mufu_ceiling(w, mask_np, attn_ms, sm_mhz, n_sm):
@@ -376,6 +382,19 @@ def attention_bytes(w, mask_np):
             q_tiles16 * w.blk * w.D * 2 + 2 * e_q + mask_np.size)
 
 
+def eight_bytes(w, mask_np):
+    """Algorithmic HBM bytes the 8-bit pairs add to attention_bytes: the MXFP8
+    copies (1 B code + 1/32 B scale per element) of the K and V tiles that some
+    query head of their group computes in 8 bits and of the Q tiles with an
+    8-bit pair, once each."""
+    nb = w.N // w.blk
+    G = w.Hq // w.Hkv
+    m = mask_np.reshape(w.B, w.Hkv, G, nb, nb) == 3
+    kv_tiles8 = int(m.any(axis=(2, 3)).sum())
+    q_tiles8 = int(m.any(axis=4).sum())
+    return (1.0 + 1.0 / 32.0) * (kv_tiles8 * 2 + q_tiles8) * w.blk * w.D
+
+
 # --------------------------------------------------------- the CPU oracle ---
 class OracleRows:
     """The oracle (plain C, FP64, OpenMP over rows) on a bounded sample of the
@@ -547,6 +566,8 @@ def run_sweep(args):
         torch.cuda.empty_cache()
     print()
     run_skip_sweep(args, dev, peaks, n_sm)
+    print()
+    run_eight_sweep(args, dev, peaks, n_sm)
 
 
 def run_skip_sweep(args, dev, peaks, n_sm):
@@ -592,6 +613,58 @@ def run_skip_sweep(args, dev, peaks, n_sm):
         print(f"| {sigma:g} | {ms:.4f} | {w.flops() / (ms * 1e-3) / 1e12:.1f} | "
               f"{(f16 + f4) / (ms * 1e-3) / 1e12:.1f} | {t_bound * 1e3 / ms:.4f} | {mufu['frac']:.4f} |", flush=True)
     del Qd, Kd, Vd, Od, qz
+    torch.cuda.empty_cache()
+
+
+def run_eight_sweep(args, dev, peaks, n_sm):
+    """8-bit block pairs (tiered selection, MXFP8) on the 32k GQA workload at
+    rho = 5%: attention ms, dense-equivalent TFLOP/s, the TFLOP/s of the pairs
+    computed, and the blended roofline (FP16 at the measured bf16 peak, MXFP8
+    at twice it, NVFP4 at four times it: the nominal dense ratios) and MUFU
+    fractions over the computed pairs."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    p16 = peaks["bf16_tflops"] * 1e12
+    p8, p4 = FP8_OVER_BF16 * p16, FP4_OVER_BF16 * p16
+    w = synth.GQA_N32K
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+    sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+    qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+    q8 = thrift.quantize_all_mxfp8(Qd, Kd, Vd, sh)
+    Od = torch.empty_like(Qd)
+    stream = torch.cuda.current_stream(dev)
+    print(f"| 8-bit budget rho8 ({w.name}, rho {w.rho:g}) | 8-bit share | attention ms | "
+          "dense-equivalent TFLOP/s | computed TFLOP/s | roofline frac (computed) | MUFU frac |")
+    print("|---:|---:|---:|---:|---:|---:|---:|")
+    for rho8 in (0.0, 0.1, 0.25, 0.5, 0.95):
+        mask = thrift.select_blocks_tiered(Qd, Kd, sh, w.rho, 0.0, rho8=rho8)
+        for _ in range(args.warmup):
+            thrift.attention_tiered(Qd, Kd, Vd, mask, qz, sh, Od, stream, q8=q8)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(2, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n):
+            thrift.attention_tiered(Qd, Kd, Vd, mask, qz, sh, Od, stream, q8=q8)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if thrift.last_device_error(stream) != 0:
+            raise RuntimeError("a kernel reported a device error in the 8-bit sweep")
+        ms = e0.elapsed_time(e1) / n
+        m = mask.cpu().numpy()
+        f16, f4 = flop_split(w, m)
+        f8 = pair_flops(w, m, 3)
+        t_bound = max(f16 / p16 + f8 / p8 + f4 / p4,
+                      (attention_bytes(w, m) + eight_bytes(w, m)) / (peaks["hbm_gbs"] * 1e9))
+        mufu = mufu_ceiling(w, m, ms, 1965.0, n_sm)
+        share = f8 / (f16 + f8 + f4)
+        print(f"| {rho8:g} | {share:.3f} | {ms:.4f} | {w.flops() / (ms * 1e-3) / 1e12:.1f} | "
+              f"{(f16 + f8 + f4) / (ms * 1e-3) / 1e12:.1f} | {t_bound * 1e3 / ms:.4f} | {mufu['frac']:.4f} |",
+              flush=True)
+    del Qd, Kd, Vd, Od, qz, q8
     torch.cuda.empty_cache()
 
 
@@ -674,16 +747,24 @@ def main(argv=None):
                     help="time the attention kernel on every workload and rho (markdown table), then exit")
     ap.add_argument("--decode-sweep", action="store_true",
                     help="time the decode step on the GQA and batched caches (markdown table), then exit")
+    ap.add_argument("--tier-sweep", action="store_true",
+                    help="time attention with skipped and with 8-bit pairs (markdown tables), then exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.sweep:
         run_sweep(args)
-    elif args.decode_sweep:
+    elif args.decode_sweep or args.tier_sweep:
         import torch
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
-        run_decode_sweep(args, dev, load_peaks()[0])
+        if args.decode_sweep:
+            run_decode_sweep(args, dev, load_peaks()[0])
+        else:
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            run_skip_sweep(args, dev, load_peaks()[0], n_sm)
+            print()
+            run_eight_sweep(args, dev, load_peaks()[0], n_sm)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -48,6 +48,28 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   return false;
 }
 
+// The same wait with its slow path (timer, abort flag, error record) out of
+// line: one try_wait, which the hardware already suspends for a while, stays
+// inline.  All warp roles' loops run at once on an SM and share its
+// instruction caches, so where a kernel's waits sit decides how often its
+// warps stall on instruction fetch; a kernel picks the form per role by
+// measurement.
+static __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                       uint32_t* err, uint32_t code) {
+  return wait_or_abort(bar, parity, abort, err, code);
+}
+
+template <bool OUT_OF_LINE>
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
+                                             uint32_t code) {
+  if constexpr (OUT_OF_LINE) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_or_abort_slow(bar, parity, abort, err, code);
+  } else {
+    return wait_or_abort(bar, parity, abort, err, code);
+  }
+}
+
 // Named barrier of the softmax threads that also ORs a per-thread flag,
 // so that every softmax thread takes the same exit decision.
 template <int NT>

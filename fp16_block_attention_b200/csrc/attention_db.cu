@@ -31,10 +31,10 @@
 // A third instantiation adds 8-bit pairs (mask 3, the MXFP8 copies of Q, K
 // and V): S from .kind::mxf8f6f4 products with E8M0 scales in tensor memory,
 // and P * 2^11 encoded per 32 keys as MXFP8 (E8M0 scale from the group's
-// maximum, E4M3 codes) into a 128-byte-swizzled shared-memory P buffer.  Its
-// K / V tiles share the fp16 tiles' slots and barriers; it keeps three NVFP4
-// ring slots instead of four to make room for the Q copy and the wider P
-// buffers.
+// maximum, E4M3 codes) into tensor memory, the A operand of the P V product,
+// double-buffered in the fp16 P columns.  An 8-bit key tile travels through
+// the NVFP4 ring as two consecutive slots (K8 and its scales, then V8 and its
+// scales), so it is prefetched like an NVFP4 tile.
 #include <cuda_fp16.h>
 
 #include "attention_common.cuh"
@@ -55,7 +55,7 @@ constexpr int kDBMmaPV = 10;
 // Tensor-memory columns (512 allocated).
 constexpr uint32_t kDColS = 0;      // S of key tile k in buffer k % 2 at 128 * (k % 2)
 constexpr uint32_t kDColO = 256;    // O, D columns
-constexpr uint32_t kDColP16 = 384;  // fp16 P, 64 columns
+constexpr uint32_t kDColP16 = 384;  // fp16 P, 64 columns (P8 of P buffer b: 32 columns at 32 b)
 constexpr uint32_t kDColSFQ = 448;  // Q4 scales, 4 columns per 64-wide chunk of D
 constexpr uint32_t kDColSFK = 456;  // K4 scales of the key tile being multiplied
 constexpr uint32_t kDColSFV = 464;  // V4 scales of the key tile being multiplied
@@ -73,9 +73,7 @@ struct SmemDB {
   static constexpr uint32_t kQ4 = kQ16 + kQ16Bytes;
   static constexpr uint32_t kQSFBytes = (D / 64) * 512;
   static constexpr uint32_t kQSF = kQ4 + kQ4Bytes;
-  // P buffer: 128 rows x 128 keys of E2M1 (64B-swizzled) or, with 8-bit
-  // pairs, of E4M3 (128B-swizzled)
-  static constexpr uint32_t kPBufBytes = EIGHT ? 16384 : 8192;
+  static constexpr uint32_t kPBufBytes = 8192;  // 128 rows x 128 keys of E2M1, 64B-swizzled
   static constexpr uint32_t kP4 = (kQSF + kQSFBytes + 1023) / 1024 * 1024;  // two buffers
   static constexpr uint32_t kQ8Bytes = EIGHT ? 128 * D : 0;                 // Q8 tile, then its scales
   static constexpr uint32_t kQ8 = kP4 + 2 * kPBufBytes;
@@ -87,7 +85,7 @@ struct SmemDB {
   static constexpr uint32_t kVSFBytes = 1024;
   static constexpr uint32_t kSlot4Bytes = (kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes + 1023) / 1024 * 1024;
   static constexpr uint32_t kSlot4 = (kQS8 + kQS8Bytes + 1023) / 1024 * 1024;
-  static constexpr int kNS = EIGHT ? 3 : 4;  // NVFP4 K/V ring slots
+  static constexpr int kNS = 4;  // NVFP4 K/V ring slots (an 8-bit tile takes two)
   static constexpr uint32_t kK16Bytes = 128 * D * 2;
   static constexpr uint32_t kSlot16 = kSlot4 + kNS * kSlot4Bytes;  // K16 then V16
   static constexpr uint32_t kMisc = kSlot16 + 2 * kK16Bytes;
@@ -95,11 +93,11 @@ struct SmemDB {
   static constexpr uint32_t kTx4 = kK4Bytes + kV4Bytes + kKSFBytes + kVSFBytes;
   static constexpr uint32_t kTx16 = kK16Bytes;
   static constexpr uint32_t kTxQ = kQ16Bytes + kQ4Bytes + kQSFBytes + kQ8Bytes + kQS8Bytes;
-  // 8-bit K / V tiles in the fp16 slots, each followed by its 512 scale bytes
+  // 8-bit K / V tiles, each in one NVFP4 ring slot followed by its 512 scale bytes
   static constexpr uint32_t kK8Bytes = 128 * D;  // 128 keys x D channels
   static constexpr uint32_t kV8Bytes = D * 128;  // D channels x 128 keys
   static constexpr uint32_t kTx8 = kK8Bytes + 512;
-  static_assert(kK8Bytes + 512 <= kK16Bytes && kV8Bytes + 512 <= kK16Bytes, "8-bit tiles must fit the fp16 slots");
+  static_assert(kK8Bytes + 512 <= kSlot4Bytes && kV8Bytes + 512 <= kSlot4Bytes, "8-bit tiles must fit a ring slot");
   static_assert(kBytes + 1024 <= 232448, "shared memory above the 227 KB per-CTA limit");
   static_assert(kQ4 % 1024 == 0 && kSlot4 % 1024 == 0 && kSlot16 % 1024 == 0 && kQ8 % 1024 == 0,
                 "TMA tiles need 1 KB alignment");
@@ -215,6 +213,11 @@ __global__ void __launch_bounds__(kDBThreads, 1)
   const auto tile_of = [&](int it) -> int { return SKIP ? (ms.lst[it] & 0x3FF) : it; };
   const auto fp16_of = [&](int it) -> bool { return SKIP ? (ms.lst[it] & 0x8000) != 0 : ms.cls[it] != 0; };
   const auto eight_of = [&](int it) -> bool { return EIGHT && (ms.lst[it] & 0x4000) != 0; };
+  // Bounded waits with the slow path out of line in the producer and issuer
+  // loops, and in the method's softmax loop too: the fastest of the four
+  // placements on B200 for each instantiation (the waits' code changes how
+  // the roles' hot loops share the instruction caches).
+  constexpr bool kOolRoles = true, kOolSoftmax = !SKIP;
 
   if (warp == kDBProducer) {
     // ======================== producer ========================
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         const int kt = tile_of(it);
         if (!fp16_of(it) && !eight_of(it)) {
           const int slot = u4 % L::kNS, use = u4 / L::kNS;
-          if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (use > 0 && !bounded_wait<kOolRoles>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
           uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
           mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx4);
@@ -251,35 +254,42 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           bulk_load(st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes,
                     p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * kt) * 512, L::kVSFBytes, &ms.bar_full4[slot]);
           ++u4;
+        } else if (EIGHT && eight_of(it)) {
+          // 8-bit tile: K8 and its scales in ring slot u4, V8 and its scales in u4 + 1
+          bool stop = false;
+          for (int part = 0; part < 2; ++part) {
+            const int slot = u4 % L::kNS, use = u4 / L::kNS;
+            if (use > 0 && !bounded_wait<kOolRoles>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
+              stop = true;
+              break;
+            }
+            uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
+            const size_t sc = (static_cast<size_t>(bhk) * p.NT + kt) * 512;
+            mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx8);
+            if (part == 0) {
+              tma_load_3d(st, &mK8, &ms.bar_full4[slot], 0, kt * 128, bhk);
+              bulk_load(st + L::kK8Bytes, p.ks8 + sc, 512, &ms.bar_full4[slot]);
+            } else {
+              tma_load_3d(st, &mV8, &ms.bar_full4[slot], kt * 128, 0, bhk);
+              bulk_load(st + L::kV8Bytes, p.vs8 + sc, 512, &ms.bar_full4[slot]);
+            }
+            ++u4;
+          }
+          if (stop) break;
         } else {
-          // fp16 or 8-bit tile: the same two slots and barriers
-          const bool eight = eight_of(it);
           uint8_t* st = sm + L::kSlot16;
-          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (u16 > 0 && !bounded_wait<kOolRoles>(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
             break;
-          if (EIGHT && eight) {
-            mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx8);
-            tma_load_3d(st, &mK8, &ms.bar_full_k16, 0, kt * 128, bhk);
-            bulk_load(st + L::kK8Bytes, p.ks8 + (static_cast<size_t>(bhk) * p.NT + kt) * 512, 512, &ms.bar_full_k16);
-          } else {
-            mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
-            for (int pnl = 0; pnl < D / 64; ++pnl)
-              tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
-          }
-          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
-            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K copy of this tile is in flight
+          mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
+          for (int pnl = 0; pnl < D / 64; ++pnl)
+            tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
+          if (u16 > 0 && !bounded_wait<kOolRoles>(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
+            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K16 copy of this tile is in flight
             break;
           }
-          if (EIGHT && eight) {
-            mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx8);
-            tma_load_3d(st + L::kK16Bytes, &mV8, &ms.bar_full_v16, kt * 128, 0, bhk);
-            bulk_load(st + L::kK16Bytes + L::kV8Bytes, p.vs8 + (static_cast<size_t>(bhk) * p.NT + kt) * 512, 512,
-                      &ms.bar_full_v16);
-          } else {
-            mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
-            for (int pnl = 0; pnl < D / 64; ++pnl)
-              tma_load_3d(st + L::kK16Bytes + pnl * 16384, &mV16, &ms.bar_full_v16, pnl * 64, kt * 128, bhk);
-          }
+          mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
+          for (int pnl = 0; pnl < D / 64; ++pnl)
+            tma_load_3d(st + L::kK16Bytes + pnl * 16384, &mV16, &ms.bar_full_v16, pnl * 64, kt * 128, bhk);
           ++u16;
         }
       }
@@ -298,7 +308,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     if (lane == 0) {
       constexpr uint32_t sbo4 = (D == 128) ? 512u : 256u;
       constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
-      bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
+      bool ok = bounded_wait<kOolRoles>(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
       tc_fence_after();
       if (ok) {
         for (int c = 0; c < D / 64; ++c)
@@ -310,21 +320,26 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         const int bb = it & 1;
         const bool fp16 = fp16_of(it), eight = eight_of(it);
         int slot = 0;
-        if (!fp16 && !eight) {
+        if (EIGHT && eight) {
+          // K8 in ring slot u4 (V8, in u4 + 1, is the P V issuer's)
           slot = u4 % L::kNS;
-          if (!(ok = wait_or_abort(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          u4 += 2;
+          tc_fence_after();
+          tmem_cp_32x128b_x4(tm + kDColSFK8, make_sdesc(sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK8Bytes, 16,
+                                                        128, LAYOUT_NONE));
+        } else if (!fp16) {
+          slot = u4 % L::kNS;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++u4;
           tc_fence_after();
           const uint32_t ksf = sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK4Bytes + L::kV4Bytes;
           for (int c = 0; c < D / 64; ++c)
             tmem_cp_32x128b_x4(tm + kDColSFK + 4 * c, make_sdesc(ksf + 512 * c, 16, 128, LAYOUT_NONE));
         } else {
-          if (!(ok = wait_or_abort(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uk16;
           tc_fence_after();
-          if (EIGHT && eight)
-            tmem_cp_32x128b_x4(tm + kDColSFK8,
-                               make_sdesc(sbase + L::kSlot16 + L::kK8Bytes, 16, 128, LAYOUT_NONE));
         }
         // Buffers bb were last used by key tile kt - 2: wait until its S was
         // loaded by the softmax threads, and until its P V product is done, so
@@ -332,9 +347,9 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         // bb and its scales without waiting themselves.  (Buffers and phases
         // count processed tiles, it, not tile indices.)
         if (it >= 2) {
-          if (!(ok = wait_or_abort(&ms.bar_s_free[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_s_free[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
             break;
-          if (!(ok = wait_or_abort(&ms.bar_o_done[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA)))
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_o_done[bb], ((it - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA)))
             break;
           tc_fence_after();
         }
@@ -343,7 +358,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           // MXFP8 along D: K = 32 per product, scale byte kk of each row's column
           constexpr uint32_t sbo8 = (D == 128) ? 1024u : 512u;
           constexpr uint32_t sw8 = (D == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
-          const uint32_t q8 = sbase + L::kQ8, k8 = sbase + L::kSlot16;
+          const uint32_t q8 = sbase + L::kQ8, k8 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
             mma_mxf8(dS, make_sdesc(q8 + 32 * kk, 16, sbo8, sw8), make_sdesc(k8 + 32 * kk, 16, sbo8, sw8),
@@ -365,11 +380,17 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           }
         }
         mma_commit(&ms.bar_s_full[bb]);
-        // the K operands of this key tile are no longer needed (V: the P V issuer)
-        if (!fp16 && !eight)
+        // the K operands of this key tile are no longer needed (V: the P V
+        // issuer).  An 8-bit tile's K slot is this thread's alone: both of its
+        // arrivals, after this thread saw the slot filled.
+        if (EIGHT && eight) {
           mma_commit(&ms.bar_empty4[slot]);
-        else
+          mma_commit(&ms.bar_empty4[slot]);
+        } else if (!fp16) {
+          mma_commit(&ms.bar_empty4[slot]);
+        } else {
           mma_commit(&ms.bar_empty_k16);
+        }
       }
       // drain: every tensor-core operation this thread issued completes before exit
       mma_commit(&ms.bar_drain[0]);
@@ -391,14 +412,23 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         // it cannot overwrite scales that product still reads.
         int slot = 0;
         uint32_t v4 = 0;
-        if (!fp16 && !eight) {
+        if (EIGHT && eight) {
+          // V8 in ring slot u4 + 1 (K8, in u4, is the S issuer's)
+          slot = (u4 + 1) % L::kNS;
+          const int use = (u4 + 1) / L::kNS;
+          u4 += 2;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          tc_fence_after();
+          v4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
+          tmem_cp_32x128b_x4(tm + kDColSFV8, make_sdesc(v4 + L::kV8Bytes, 16, 128, LAYOUT_NONE));
+        } else if (!fp16) {
           slot = u4 % L::kNS;
           const int use = u4 / L::kNS;
           ++u4;
           // V4 landed with K4 in one barrier phase; wait on it here too so that
           // this thread observes the copy itself.  The producer cannot refill the
           // slot before this thread releases it.
-          if (!(ok = wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           tc_fence_after();
           const uint32_t st = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
           v4 = st + L::kK4Bytes;
@@ -406,28 +436,20 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           for (int c = 0; c < 2; ++c)
             tmem_cp_32x128b_x4(tm + kDColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
         } else {
-          if (!(ok = wait_or_abort(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles>(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uv16;
-          if (EIGHT && eight) {
-            tc_fence_after();
-            tmem_cp_32x128b_x4(tm + kDColSFV8, make_sdesc(sbase + L::kSlot16 + L::kK16Bytes + L::kV8Bytes, 16, 128,
-                                                          LAYOUT_NONE));
-          }
         }
-        if (!(ok = wait_or_abort(&ms.bar_p_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        if (!(ok = bounded_wait<kOolRoles>(&ms.bar_p_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
         tc_fence_after();
         const uint32_t dO = tm + kDColO;
         if (EIGHT && eight) {
-          // P8 (128 x 128 keys, 128B-swizzled) times V8 (D x 128 keys): K = 32
-          // per product; P's scale for keys 32 kk .. is byte kk % 2 of column
-          // 4 (kk / 2) + r / 32, V's byte kk of column d / 32
-          const uint32_t p8s = sbase + L::kP4 + bb * L::kPBufBytes;
-          const uint32_t v8 = sbase + L::kSlot16 + L::kK16Bytes;
+          // P8 (tensor memory, 32 columns of buffer bb) times V8 (D x 128 keys,
+          // 128B-swizzled): K = 32 per product; P's scale for keys 32 kk .. is
+          // byte kk % 2 of column 4 (kk / 2) + r / 32, V's byte kk of column d / 32
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            mma_mxf8(dO, make_sdesc(p8s + 32 * kk, 16, 1024, LAYOUT_SW128),
-                     make_sdesc(v8 + 32 * kk, 16, 1024, LAYOUT_SW128), idesc_mxf8(128, D, kk & 1, kk),
-                     tm + kDColSFP + 8 * bb + 4 * (kk >> 1), tm + kDColSFV8, acc);
+            mma_mxf8_ts(dO, tm + kDColP16 + 32 * bb + 8 * kk, make_sdesc(v4 + 32 * kk, 16, 1024, LAYOUT_SW128),
+                        idesc_mxf8(128, D, kk & 1, kk), tm + kDColSFP + 8 * bb + 4 * (kk >> 1), tm + kDColSFV8, acc);
             acc = 1;
           }
         } else if (!fp16) {
@@ -448,10 +470,14 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           }
         }
         mma_commit(&ms.bar_o_done[bb]);
-        if (!fp16 && !eight)
+        if (EIGHT && eight) {  // the V8 slot is this thread's alone: both arrivals
           mma_commit(&ms.bar_empty4[slot]);
-        else
+          mma_commit(&ms.bar_empty4[slot]);
+        } else if (!fp16) {
+          mma_commit(&ms.bar_empty4[slot]);
+        } else {
           mma_commit(&ms.bar_empty_v16);
+        }
       }
       mma_commit(&ms.bar_drain[1]);
       mbar_wait(&ms.bar_drain[1], 0, kWaitNs);
@@ -479,7 +505,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       const int bb = it & 1;
       const int kt = tile_of(it);
       const bool fp16 = fp16_of(it), eight = eight_of(it);
-      if (!failed) failed = !wait_or_abort(&ms.bar_s_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (!failed) failed = !bounded_wait<kOolSoftmax>(&ms.bar_s_full[bb], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) {
         turn_in();
@@ -544,13 +570,15 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         // E8M0 byte = that exponent - 8 (biased), clamped at 0.  A group whose
         // byte would be 0 (amax below 2^-118, P below 2^-129) is encoded as
         // zeros; the codes are E4M3(P * 2^11 / X) with -log2 X in the bias.
+        // Both 16-key halves of a group take its X and bias, so that the
+        // exponentials below are the NVFP4 tiles' code.
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const float amax = ex2(fmaf(fmaxf(gh[2 * c], gh[2 * c + 1]), c2, base));
           const int eb = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
           const bool live = eb > 8;
-          sce[c] = live ? __uint_as_float(static_cast<uint32_t>(eb - 8) << 23) : 0.f;  // X
-          bias[c] = live ? base + static_cast<float>(135 - eb) : -INFINITY;
+          sce[2 * c] = sce[2 * c + 1] = live ? __uint_as_float(static_cast<uint32_t>(eb - 8) << 23) : 0.f;  // X
+          bias[2 * c] = bias[2 * c + 1] = live ? base + static_cast<float>(135 - eb) : -INFINITY;
           sfw |= static_cast<uint32_t>(live ? eb - 8 : 0) << (8 * c);
         }
       } else if (!fp16) {
@@ -568,9 +596,10 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // P buffer bb (and its scales) is free: the S issuer waited for the P V
       // product of key tile kt - 2 before issuing S(kt).  The fp16 P columns
       // are single-buffered, so an fp16 tile waits for the previous key tile's
-      // product.
-      if (fp16 && it >= 1) {
-        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      // product, and so does an 8-bit tile (whose P takes half of those
+      // columns) after an fp16 tile.
+      if (it >= 1 && (fp16 || (EIGHT && eight && fp16_of(it - 1)))) {
+        failed = !bounded_wait<kOolSoftmax>(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
         failed = __any_sync(0xffffffffu, failed);
         if (failed) {
           turn_in();
@@ -597,31 +626,6 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
         rs = (sum16(&s[0]) + sum16(&s[16])) + (sum16(&s[32]) + sum16(&s[48]));
         tmem_st32(lane_base + kDColP16 + 32 * half, w);
-      } else if (EIGHT && eight) {
-        uint8_t* d8 = sm + L::kP4 + bb * L::kPBufBytes;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const float2 bv = make_float2(bias[c], bias[c]);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 pp = ex2_fma2(s[32 * c + i], s[32 * c + i + 1], c2v, bv);
-            s[32 * c + i] = pp.x;
-            s[32 * c + i + 1] = pp.y;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) rs = fmaf(sum16(&s[32 * c]) + sum16(&s[32 * c + 16]), sce[c], rs);
-        // 16 keys per 16-byte chunk; this half's keys are chunks 4 h .. 4 h + 3
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w[i] = (cvt_e4m3x2(s[16 * q + 4 * i], s[16 * q + 4 * i + 1]) & 0xFFFFu) |
-                   (cvt_e4m3x2(s[16 * q + 4 * i + 2], s[16 * q + 4 * i + 3]) << 16);
-          *reinterpret_cast<uint4*>(d8 + sw128_off(r, 4 * half + q)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        tmem_st1(lane_base + kDColSFP + 8 * bb + 4 * half + quad, sfw);
       } else {
         uint8_t* d4 = sm + L::kP4 + bb * L::kPBufBytes;
         // exponentials with 1/scale folded in, then sums and codes
@@ -637,14 +641,25 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) rs = fmaf(sum16(&s[16 * g]), sce[g], rs);
+        if (EIGHT && eight) {
+          // 8-bit tile: four E4M3 codes per tensor-memory column, this half's
+          // 64 keys in columns 16 h .. 16 h + 15 of P buffer bb
+          uint32_t w8[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 w = make_uint4(cvt_e2m1x8(&s[32 * c]), cvt_e2m1x8(&s[32 * c + 8]), cvt_e2m1x8(&s[32 * c + 16]),
-                                     cvt_e2m1x8(&s[32 * c + 24]));
-          *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + c)) = w;
+          for (int j = 0; j < 16; ++j)
+            w8[j] = (cvt_e4m3x2(s[4 * j], s[4 * j + 1]) & 0xFFFFu) | (cvt_e4m3x2(s[4 * j + 2], s[4 * j + 3]) << 16);
+          tmem_st16(lane_base + kDColP16 + 32 * bb + 16 * half, w8);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint4 w = make_uint4(cvt_e2m1x8(&s[32 * c]), cvt_e2m1x8(&s[32 * c + 8]),
+                                       cvt_e2m1x8(&s[32 * c + 16]), cvt_e2m1x8(&s[32 * c + 24]));
+            *reinterpret_cast<uint4*>(d4 + sw64_off(r, 2 * half + c)) = w;
+          }
         }
         // Scale factors of a 128-row A operand: the MMA reads row r's four
-        // scales of K chunk c from lane r, column base + 4c + r / 32.
+        // scales of K chunk c from lane r, column base + 4c + r / 32 (8-bit:
+        // byte c of column base + 4 h + r / 32 for keys 64 h + 32 c ..).
         tmem_st1(lane_base + kDColSFP + 8 * bb + 4 * half + quad, sfw);
       }
       turn_out();
@@ -653,7 +668,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // = 1 are unchanged); O is stable once the previous key tile's P V
       // product is done.
       if (it > 0 && __any_sync(0xffffffffu, Mn > M)) {
-        failed = !wait_or_abort(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = !bounded_wait<kOolSoftmax>(&ms.bar_o_done[bb ^ 1], ((it - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
         failed = __any_sync(0xffffffffu, failed);
         if (failed) continue;
         tc_fence_after();
@@ -685,7 +700,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     // ---- epilogue: O / l -> fp16 (both carry the 2^11 pre-scale) ----
     if (np > 0) {
       if (!failed)
-        failed = !wait_or_abort(&ms.bar_o_done[(np - 1) & 1], ((np - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = !bounded_wait<kOolSoftmax>(&ms.bar_o_done[(np - 1) & 1], ((np - 1) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
       ms.lsum[half][r] = l;
       // every softmax thread takes the same exit decision (and sees lsum)
       failed = softmax_bar_or<kDBSoftmax>(failed);
