@@ -62,22 +62,49 @@ SelectWs carve(void* ws, const thrift_shape& s) {
   return w;
 }
 
-// grid (nb, BH), block D/2 threads, two channels per thread.
-__global__ void pool_kernel(const __half* __restrict__ x, int N, int D, int blk, float* __restrict__ out) {
+// grid (nb, BH), block kPoolThreads: the block of blk rows x D channels is
+// read in 16-byte pieces (8 channels), thread t taking chunk t % (D/8) of rows
+// t / (D/8), + kPoolThreads / (D/8), ..., all its loads in flight at once;
+// the row groups' partial sums meet in shared memory.  FP64 sums of fp16
+// values are exact in any order (every fp16 value is a multiple of 2^-24 below
+// 2^16), so the mean is fl32(exact sum / blk) whatever the split.
+constexpr int kPoolThreads = 256;
+
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __half* __restrict__ x, int N, int D, int blk,
+                                                            float* __restrict__ out) {
+  __shared__ double part[kPoolThreads * 8];  // [row group][D]
   const int nb = N / blk;
   const size_t bh = blockIdx.y;
   const int i = blockIdx.x;
-  const int c = threadIdx.x;  // channel pair
-  const __half2* src = reinterpret_cast<const __half2*>(x + (bh * N + static_cast<size_t>(i) * blk) * D) + c;
-  double s0 = 0.0, s1 = 0.0;
-  for (int r = 0; r < blk; ++r) {
-    const float2 f = __half22float2(src[static_cast<size_t>(r) * (D / 2)]);
-    s0 += static_cast<double>(f.x);
-    s1 += static_cast<double>(f.y);
+  const int chunks = D / 8, groups = kPoolThreads / chunks, rows = blk / groups;
+  const int cc = threadIdx.x % chunks, rg = threadIdx.x / chunks;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (bh * N + static_cast<size_t>(i) * blk) * D) + cc;
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+  constexpr int kMaxRows = 8;  // blk <= 128, D >= 64: at most 128 / 16 rows per thread
+  uint4 v[kMaxRows];
+#pragma unroll
+  for (int q = 0; q < kMaxRows; ++q)
+    if (q < rows) v[q] = __ldg(src + static_cast<size_t>(rg + q * groups) * chunks);
+#pragma unroll
+  for (int q = 0; q < kMaxRows; ++q) {
+    if (q < rows) {
+      const __half2* h = reinterpret_cast<const __half2*>(&v[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        acc[2 * e] += static_cast<double>(f.x);
+        acc[2 * e + 1] += static_cast<double>(f.y);
+      }
+    }
   }
-  float* dst = out + (bh * nb + i) * D + 2 * c;
-  dst[0] = static_cast<float>(s0 / blk);
-  dst[1] = static_cast<float>(s1 / blk);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rg * D + 8 * cc + e] = acc[e];
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kPoolThreads) {
+    double sum = 0.0;
+    for (int g = 0; g < groups; ++g) sum += part[g * D + d];
+    out[(bh * nb + i) * D + d] = static_cast<float>(sum / blk);
+  }
 }
 
 // grid (ceil(nb/32), ceil(nb/32), B*Hq), block 256: a 32x32 tile of scores,
@@ -214,6 +241,13 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
 
   // Key of the kk-th largest valid pair (1 <= kk < valid) by an 8-bit radix
   // select: the first kk pairs are exactly those with key >= the result.
+  // Each pass histograms the digit of the keys that match the prefix found so
+  // far: warp w walks rows w, w + 32, ... (only the valid columns), so all
+  // lanes of a warp run the same trip count; lanes with equal digits add
+  // their count once (the top digits of the keys are shared by most pairs);
+  // warp 0 then finds the digit that holds the kk-th key with a shuffle scan.
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nwarps = blockDim.x / 32;
   const auto kth_largest = [&](long long kk) -> uint64_t {
     __syncthreads();  // every thread has read the previous result
     if (threadIdx.x == 0) {
@@ -226,27 +260,65 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
       for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
       __syncthreads();
       const uint64_t prefix = s_prefix;
-      for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
-        const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
-        if (causal && j > i) continue;
-        const uint64_t key = key_of(sc[idx], i, j);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      for (int i = warp; i < nb; i += nwarps) {
+        const int ncol = causal ? i + 1 : nb;
+        const float* row = sc + static_cast<size_t>(i) * nb;
+        for (int j0 = 0; j0 < ncol; j0 += 128) {  // four column chunks, loads first
+          float v[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) v[q] = (j0 + 32 * q + lane < ncol) ? row[j0 + 32 * q + lane] : 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j = j0 + 32 * q + lane;
+            bool match = false;
+            uint32_t bin = 0;
+            if (j < ncol) {
+              const uint64_t key = key_of(v[q], i, j);
+              match = (key & pmask) == prefix;
+              bin = static_cast<uint32_t>(key >> shift) & 255u;
+            }
+            const uint32_t active = __ballot_sync(0xffffffffu, match);
+            if (match) {
+              const uint32_t peers = __match_any_sync(active, bin);
+              if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned int>(__popc(peers)));
+            }
+          }
+        }
       }
       __syncthreads();
-      if (threadIdx.x == 0) {
-        long long rem = s_remaining, cum = 0;
-        int digit = 0;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + hist[d] >= rem) {
-            digit = d;
-            break;
-          }
-          cum += hist[d];
+      if (warp == 0) {
+        // lane l holds bins 255 - 8 l .. 248 - 8 l, highest first
+        uint32_t c[8], tot = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          c[t] = hist[255 - 8 * lane - t];
+          tot += c[t];
         }
-        rem -= cum;
-        s_prefix = prefix | (static_cast<uint64_t>(digit) << shift);
-        s_remaining = rem;
-        s_done = (static_cast<long long>(hist[digit]) == rem);
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const long long rem = s_remaining;
+        const long long excl = static_cast<long long>(incl) - tot;
+        if (excl < rem && rem <= static_cast<long long>(incl)) {  // exactly one lane
+          long long cum = excl;
+          int digit = 0;
+          long long cnt = 0;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (cum + c[t] >= rem) {
+              digit = 255 - 8 * lane - t;
+              cnt = c[t];
+              break;
+            }
+            cum += c[t];
+          }
+          s_prefix = prefix | (static_cast<uint64_t>(digit) << shift);
+          s_remaining = rem - cum;
+          s_done = (cnt == rem - cum);
+        }
       }
       __syncthreads();
       pmask |= 255ull << shift;
@@ -301,8 +373,8 @@ long long budget_pairs(const thrift_shape& s, double rho) {
 
 void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s, const SelectWs& w, cudaStream_t st) {
   const int nb = s.N / s.blk;
-  pool_kernel<<<dim3(nb, s.B * s.Hq), s.D / 2, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
-  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
+  pool_kernel<<<dim3(nb, s.B * s.Hq), kPoolThreads, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
+  pool_kernel<<<dim3(nb, s.B * s.Hkv), kPoolThreads, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
   const int tiles = (nb + 31) / 32;
   score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
                                                                s.sm_scale, w.scores);
@@ -311,7 +383,7 @@ void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s,
 
 cudaError_t launch_pool_keys(const void* K, const thrift_shape& s, float* km, cudaStream_t st) {
   const int nb = s.N / s.blk;
-  pool_kernel<<<dim3(nb, s.B * s.Hkv), s.D / 2, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, km);
+  pool_kernel<<<dim3(nb, s.B * s.Hkv), kPoolThreads, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, km);
   return cudaGetLastError();
 }
 
