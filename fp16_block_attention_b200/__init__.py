@@ -83,6 +83,9 @@ def _load():
         "thrift_attention_tiered": ([vp] * 16 + [psh, vp, vp], st),
         "thrift_fused_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
         "thrift_attention_fused": ([vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
+        "thrift_fused_tiered_workspace_bytes": ([psh, ctypes.c_double, ctypes.POINTER(sz)], st),
+        "thrift_attention_fused_tiered": ([vp, vp, vp, psh, ctypes.c_double, ctypes.c_double, ctypes.c_double, vp, vp,
+                                           sz, vp], st),
         "thrift_pool_keys": ([vp, psh, vp, vp], st),
         "thrift_decode_select": ([vp, vp, psh, ctypes.c_double, vp, vp], st),
         "thrift_decode_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
@@ -107,7 +110,8 @@ EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quant8_bytes",
            "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_select_blocks_tiered",
            "thrift_attention", "thrift_attention_tiered",
            "thrift_fused_workspace_bytes",
-           "thrift_attention_fused", "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
+           "thrift_attention_fused", "thrift_fused_tiered_workspace_bytes", "thrift_attention_fused_tiered",
+           "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
            "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error", "thrift_mma_rate_probe",
            "thrift_strerror")
 
@@ -354,6 +358,29 @@ def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, str
     _check("thrift_attention_fused", _lib.thrift_attention_fused(
         _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(),
         _stream(stream)))
+    return out
+
+
+def fused_tiered_workspace_bytes(shape: Shape, rho8: float = 0.0) -> int:
+    n = ctypes.c_size_t()
+    _check("thrift_fused_tiered_workspace_bytes", _lib.thrift_fused_tiered_workspace_bytes(
+        ctypes.byref(shape.c()), float(rho8), ctypes.byref(n)))
+    return n.value
+
+
+def attention_fused_tiered(Qt, Kt, Vt, shape: Shape, rho: float, rho8: float = 0.0, sigma: float = 0.0, out=None,
+                           ws=None, stream=None):
+    """Quantise (NVFP4, and MXFP8 when rho8 > 0), select four classes (FP16
+    budget rho, 8-bit budget rho8, skipped share sigma) and attend in one call."""
+    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
+        _dev(t, n, torch.float16)
+    if out is None:
+        out = torch.empty_like(Qt)
+    if ws is None:
+        ws = torch.empty(fused_tiered_workspace_bytes(shape, rho8), dtype=torch.uint8, device=Qt.device)
+    _check("thrift_attention_fused_tiered", _lib.thrift_attention_fused_tiered(
+        _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(out),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

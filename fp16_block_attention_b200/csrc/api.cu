@@ -44,10 +44,11 @@ QuantSizes quant_sizes(const thrift_shape& s, thrift_operand op) {
 struct FusedWs {
   uint8_t *q4, *qs, *k4, *ks, *v4, *vs, *mask;
   void* sel;
+  uint8_t *q8, *qs8, *k8, *ks8, *v8, *vs8;  // MXFP8 copies (eight only)
   size_t total;
 };
 
-FusedWs carve_fused(void* base, const thrift_shape& s) {
+FusedWs carve_fused(void* base, const thrift_shape& s, bool eight = false) {
   FusedWs w;
   char* p = static_cast<char*>(base);
   size_t off = 0;
@@ -66,6 +67,15 @@ FusedWs carve_fused(void* base, const thrift_shape& s) {
   const size_t nb = s.N / s.blk;
   w.mask = take(static_cast<size_t>(s.B) * s.Hq * nb * nb);
   w.sel = take(select_workspace_bytes(s));
+  w.q8 = w.qs8 = w.k8 = w.ks8 = w.v8 = w.vs8 = nullptr;
+  if (eight) {
+    w.q8 = take(mx8_codes_bytes(s, THRIFT_Q));
+    w.qs8 = take(mx8_scales_bytes(s, THRIFT_Q));
+    w.k8 = take(mx8_codes_bytes(s, THRIFT_K));
+    w.ks8 = take(mx8_scales_bytes(s, THRIFT_K));
+    w.v8 = take(mx8_codes_bytes(s, THRIFT_V));
+    w.vs8 = take(mx8_scales_bytes(s, THRIFT_V));
+  }
   w.total = off;
   return w;
 }
@@ -274,6 +284,49 @@ thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V
     return THRIFT_ERR_CUDA;
   if (launch_select(Q, K, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
   return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, false, nullptr, err, cs));
+}
+
+thrift_status thrift_fused_tiered_workspace_bytes(const thrift_shape* shape, double rho8, size_t* bytes) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!bytes || !(rho8 >= 0.0 && rho8 <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  *bytes = carve_fused(nullptr, *shape, rho8 > 0.0).total;
+  return THRIFT_OK;
+}
+
+thrift_status thrift_attention_fused_tiered(const void* Q, const void* K, const void* V, const thrift_shape* shape,
+                                            double rho, double rho8, double sigma, void* O, void* ws,
+                                            size_t ws_bytes, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!Q || !K || !V || !O || !(rho >= 0.0 && rho <= 1.0) || !(rho8 >= 0.0 && rho8 <= 1.0) ||
+      !(sigma >= 0.0 && sigma <= 1.0))
+    return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return THRIFT_ERR_INVALID_ARG;
+  const bool eight = rho8 > 0.0;
+  if (eight && shape->blk != 128) return THRIFT_ERR_UNSUPPORTED;
+  const FusedWs need = carve_fused(nullptr, *shape, eight);
+  if (!ws || ws_bytes < need.total || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  const FusedWs w = carve_fused(ws, *shape, eight);
+  const thrift_shape& s = *shape;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint32_t* err = device_error_word();
+  if (!err) return THRIFT_ERR_CUDA;
+  if (launch_quantize_qk(Q, static_cast<size_t>(s.B) * s.Hq * s.N, s.N, s.D, w.q4, w.qs, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (launch_quantize_qk(K, static_cast<size_t>(s.B) * s.Hkv * s.N, s.N, s.D, w.k4, w.ks, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
+    return THRIFT_ERR_CUDA;
+  Mx8Copies copies = {w.q8, w.qs8, w.k8, w.ks8, w.v8, w.vs8};
+  if (eight) {
+    if (launch_quantize_mx8(Q, THRIFT_Q, s, w.q8, w.qs8, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+    if (launch_quantize_mx8(K, THRIFT_K, s, w.k8, w.ks8, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+    if (launch_quantize_mx8(V, THRIFT_V, s, w.v8, w.vs8, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  }
+  if (launch_select_tiered(Q, K, s, rho, rho8, sigma, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, true,
+                                    eight ? &copies : nullptr, err, cs));
 }
 
 namespace {

@@ -242,6 +242,21 @@ THRIFT_API thrift_status thrift_fused_workspace_bytes(const thrift_shape* shape,
 THRIFT_API thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V, const thrift_shape* shape,
                                      double rho, void* O, void* ws, size_t ws_bytes, void* stream);
 
+/* Workspace bytes of thrift_attention_fused_tiered for a given 8-bit budget
+ * (the NVFP4 copies, mask, selection workspace and, when rho8 > 0, the MXFP8
+ * copies; each part 256-byte aligned). */
+THRIFT_API thrift_status thrift_fused_tiered_workspace_bytes(const thrift_shape* shape, double rho8, size_t* bytes);
+
+/* The tiered path in one call: quantise Q, K, V to NVFP4 (and, when rho8 > 0,
+ * to MXFP8), select with thrift_select_blocks_tiered(rho, rho8, sigma), attend
+ * with thrift_attention_tiered.  The result equals those calls made one by
+ * one.  rho8 > 0 needs blk = 128 (THRIFT_ERR_UNSUPPORTED otherwise).
+ * ws: device workspace of thrift_fused_tiered_workspace_bytes(shape, rho8). */
+THRIFT_API thrift_status thrift_attention_fused_tiered(const void* Q, const void* K, const void* V,
+                                                       const thrift_shape* shape, double rho, double rho8,
+                                                       double sigma, void* O, void* ws, size_t ws_bytes,
+                                                       void* stream);
+
 /* ---- decode: one new query row per (batch, query head) ----------------------
  * One decode step over the caches that prefill leaves behind: the fp16 K and
  * V and their NVFP4 copies from thrift_quantize_nvfp4.  The ThriftAttention

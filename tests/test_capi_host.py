@@ -71,6 +71,12 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert tr(fake, fake, sh, 0.05, 0.1, 0.1, fake, fake, 16, None) == 5
     assert lib.thrift_quantize_mxfp8(fake, 3, sh, fake, fake, None) == 1
     assert lib.thrift_quantize_mxfp8(fake, 0, sh, None, fake, None) == 1
+    ft = lib.thrift_attention_fused_tiered
+    assert ft(fake, fake, fake, sh, 0.05, 1.5, 0.0, fake, fake, 1 << 30, None) == 1          # rho8 out of range
+    assert ft(fake, fake, fake, sh, 0.05, 0.1, -0.5, fake, fake, 1 << 30, None) == 1         # sigma out of range
+    assert ft(fake, fake, fake, ctypes.byref(_c(blk=64)), 0.05, 0.1, 0.0, fake, fake, 1 << 30, None) == 2
+    assert ft(fake, fake, fake, sh, 0.05, 0.1, 0.0, fake, fake, 16, None) == 5
+    assert ft(fake, None, fake, sh, 0.05, 0.0, 0.0, fake, fake, 1 << 30, None) == 1
     at = lib.thrift_attention_tiered
     assert at(*[fake] * 10, fake, None, fake, fake, fake, fake, sh, fake, None) == 1        # some copies missing
     assert at(*[fake] * 10, fake, ctypes.c_void_p(264), fake, fake, fake, fake, sh, fake, None) == 1  # misaligned
@@ -94,6 +100,14 @@ def test_workspace_sizes_cover_the_parts():
     need = thrift.fused_workspace_bytes(sh)
     parts = sum(sum(thrift.quant_bytes(sh, op)) for op in (0, 1, 2)) + 4 * 8 * 8 + thrift.select_workspace_bytes(sh)
     assert need >= parts
+
+
+def test_fused_tiered_workspace_adds_the_mxfp8_copies_only_for_an_eight_bit_budget():
+    sh = thrift.Shape(1, 4, 2, 1024, 128, 128, True, 0.088)
+    w0, w8 = thrift.fused_tiered_workspace_bytes(sh, 0.0), thrift.fused_tiered_workspace_bytes(sh, 0.25)
+    assert w0 == thrift.fused_workspace_bytes(sh)
+    mx8 = sum(sum(thrift.quant8_bytes(sh, op)) for op in (thrift.Q, thrift.K, thrift.V))
+    assert mx8 <= w8 - w0 <= mx8 + 6 * 256      # each part 256-byte aligned
 
 
 def test_strerror_names_every_status():

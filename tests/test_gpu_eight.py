@@ -12,6 +12,7 @@ with blk 64) and the quality series of the 8-bit budget beside the oracle's.
 """
 import numpy as np
 import pytest
+import torch
 
 import fp16_block_attention_b200 as thrift
 import oracle
@@ -54,6 +55,21 @@ def test_attention_with_eight_bit_pairs_matches_oracle(w, rho, rho8, sigma):
                                              w.causal, w.sm_scale, qz)
     assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
     assert resolved <= max(1, rows.shape[0] // 1000), resolved
+
+
+@pytest.mark.parametrize("rho,rho8,sigma", [(0.05, 0.2, 0.0), (0.05, 0.0, 0.4), (0.1, 0.3, 0.3)])
+@pytest.mark.parametrize("w", CASES[:2], ids=IDS[:2])
+def test_fused_tiered_equals_the_separate_calls(w, rho, rho8, sigma):
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    sh = shape_of(w)
+    o1 = thrift.attention_fused_tiered(Qd, Kd, Vd, sh, rho, rho8, sigma)
+    assert thrift.last_device_error() == 0
+    m = thrift.select_blocks_tiered(Qd, Kd, sh, rho, sigma, rho8=rho8)
+    q8 = thrift.quantize_all_mxfp8(Qd, Kd, Vd, sh) if rho8 > 0 else None
+    o2 = thrift.attention_tiered(Qd, Kd, Vd, m, thrift.quantize_all(Qd, Kd, Vd, sh), sh, q8=q8)
+    assert thrift.last_device_error() == 0
+    assert torch.equal(o1, o2)
 
 
 def test_eight_bit_mask_without_the_copies_is_reported():
