@@ -15,19 +15,19 @@
 namespace thrift {
 namespace {
 
-// One thread per group of 16 along D.  rows = B*H*N.
+// One thread per group of 16 along D, two groups (a grid stride apart) per
+// step with all four 16-byte loads in flight before either is encoded.
+// rows = B*H*N.
 __global__ void __launch_bounds__(256) quantize_qk_kernel(const __half* __restrict__ x, size_t rows, int N, int D,
                                                           uint8_t* __restrict__ codes,
                                                           uint8_t* __restrict__ scales) {
   const int gpr = D / 16;  // groups per row
   const size_t total = rows * gpr;
   const int NT = num_tiles(N);
-  for (size_t gi = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; gi < total;
-       gi += static_cast<size_t>(gridDim.x) * blockDim.x) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const auto encode_store = [&](size_t gi, const uint4& a, const uint4& b) {
     const size_t row = gi / gpr;
     const int g = static_cast<int>(gi % gpr);
-    const uint4* src = reinterpret_cast<const uint4*>(x + row * D + g * 16);
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
     float v[16];
     const __half2* ha = reinterpret_cast<const __half2*>(&a);
     const __half2* hb = reinterpret_cast<const __half2*>(&b);
@@ -44,6 +44,20 @@ __global__ void __launch_bounds__(256) quantize_qk_kernel(const __half* __restri
     const size_t bh = row / N;
     const int n = static_cast<int>(row % N);
     scales[qk_scale_index(bh, n, g, NT, D)] = static_cast<uint8_t>(q.scale);
+  };
+  for (size_t gi = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; gi < total; gi += 2 * stride) {
+    const size_t gj = gi + stride;
+    const bool two = gj < total;
+    const uint4* s0 = reinterpret_cast<const uint4*>(x + gi * 16);  // group gi starts at element 16 gi
+    const uint4 a0 = __ldg(s0), b0 = __ldg(s0 + 1);
+    uint4 a1 = make_uint4(0u, 0u, 0u, 0u), b1 = a1;
+    if (two) {
+      const uint4* s1 = reinterpret_cast<const uint4*>(x + gj * 16);
+      a1 = __ldg(s1);
+      b1 = __ldg(s1 + 1);
+    }
+    encode_store(gi, a0, b0);
+    if (two) encode_store(gj, a1, b1);
   }
 }
 
@@ -62,46 +76,58 @@ __global__ void zero_qk_scale_padding(size_t bh_count, int N, int D, uint8_t* __
   }
 }
 
-// V along keys: one CTA per (bh, 64-key chunk).  The chunk [64][D] is staged
-// through shared memory; thread (d, k16) encodes keys k16*16 .. +15 of
-// channel d.  Chunks past N (padding to whole 128-key tiles) are all zero.
-__global__ void __launch_bounds__(256) quantize_v_kernel(const __half* __restrict__ v, int N, int D,
-                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  __shared__ __half tile[64][128 + 2];
+// V along keys: one CTA per (bh, 128-key tile).  The tile [nk][D] (nk = 128,
+// or 64 for the last tile when N is an odd multiple of 64) is staged through
+// shared memory with 16-byte loads, all of a thread's loads in flight at once;
+// task (d, k16) then encodes keys k16*16 .. +15 of channel d, consecutive lanes
+// taking consecutive channels (conflict-free column reads).  The scale blocks
+// of a tile are its two 64-key chunks; a chunk past N is all zero, and so are
+// the channels >= D of every block.
+constexpr int kVTile = 128, kVThreads = 256;
+
+__global__ void __launch_bounds__(kVThreads) quantize_v_kernel(const __half* __restrict__ v, int N, int D,
+                                                               uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ scales) {
+  __shared__ __half tile[kVTile][128 + 2];
   const int NT = num_tiles(N);
   const size_t bh = blockIdx.y;
-  const int chunk = blockIdx.x;  // 0 .. 2*NT-1
-  const int n0 = chunk * 64;
+  const int n0 = blockIdx.x * kVTile;
+  const int nk = min(kVTile, N - n0);  // 64 or 128 keys
   const int tid = threadIdx.x;
-  uint8_t* sc_block = scales + (bh * 2 * NT + chunk) * 512;
-  if (n0 >= N) {
-    for (int i = tid; i < 512; i += blockDim.x) sc_block[i] = 0;
-    return;
+  uint8_t* sc_block = scales + (bh * 2 * NT + 2 * blockIdx.x) * 512;  // two 512-byte chunks
+  for (int i = tid; i < 1024; i += kVThreads) {
+    const int chunk = i / 512, r = (i % 512) / 16, c = (i % 16) / 4;
+    if (chunk * 64 >= nk || c * 32 + r >= D) sc_block[i] = 0;  // padding: written by nobody else
   }
-  // stage 64 keys x D channels (N is a multiple of 64, so the chunk is whole)
-  const __half* src = v + (bh * N + n0) * D;
-  for (int i = tid; i < 64 * D / 2; i += blockDim.x) {
-    const int k = (2 * i) / D, d = (2 * i) % D;
-    const __half2 h = reinterpret_cast<const __half2*>(src)[i];
-    tile[k][d] = h.x;
-    tile[k][d + 1] = h.y;
+  const int vpr = D / 8;  // 16-byte pieces per key row
+  const uint4* src = reinterpret_cast<const uint4*>(v + (bh * N + n0) * D);
+  constexpr int kMaxLoads = kVTile * 128 / 8 / kVThreads;  // 8
+  uint4 buf[kMaxLoads];
+#pragma unroll
+  for (int q = 0; q < kMaxLoads; ++q) {
+    const int i = tid + q * kVThreads;
+    if (i < nk * vpr) buf[q] = __ldg(src + i);
   }
-  for (int i = tid; i < 512; i += blockDim.x) {
-    // channels >= D of the scale block are padding
-    const int r = i / 16, c = (i % 16) / 4;
-    const int d = c * 32 + r;
-    if (d >= D) sc_block[i] = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxLoads; ++q) {
+    const int i = tid + q * kVThreads;
+    if (i < nk * vpr) {
+      const int k = i / vpr, d = (i % vpr) * 8;
+      const __half2* h = reinterpret_cast<const __half2*>(&buf[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) *reinterpret_cast<__half2*>(&tile[k][d + 2 * e]) = h[e];
+    }
   }
   __syncthreads();
-  for (int t = tid; t < D * 4; t += blockDim.x) {
-    const int d = t / 4, k16 = t % 4;
+  for (int t = tid; t < D * (nk / 16); t += kVThreads) {
+    const int d = t % D, k16 = t / D;
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] = __half2float(tile[k16 * 16 + i][d]);
     const Group16 q = encode16(x);
     *reinterpret_cast<uint2*>(codes + (bh * D + d) * (static_cast<size_t>(N) / 2) + n0 / 2 + k16 * 8) =
         make_uint2(q.lo, q.hi);
-    sc_block[(d % 32) * 16 + (d / 32) * 4 + k16] = static_cast<uint8_t>(q.scale);
+    sc_block[(k16 / 4) * 512 + (d % 32) * 16 + (d / 32) * 4 + k16 % 4] = static_cast<uint8_t>(q.scale);
   }
 }
 
@@ -126,8 +152,8 @@ cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* c
 }
 
 cudaError_t launch_quantize_v(const void* v, size_t bh, int N, int D, void* codes, void* scales, cudaStream_t st) {
-  dim3 grid(2 * num_tiles(N), static_cast<unsigned>(bh));
-  quantize_v_kernel<<<grid, 256, 0, st>>>(static_cast<const __half*>(v), N, D, static_cast<uint8_t*>(codes),
+  dim3 grid(num_tiles(N), static_cast<unsigned>(bh));
+  quantize_v_kernel<<<grid, kVThreads, 0, st>>>(static_cast<const __half*>(v), N, D, static_cast<uint8_t*>(codes),
                                           static_cast<uint8_t*>(scales));
   return cudaGetLastError();
 }
