@@ -2,8 +2,8 @@
 // and bulk copies, and the tcgen05 tensor-core / tensor-memory instructions.
 //
 // Descriptor formats follow the PTX ISA (shared-memory matrix descriptor and
-// the tcgen05 instruction descriptors for .kind::f16 and
-// .kind::mxf4nvf4.block_scale).
+// the tcgen05 instruction descriptors for .kind::f16,
+// .kind::mxf4nvf4.block_scale and .kind::mxf8f6f4.block_scale).
 #pragma once
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -55,20 +55,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking: has phase `parity` of `bar` completed?  (try_wait may suspend
-// the thread for a while; test_wait returns at once.)
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -329,15 +315,12 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 // ------------------------------------------------------ swizzled offsets ----
 // Byte offset of 16-byte chunk `c` of row `r` in a K-major tile whose rows are
-// 128 / 64 / 32 bytes long, stored with the matching TMA / UMMA swizzle
-// (XOR of address bits [4,7) with [7,10) for 128 B, [4,6) with [7,9) for 64 B,
-// bit 4 with bit 7 for 32 B).  The tile base must be 1024-byte aligned.
+// 128 / 64 bytes long, stored with the matching TMA / UMMA swizzle (XOR of
+// address bits [4,7) with [7,10) for 128 B, [4,6) with [7,9) for 64 B).  The
+// tile base must be 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
 __device__ __forceinline__ uint32_t sw64_off(uint32_t r, uint32_t c) {
   return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
-}
-__device__ __forceinline__ uint32_t sw32_off(uint32_t r, uint32_t c) {
-  return r * 32u + ((c ^ ((r >> 2) & 1u)) << 4);
 }
 
 // --------------------------------------------------------- conversions ------
