@@ -203,7 +203,8 @@ THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* 
 /* Stage 2 (ThriftAttention abstract: picked pairs in FP16, the others in
  * FP4, one online softmax merging both): O [B][Hq][N][D] fp16.
  * mask: as written by thrift_select_blocks (1 FP16, 0 NVFP4; any nonzero
- * byte counts as FP16); q4/qs, k4/ks, v4/vs: the NVFP4
+ * byte counts as FP16, so masks with skipped or 8-bit pairs go to
+ * thrift_attention_tiered instead); q4/qs, k4/ks, v4/vs: the NVFP4
  * copies written by thrift_quantize_nvfp4 for Q, K and V. */
 THRIFT_API thrift_status thrift_attention(const void* Q, const void* K, const void* V, const uint8_t* mask, const void* q4,
                                const void* qs, const void* k4, const void* ks, const void* v4, const void* vs,
