@@ -72,6 +72,42 @@ def test_fused_tiered_equals_the_separate_calls(w, rho, rho8, sigma):
     assert torch.equal(o1, o2)
 
 
+EDGE = [
+    synth.GQA_N32K.with_(N=128, Hq=2, Hkv=1),                          # one key tile
+    synth.TINY_NONCAUSAL_D64.with_(N=256, blk=128, Hq=1, Hkv=1),       # two tiles, non-causal, D 64
+    synth.BATCHED_GQA_N16K.with_(N=384, B=1, Hq=2, Hkv=2),             # three tiles, Hq = Hkv
+]
+
+
+@pytest.mark.parametrize("fill", ["all8", "all8_diag16", "alternate"])
+@pytest.mark.parametrize("w", EDGE, ids=[f"N{w.N}-D{w.D}-{'c' if w.causal else 'nc'}" for w in EDGE])
+def test_eight_bit_edge_masks(w, fill):
+    """Hand-made masks on one to three key tiles: every valid pair 8-bit; all
+    8-bit but the diagonal in FP16; 8-bit and NVFP4 alternating by key tile
+    (so consecutive tiles change ring slot use), against the oracle."""
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    sh = shape_of(w)
+    nb = w.N // w.blk
+    m = np.full((w.B, w.Hq, nb, nb), 3, np.uint8)
+    if fill == "all8_diag16":
+        m[:, :, np.arange(nb), np.arange(nb)] = 1
+    elif fill == "alternate":
+        m[..., 1::2] = 0
+    if w.causal:
+        m &= np.tril(np.ones((nb, nb), np.uint8))[None, None] * 255
+    md, = to_dev(m)
+    o = thrift.attention_tiered(Qd, Kd, Vd, md, thrift.quantize_all(Qd, Kd, Vd, sh), sh,
+                                q8=thrift.quantize_all_mxfp8(Qd, Kd, Vd, sh))
+    assert thrift.last_device_error() == 0
+    o = o.cpu().numpy()
+    rows = oracle.all_rows(w.B, w.Hq, w.N)
+    mx, mean, resolved = compare_o_with_ties(o[rows[:, 0], rows[:, 1], rows[:, 2]], Q, K, V, m, rows, w.blk,
+                                             w.causal, w.sm_scale, oracle.Quantised(Q, K, V, mx8=True))
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
+    assert resolved <= 1, resolved
+
+
 def test_eight_bit_mask_without_the_copies_is_reported():
     """A 3 in the mask with no MXFP8 copies: the call returns, the device
     error word says invalid argument (1), the tile is computed in NVFP4."""
