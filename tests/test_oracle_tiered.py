@@ -129,3 +129,19 @@ def test_eight_bit_pairs_come_next_in_rank(causal):
             free8 = (mh == 3) & ~forced
             if free8.any() and free4.any():
                 assert sc[free8].min() >= sc[free4].max()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_full_eight_bit_budget_leaves_no_nvfp4_or_skipped_pair(causal):
+    """rho8 = 1: k8 = #valid - k16, so every valid pair is FP16 or 8-bit and
+    the skip budget is capped at zero whatever sigma asks; rho = 1 leaves no
+    room for 8-bit pairs."""
+    w, Q, K, V = _case(N=512, Hq=2, Hkv=1, causal=causal)
+    nb = w.N // w.blk
+    valid = _valid(nb, causal)
+    for sigma in (0.0, 0.7):
+        m = oracle.select_tiered(Q, K, w.blk, causal, w.sm_scale, 0.05, sigma, 1.0)
+        assert np.all(np.isin(m[:, :, valid], (1, 3))) and not np.any(m[:, :, ~valid])
+        assert np.array_equal(m == 1, oracle.select_tiered(Q, K, w.blk, causal, w.sm_scale, 0.05, 0.0) == 1)
+    m = oracle.select_tiered(Q, K, w.blk, causal, w.sm_scale, 1.0, 0.5, 0.5)
+    assert np.all(m[:, :, valid] == 1)
