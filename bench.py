@@ -502,6 +502,9 @@ def run_sweep(args):
     mask = torch.empty((w.B, w.Hq, sh.nb, sh.nb), dtype=torch.uint8, device=dev)
     sel_ws = torch.empty(thrift.select_workspace_bytes(sh), dtype=torch.uint8, device=dev)
     q_el, kv_el = Qd.numel(), Kd.numel()
+    q8 = thrift.quantize_mxfp8(Qd, thrift.Q, sh)      # buffers for the MXFP8 stages, allocated once
+    k8 = thrift.quantize_mxfp8(Kd, thrift.K, sh)
+    v8 = thrift.quantize_mxfp8(Vd, thrift.V, sh)
     stages = [
         ("quantise Q (NVFP4 along D)", lambda: thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, stream),
          q_el * (2 + 0.5625)),
@@ -514,6 +517,15 @@ def run_sweep(args):
         ("select, vertical-line / window W=1 (pool, score, column rank, top-k)",
          lambda: thrift.select_blocks_vertical_window(Qd, Kd, sh, w.rho, 1, mask, sel_ws, stream),
          (q_el + kv_el) * 2),
+        ("select, tiered (rho8 10%, sigma 25%: three cuts of one ranking)",
+         lambda: thrift.select_blocks_tiered(Qd, Kd, sh, w.rho, 0.25, mask, sel_ws, stream, rho8=0.1),
+         (q_el + kv_el) * 2),
+        ("quantise Q (MXFP8 along D, 8-bit pairs)",
+         lambda: thrift.quantize_mxfp8(Qd, thrift.Q, sh, q8[0], q8[1], stream), q_el * (2 + 1 + 1 / 32)),
+        ("quantise K (MXFP8 along D)", lambda: thrift.quantize_mxfp8(Kd, thrift.K, sh, k8[0], k8[1], stream),
+         kv_el * (2 + 1 + 1 / 32)),
+        ("quantise V (MXFP8 along keys)", lambda: thrift.quantize_mxfp8(Vd, thrift.V, sh, v8[0], v8[1], stream),
+         kv_el * (2 + 1 + 1 / 32)),
     ]
     print(f"| stage ({w.name}) | ms | algorithmic GB | achieved GB/s |")
     print("|---|---:|---:|---:|")

@@ -88,8 +88,9 @@ __global__ void __launch_bounds__(256) quantize_qk_mx8_kernel(const __half* __re
 }
 
 // V along keys: one CTA per (bh, 128-key tile).  The tile [128][D] is staged
-// through shared memory; thread (d, g) encodes keys 32 g .. 32 g + 31 of
-// channel d.  Groups past N (N a multiple of 64) keep scale 0 and write no codes.
+// through shared memory with 16-byte loads, all of a thread's loads in flight
+// at once; thread (d, g) encodes keys 32 g .. 32 g + 31 of channel d.  Groups
+// past N (N a multiple of 64) keep scale 0 and write no codes.
 __global__ void __launch_bounds__(256) quantize_v_mx8_kernel(const __half* __restrict__ v, int N, int D,
                                                              uint8_t* __restrict__ codes,
                                                              uint8_t* __restrict__ scales) {
@@ -99,17 +100,29 @@ __global__ void __launch_bounds__(256) quantize_v_mx8_kernel(const __half* __res
   const int n0 = blockIdx.x * kTile;
   const int nk = min(kTile, N - n0);  // 64 or 128 keys
   const int tid = threadIdx.x;
-  const __half* src = v + (bh * N + n0) * D;
-  for (int i = tid; i < nk * D / 2; i += blockDim.x) {
-    const int k = (2 * i) / D, d = (2 * i) % D;
-    const __half2 h = reinterpret_cast<const __half2*>(src)[i];
-    tile[k][d] = h.x;
-    tile[k][d + 1] = h.y;
+  const int vpr = D / 8;  // 16-byte pieces per key row
+  const uint4* src = reinterpret_cast<const uint4*>(v + (bh * N + n0) * D);
+  constexpr int kMaxLoads = 128 * 128 / 8 / 256;  // 8
+  uint4 buf[kMaxLoads];
+#pragma unroll
+  for (int q = 0; q < kMaxLoads; ++q) {
+    const int i = tid + q * 256;
+    if (i < nk * vpr) buf[q] = __ldg(src + i);
+  }
+#pragma unroll
+  for (int q = 0; q < kMaxLoads; ++q) {
+    const int i = tid + q * 256;
+    if (i < nk * vpr) {
+      const int k = i / vpr, d = (i % vpr) * 8;
+      const __half2* h = reinterpret_cast<const __half2*>(&buf[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) *reinterpret_cast<__half2*>(&tile[k][d + 2 * e]) = h[e];
+    }
   }
   __syncthreads();
   uint8_t* sc_block = scales + (bh * NT + blockIdx.x) * 512;
   for (int t = tid; t < D * 4; t += blockDim.x) {
-    const int d = t / 4, g = t % 4;
+    const int d = t % D, g = t / D;  // consecutive lanes, consecutive channels: conflict-free column reads
     if (32 * g >= nk) continue;
     float x[32];
     float amax = 0.f;
