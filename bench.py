@@ -476,19 +476,20 @@ def run_sweep(args):
     p16 = peaks["bf16_tflops"] * 1e12
     p4 = FP4_OVER_BF16 * p16
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-    # tensor-pipe rates of the two MMA kinds (measurement helper of the library)
+    # tensor-pipe rates of the two MMA kinds (the separate probe library)
+    from fp16_block_attention_b200 import probe
     stream = torch.cuda.current_stream(dev)
     for kind, name, iters in ((0, "NVFP4 mxf4nvf4 M128 N256 K64", 20000), (1, "fp16 f16 M128 N256 K16", 20000)):
-        thrift.mma_rate_probe(kind, 100, stream)
+        probe.mma_rate(kind, 100, stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        thrift.mma_rate_probe(kind, iters, stream)
+        probe.mma_rate(kind, iters, stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        if thrift.last_device_error(stream) != 0:
+        if probe.last_error(stream) != 0:
             raise RuntimeError("the MMA rate probe reported a bounded-wait timeout")
-        tf = n_sm * iters * thrift.MMA_RATE_FLOP[kind] / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        tf = n_sm * iters * probe.FLOP[kind] / (e0.elapsed_time(e1) * 1e-3) / 1e12
         print(f"tensor-pipe rate, {name}: {tf:.1f} TFLOP/s ({n_sm} SMs)")
     print()
     cases = [(w, w.rho) for w in synth.WORKLOADS] + [(synth.GQA_N32K, r) for r in (0.0, 0.01, 0.10, 1.0)]

@@ -92,7 +92,6 @@ def _load():
         "thrift_decode_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp, sz, vp], st),
         "thrift_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_last_device_error": ([vp], st),
-        "thrift_mma_rate_probe": ([st, st, vp], st),
         "thrift_strerror": ([st], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -112,7 +111,7 @@ EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quant8_bytes",
            "thrift_fused_workspace_bytes",
            "thrift_attention_fused", "thrift_fused_tiered_workspace_bytes", "thrift_attention_fused_tiered",
            "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
-           "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error", "thrift_mma_rate_probe",
+           "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error",
            "thrift_strerror")
 
 
@@ -129,12 +128,6 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
-
-
 def _dev(t: torch.Tensor, name: str, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -143,6 +136,51 @@ def _dev(t: torch.Tensor, name: str, dtype=None):
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}")
     return t
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def _guard(*specs) -> torch.device:
+    """Check the tensors of one call before the library reads them.
+
+    Each spec is (tensor, name, dtype, count, kind): a contiguous CUDA tensor
+    of `dtype` (None: any) holding exactly `count` elements (kind "n"), or at
+    least `count` bytes (kind "b", caller buffers); a None tensor is skipped.
+    All tensors must sit on one device, which is returned: the library takes
+    its stream and its static device memory from the current device, so a
+    tensor on another device, or one smaller than the shape implies, would be
+    read out of bounds on the GPU."""
+    dev = None
+    for t, name, dtype, count, kind in specs:
+        if t is None:
+            continue
+        _dev(t, name, dtype)
+        if kind == "n" and t.numel() != count:
+            raise ValueError(f"{name} holds {t.numel()} elements; the shape needs {count}")
+        if kind == "b" and _nbytes(t) < count:
+            raise ValueError(f"{name} holds {_nbytes(t)} bytes; the shape needs at least {count}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}; the call's other tensors are on {dev}")
+    return dev
+
+
+def _stream(stream, dev: torch.device):
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    elif stream.device != dev:
+        raise ValueError(f"the stream is on {stream.device}; the tensors are on {dev}")
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _counts(shape: Shape):
+    """Element counts of Q (and O), K / V and the block mask for `shape`."""
+    nq = shape.B * shape.Hq * shape.N * shape.D
+    nk = shape.B * shape.Hkv * shape.N * shape.D
+    return nq, nk, shape.B * shape.Hq * shape.nb * shape.nb
 
 
 def shape_of(Q: torch.Tensor, K: torch.Tensor, blk: int = 128, causal: bool = True,
@@ -160,14 +198,17 @@ def quant_bytes(shape: Shape, op: int):
 
 def quantize_nvfp4(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=None, stream=None):
     """NVFP4 copy of Q/K (along D) or V (along keys): (codes u8, scales u8)."""
-    _dev(x, "x", torch.float16)
+    nq, nk, _ = _counts(shape)
     nc, ns = quant_bytes(shape, op)
+    dev = _guard((x, "x", torch.float16, nq if op == Q else nk, "n"), (codes, "codes", None, nc, "b"),
+                 (scales, "scales", None, ns, "b"))
     if codes is None:
-        codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
+        codes = torch.empty(nc, dtype=torch.uint8, device=dev)
     if scales is None:
-        scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
-    _check("thrift_quantize_nvfp4", _lib.thrift_quantize_nvfp4(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
-                                                               _ptr(scales), _stream(stream)))
+        scales = torch.empty(ns, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_quantize_nvfp4", _lib.thrift_quantize_nvfp4(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
+                                                                   _ptr(scales), _stream(stream, dev)))
     return codes, scales
 
 
@@ -180,14 +221,17 @@ def quant8_bytes(shape: Shape, op: int):
 
 def quantize_mxfp8(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=None, stream=None):
     """MXFP8 copy of Q/K (along D) or V (along keys): (codes u8, scales u8)."""
-    _dev(x, "x", torch.float16)
+    nq, nk, _ = _counts(shape)
     nc, ns = quant8_bytes(shape, op)
+    dev = _guard((x, "x", torch.float16, nq if op == Q else nk, "n"), (codes, "codes", None, nc, "b"),
+                 (scales, "scales", None, ns, "b"))
     if codes is None:
-        codes = torch.empty(nc, dtype=torch.uint8, device=x.device)
+        codes = torch.empty(nc, dtype=torch.uint8, device=dev)
     if scales is None:
-        scales = torch.empty(ns, dtype=torch.uint8, device=x.device)
-    _check("thrift_quantize_mxfp8", _lib.thrift_quantize_mxfp8(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
-                                                               _ptr(scales), _stream(stream)))
+        scales = torch.empty(ns, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_quantize_mxfp8", _lib.thrift_quantize_mxfp8(_ptr(x), op, ctypes.byref(shape.c()), _ptr(codes),
+                                                                   _ptr(scales), _stream(stream, dev)))
     return codes, scales
 
 
@@ -208,17 +252,27 @@ def select_workspace_bytes(shape: Shape) -> int:
     return n.value
 
 
+def _select_args(Qt, Kt, shape: Shape, mask, ws):
+    """Checks shared by the selection calls; allocates the missing mask and
+    workspace (ws=False: the call takes none)."""
+    nq, nk, nm = _counts(shape)
+    need = select_workspace_bytes(shape) if ws is not False else 0
+    dev = _guard((Qt, "Q", torch.float16, nq, "n"), (Kt, "K", torch.float16, nk, "n"),
+                 (mask, "mask", torch.uint8, nm, "n"), (ws if ws is not False else None, "ws", None, need, "b"))
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=dev)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    return dev, mask, ws
+
+
 def select_blocks(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: float, mask=None, ws=None, stream=None):
     """Selection mask [B, Hq, nb, nb] (u8): 1 = FP16 block pair."""
-    _dev(Qt, "Q", torch.float16)
-    _dev(Kt, "K", torch.float16)
-    if mask is None:
-        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
-    if ws is None:
-        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
-                                                             float(rho), _ptr(mask), _ptr(ws), ws.numel(),
-                                                             _stream(stream)))
+    dev, mask, ws = _select_args(Qt, Kt, shape, mask, ws)
+    with torch.cuda.device(dev):
+        _check("thrift_select_blocks", _lib.thrift_select_blocks(_ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()),
+                                                                 float(rho), _ptr(mask), _ptr(ws), _nbytes(ws),
+                                                                 _stream(stream, dev)))
     return mask
 
 
@@ -227,15 +281,11 @@ def select_blocks_tiered(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: 
     """Tiered selection mask [B, Hq, nb, nb] (u8): 1 FP16, 3 MXFP8 (the next
     rho8 of the ranking), 0 NVFP4, 2 skipped (the lowest-ranked pairs, never
     forced, FP16 or 8-bit ones)."""
-    _dev(Qt, "Q", torch.float16)
-    _dev(Kt, "K", torch.float16)
-    if mask is None:
-        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
-    if ws is None:
-        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_select_blocks_tiered", _lib.thrift_select_blocks_tiered(
-        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(mask), _ptr(ws), ws.numel(),
-        _stream(stream)))
+    dev, mask, ws = _select_args(Qt, Kt, shape, mask, ws)
+    with torch.cuda.device(dev):
+        _check("thrift_select_blocks_tiered", _lib.thrift_select_blocks_tiered(
+            _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(mask), _ptr(ws),
+            _nbytes(ws), _stream(stream, dev)))
     return mask
 
 
@@ -245,15 +295,11 @@ def select_blocks_vertical_window(Qt: torch.Tensor, Kt: torch.Tensor, shape: Sha
     local window of `window` blocks, then whole key-block columns ranked by
     the pooled attention mass they receive, on the same budget as
     select_blocks."""
-    _dev(Qt, "Q", torch.float16)
-    _dev(Kt, "K", torch.float16)
-    if mask is None:
-        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
-    if ws is None:
-        ws = torch.empty(select_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_select_blocks_vertical_window", _lib.thrift_select_blocks_vertical_window(
-        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), int(window), _ptr(mask), _ptr(ws), ws.numel(),
-        _stream(stream)))
+    dev, mask, ws = _select_args(Qt, Kt, shape, mask, ws)
+    with torch.cuda.device(dev):
+        _check("thrift_select_blocks_vertical_window", _lib.thrift_select_blocks_vertical_window(
+            _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), int(window), _ptr(mask), _ptr(ws), _nbytes(ws),
+            _stream(stream, dev)))
     return mask
 
 
@@ -267,12 +313,10 @@ def select_blocks_static(Qt: torch.Tensor, Kt: torch.Tensor, shape: Shape, rho: 
     16 MiB scratch per device; larger selection workspaces are rejected.  Calls
     that overlap on the GPU race on the shared scratch.  (This binding still
     lets torch allocate the mask when none is given.)"""
-    _dev(Qt, "Q", torch.float16)
-    _dev(Kt, "K", torch.float16)
-    if mask is None:
-        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_select_blocks_static", _lib.thrift_select_blocks_static(
-        _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), _ptr(mask), _stream(stream)))
+    dev, mask, _ = _select_args(Qt, Kt, shape, mask, False)
+    with torch.cuda.device(dev):
+        _check("thrift_select_blocks_static", _lib.thrift_select_blocks_static(
+            _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), _ptr(mask), _stream(stream, dev)))
     return mask
 
 
@@ -293,16 +337,38 @@ def quantize_all(Qt, Kt, Vt, shape: Shape, stream=None) -> Quantised:
     return Quantised(q4, qs, k4, ks, v4, vs)
 
 
-def attention(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None):
-    """Mixed FP16/NVFP4 attention output O (fp16, shaped like Q)."""
-    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
-    _dev(mask, "mask", torch.uint8)
+def _qz_specs(qz, shape: Shape, with_q: bool = True):
+    """Guard specs of the NVFP4 copies (byte counts from thrift_quant_bytes)."""
+    specs = []
+    for op, names in ((Q, ("q4", "qs")), (K, ("k4", "ks")), (V, ("v4", "vs"))):
+        if op == Q and not with_q:
+            continue
+        nc, ns = quant_bytes(shape, op)
+        specs.append((getattr(qz, names[0]), names[0], None, nc, "b"))
+        specs.append((getattr(qz, names[1]), names[1], None, ns, "b"))
+    return specs
+
+
+def _attention_args(Qt, Kt, Vt, mask, qz, shape: Shape, out, extra=()):
+    nq, nk, nm = _counts(shape)
+    for t, n in ((qz.q4, "q4"), (qz.qs, "qs"), (qz.k4, "k4"), (qz.ks, "ks"), (qz.v4, "v4"), (qz.vs, "vs")):
+        if t is None:
+            raise ValueError(f"{n} is missing")
+    dev = _guard((Qt, "Q", torch.float16, nq, "n"), (Kt, "K", torch.float16, nk, "n"),
+                 (Vt, "V", torch.float16, nk, "n"), (mask, "mask", torch.uint8, nm, "n"),
+                 (out, "out", torch.float16, nq, "n"), *_qz_specs(qz, shape), *extra)
     if out is None:
         out = torch.empty_like(Qt)
-    _check("thrift_attention", _lib.thrift_attention(
-        _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
-        _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
+    return dev, out
+
+
+def attention(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, stream=None):
+    """Mixed FP16/NVFP4 attention output O (fp16, shaped like Q)."""
+    dev, out = _attention_args(Qt, Kt, Vt, mask, qz, shape, out)
+    with torch.cuda.device(dev):
+        _check("thrift_attention", _lib.thrift_attention(
+            _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
+            _ptr(qz.v4), _ptr(qz.vs), ctypes.byref(shape.c()), _ptr(out), _stream(stream, dev)))
     return out
 
 
@@ -328,15 +394,17 @@ def attention_tiered(Qt, Kt, Vt, mask, qz: Quantised, shape: Shape, out=None, st
     """attention() for masks that may hold 2 (skipped pairs, absent from the
     softmax) and, given the MXFP8 copies q8, 3 (8-bit pairs), as from
     select_blocks_tiered."""
-    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
-    _dev(mask, "mask", torch.uint8)
-    if out is None:
-        out = torch.empty_like(Qt)
+    extra = []
+    if q8 is not None:
+        for op, names in ((Q, ("q8", "qs8")), (K, ("k8", "ks8")), (V, ("v8", "vs8"))):
+            nc, ns = quant8_bytes(shape, op)
+            extra += [(getattr(q8, names[0]), names[0], None, nc, "b"), (getattr(q8, names[1]), names[1], None, ns, "b")]
+    dev, out = _attention_args(Qt, Kt, Vt, mask, qz, shape, out, extra)
     p8 = [None] * 6 if q8 is None else [_ptr(t) for t in (q8.q8, q8.qs8, q8.k8, q8.ks8, q8.v8, q8.vs8)]
-    _check("thrift_attention_tiered", _lib.thrift_attention_tiered(
-        _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
-        _ptr(qz.v4), _ptr(qz.vs), *p8, ctypes.byref(shape.c()), _ptr(out), _stream(stream)))
+    with torch.cuda.device(dev):
+        _check("thrift_attention_tiered", _lib.thrift_attention_tiered(
+            _ptr(Qt), _ptr(Kt), _ptr(Vt), _ptr(mask), _ptr(qz.q4), _ptr(qz.qs), _ptr(qz.k4), _ptr(qz.ks),
+            _ptr(qz.v4), _ptr(qz.vs), *p8, ctypes.byref(shape.c()), _ptr(out), _stream(stream, dev)))
     return out
 
 
@@ -347,17 +415,24 @@ def fused_workspace_bytes(shape: Shape) -> int:
     return n.value
 
 
-def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, stream=None):
-    """Quantise, select (budget rho) and attend in one call."""
-    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
+def _fused_args(Qt, Kt, Vt, shape: Shape, out, ws, need):
+    nq, nk, _ = _counts(shape)
+    dev = _guard((Qt, "Q", torch.float16, nq, "n"), (Kt, "K", torch.float16, nk, "n"),
+                 (Vt, "V", torch.float16, nk, "n"), (out, "out", torch.float16, nq, "n"), (ws, "ws", None, need, "b"))
     if out is None:
         out = torch.empty_like(Qt)
     if ws is None:
-        ws = torch.empty(fused_workspace_bytes(shape), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_attention_fused", _lib.thrift_attention_fused(
-        _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(),
-        _stream(stream)))
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    return dev, out, ws
+
+
+def attention_fused(Qt, Kt, Vt, shape: Shape, rho: float, out=None, ws=None, stream=None):
+    """Quantise, select (budget rho) and attend in one call."""
+    dev, out, ws = _fused_args(Qt, Kt, Vt, shape, out, ws, fused_workspace_bytes(shape))
+    with torch.cuda.device(dev):
+        _check("thrift_attention_fused", _lib.thrift_attention_fused(
+            _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), _nbytes(ws),
+            _stream(stream, dev)))
     return out
 
 
@@ -372,39 +447,44 @@ def attention_fused_tiered(Qt, Kt, Vt, shape: Shape, rho: float, rho8: float = 0
                            ws=None, stream=None):
     """Quantise (NVFP4, and MXFP8 when rho8 > 0), select four classes (FP16
     budget rho, 8-bit budget rho8, skipped share sigma) and attend in one call."""
-    for t, n in ((Qt, "Q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
-    if out is None:
-        out = torch.empty_like(Qt)
-    if ws is None:
-        ws = torch.empty(fused_tiered_workspace_bytes(shape, rho8), dtype=torch.uint8, device=Qt.device)
-    _check("thrift_attention_fused_tiered", _lib.thrift_attention_fused_tiered(
-        _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(out),
-        _ptr(ws), ws.numel(), _stream(stream)))
+    dev, out, ws = _fused_args(Qt, Kt, Vt, shape, out, ws, fused_tiered_workspace_bytes(shape, rho8))
+    with torch.cuda.device(dev):
+        _check("thrift_attention_fused_tiered", _lib.thrift_attention_fused_tiered(
+            _ptr(Qt), _ptr(Kt), _ptr(Vt), ctypes.byref(shape.c()), float(rho), float(rho8), float(sigma), _ptr(out),
+            _ptr(ws), _nbytes(ws), _stream(stream, dev)))
     return out
 
 
-MMA_RATE_FLOP = {0: 2 * 128 * 256 * 64, 1: 2 * 128 * 256 * 16}  # per product: NVFP4, fp16
-
-
 # ---- decode ------------------------------------------------------------------
+def _decode_counts(shape: Shape):
+    """Element counts of q / O [B, Hq, D], the block means [B, Hkv, nb, D] and
+    the decode mask [B, Hq, nb]."""
+    return (shape.B * shape.Hq * shape.D, shape.B * shape.Hkv * shape.nb * shape.D, shape.B * shape.Hq * shape.nb)
+
+
 def pool_keys(Kt: torch.Tensor, shape: Shape, km=None, stream=None):
     """FP32 block means of K: [B, Hkv, nb, D]."""
-    _dev(Kt, "K", torch.float16)
+    _, nk, _ = _counts(shape)
+    _, nkm, _ = _decode_counts(shape)
+    dev = _guard((Kt, "K", torch.float16, nk, "n"), (km, "km", torch.float32, nkm, "n"))
     if km is None:
-        km = torch.empty((shape.B, shape.Hkv, shape.nb, shape.D), dtype=torch.float32, device=Kt.device)
-    _check("thrift_pool_keys", _lib.thrift_pool_keys(_ptr(Kt), ctypes.byref(shape.c()), _ptr(km), _stream(stream)))
+        km = torch.empty((shape.B, shape.Hkv, shape.nb, shape.D), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_pool_keys", _lib.thrift_pool_keys(_ptr(Kt), ctypes.byref(shape.c()), _ptr(km),
+                                                         _stream(stream, dev)))
     return km
 
 
 def decode_select(qt: torch.Tensor, km: torch.Tensor, shape: Shape, rho: float, mask=None, stream=None):
     """Decode selection mask [B, Hq, nb] (u8, 1 = FP16 block) of q [B, Hq, D]."""
-    _dev(qt, "q", torch.float16)
-    _dev(km, "km", torch.float32)
+    nqd, nkm, nmask = _decode_counts(shape)
+    dev = _guard((qt, "q", torch.float16, nqd, "n"), (km, "km", torch.float32, nkm, "n"),
+                 (mask, "mask", torch.uint8, nmask, "n"))
     if mask is None:
-        mask = torch.empty((shape.B, shape.Hq, shape.nb), dtype=torch.uint8, device=qt.device)
-    _check("thrift_decode_select", _lib.thrift_decode_select(_ptr(qt), _ptr(km), ctypes.byref(shape.c()),
-                                                             float(rho), _ptr(mask), _stream(stream)))
+        mask = torch.empty((shape.B, shape.Hq, shape.nb), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_decode_select", _lib.thrift_decode_select(_ptr(qt), _ptr(km), ctypes.byref(shape.c()),
+                                                                 float(rho), _ptr(mask), _stream(stream, dev)))
     return mask
 
 
@@ -415,32 +495,43 @@ def decode_workspace_bytes(shape: Shape) -> int:
     return n.value
 
 
+def _decode_args(qt, Kt, Vt, kq, shape: Shape, out, ws, extra=()):
+    _, nk, _ = _counts(shape)
+    nqd, _, _ = _decode_counts(shape)
+    for t, n in ((kq.k4, "k4"), (kq.ks, "ks"), (kq.v4, "v4"), (kq.vs, "vs")):
+        if t is None:
+            raise ValueError(f"{n} is missing")
+    need = decode_workspace_bytes(shape)
+    dev = _guard((qt, "q", torch.float16, nqd, "n"), (Kt, "K", torch.float16, nk, "n"),
+                 (Vt, "V", torch.float16, nk, "n"), (out, "out", torch.float16, nqd, "n"), (ws, "ws", None, need, "b"),
+                 *_qz_specs(kq, shape, with_q=False), *extra)
+    if out is None:
+        out = torch.empty((shape.B, shape.Hq, shape.D), dtype=torch.float16, device=dev)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    return dev, out, ws
+
+
 def decode_attention(qt, Kt, Vt, kq: "Quantised", mask, shape: Shape, out=None, ws=None, stream=None):
     """Decode output [B, Hq, D] fp16 for the given block mask; kq holds the
     NVFP4 copies of K and V (its q4 / qs fields are not read)."""
-    for t, n in ((qt, "q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
-    if out is None:
-        out = torch.empty((shape.B, shape.Hq, shape.D), dtype=torch.float16, device=qt.device)
-    if ws is None:
-        ws = torch.empty(decode_workspace_bytes(shape), dtype=torch.uint8, device=qt.device)
-    _check("thrift_decode_attention", _lib.thrift_decode_attention(
-        _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(mask),
-        ctypes.byref(shape.c()), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    _, _, nmask = _decode_counts(shape)
+    dev, out, ws = _decode_args(qt, Kt, Vt, kq, shape, out, ws, [(mask, "mask", torch.uint8, nmask, "n")])
+    with torch.cuda.device(dev):
+        _check("thrift_decode_attention", _lib.thrift_decode_attention(
+            _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(mask),
+            ctypes.byref(shape.c()), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream, dev)))
     return out
 
 
 def decode_step(qt, Kt, Vt, kq: "Quantised", km, shape: Shape, rho: float, out=None, ws=None, stream=None):
     """Selection and attention of one decode step: O [B, Hq, D] fp16."""
-    for t, n in ((qt, "q"), (Kt, "K"), (Vt, "V")):
-        _dev(t, n, torch.float16)
-    if out is None:
-        out = torch.empty((shape.B, shape.Hq, shape.D), dtype=torch.float16, device=qt.device)
-    if ws is None:
-        ws = torch.empty(decode_workspace_bytes(shape), dtype=torch.uint8, device=qt.device)
-    _check("thrift_decode_step", _lib.thrift_decode_step(
-        _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(km),
-        ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    _, nkm, _ = _decode_counts(shape)
+    dev, out, ws = _decode_args(qt, Kt, Vt, kq, shape, out, ws, [(km, "km", torch.float32, nkm, "n")])
+    with torch.cuda.device(dev):
+        _check("thrift_decode_step", _lib.thrift_decode_step(
+            _ptr(qt), _ptr(Kt), _ptr(Vt), _ptr(kq.k4), _ptr(kq.ks), _ptr(kq.v4), _ptr(kq.vs), _ptr(km),
+            ctypes.byref(shape.c()), float(rho), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream, dev)))
     return out
 
 
@@ -451,16 +542,13 @@ def quantize_kv(Kt, Vt, shape: Shape, stream=None) -> "Quantised":
     return Quantised(None, None, k4, ks, v4, vs)
 
 
-def mma_rate_probe(kind: int, iters: int, stream=None):
-    """Launch the tensor-pipe rate probe (measurement helper, see thrift.h):
-    one CTA per SM issues `iters` products of MMA_RATE_FLOP[kind] flop each."""
-    _check("thrift_mma_rate_probe", _lib.thrift_mma_rate_probe(int(kind), int(iters), _stream(stream)))
-
-
 def last_device_error(stream=None) -> int:
-    """Synchronise and read/clear the device error word (0 = none, 4 = a bounded wait timed out,
-    1 = a kernel met a mask byte it cannot compute)."""
-    return int(_lib.thrift_last_device_error(_stream(stream)))
+    """Synchronise and read/clear the device error word of the current device
+    (or of `stream`'s device): 0 = none, 4 = a bounded wait timed out, 1 = a
+    kernel met a mask byte it cannot compute."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if stream is None else stream.device
+    with torch.cuda.device(dev):
+        return int(_lib.thrift_last_device_error(_stream(stream, dev)))
 
 
 def qk_scale_index(bh, n, g, NT, D):

@@ -1,6 +1,7 @@
 // C ABI of the library (declared in include/thrift.h): argument checks,
 // workspace carving and kernel launches.  Nothing here allocates device
 // memory.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -15,7 +16,9 @@ namespace {
 __device__ uint32_t g_device_error;
 
 constexpr int kMaxDevices = 64;
-uint32_t* g_err_ptr[kMaxDevices] = {nullptr};
+// Device address of the error word per device (atomic: first calls from
+// several host threads may overlap).
+std::atomic<uint32_t*> g_err_ptr[kMaxDevices];
 
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -85,12 +88,14 @@ FusedWs carve_fused(void* base, const thrift_shape& s, bool eight = false) {
 uint32_t* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!g_err_ptr[dev]) {
+  uint32_t* w = g_err_ptr[dev].load(std::memory_order_relaxed);
+  if (!w) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+    w = static_cast<uint32_t*>(p);
+    g_err_ptr[dev].store(w, std::memory_order_relaxed);
   }
-  return g_err_ptr[dev];
+  return w;
 }
 
 thrift_status check_shape(const thrift_shape* s) {
@@ -409,16 +414,6 @@ thrift_status thrift_last_device_error(void* stream) {
     return v == DEV_BAD_ARG ? THRIFT_ERR_INVALID_ARG : THRIFT_ERR_TIMEOUT;
   }
   return THRIFT_OK;
-}
-
-thrift_status thrift_mma_rate_probe(int kind, int iters, void* stream) {
-  if (kind < 0 || kind > 1 || iters <= 0 || iters > (1 << 24)) return THRIFT_ERR_INVALID_ARG;
-  int dev = 0, nsm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return THRIFT_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return THRIFT_ERR_CUDA;
-  uint32_t* err = device_error_word();
-  if (!err) return THRIFT_ERR_CUDA;
-  return from_cuda(launch_mma_rate(kind, iters, nsm, err, static_cast<cudaStream_t>(stream)));
 }
 
 const char* thrift_strerror(thrift_status status) {

@@ -80,9 +80,6 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
                                     const void* v4, const void* vs, const uint8_t* mask, const thrift_shape& s,
                                     void* O, const DecodeWs& w, uint32_t* err, cudaStream_t st);
 
-// Measurement helper (mma_rate.cu): back-to-back tcgen05 products, one CTA per SM.
-cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st);
-
 // MXFP8 copies of Q, K, V (codes and scales, as launch_quantize_mx8 writes them).
 struct Mx8Copies {
   const void *q8, *qs8, *k8, *ks8, *v8, *vs8;

@@ -4,8 +4,11 @@
 //
 // x / scale must be rounded exactly like a correctly rounded division: for
 // fp16 x and an E4M3 scale the quotient is either exactly an E2M1 rounding
-// tie or at least 2^-12 (relative) away from one.  q1 = x * (1/s) is within
-// 1.5 ulp of x/s; one residual step e = x - q1*s (exact by FMA),
+// tie or at least 2^-12 (relative) away from one.  The division follows
+// Markstein's correction of a reciprocal-multiply quotient (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): q1 = x * (1/s) is within
+// 1.5 ulp of x/s; the residual e = x - q1*s is exact by FMA, and
 // q = q1 + e*(1/s) lands exactly on the quotient whenever the quotient is
 // representable (the tie case) and within an ulp otherwise, which cannot move
 // it across a tie.  The scale uses the correctly rounded division amax/6.

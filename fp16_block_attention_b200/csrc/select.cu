@@ -31,6 +31,7 @@
 //            of the local window (i - W < j <= i, or |i - j| < W without the
 //            causal mask) first, then whole columns in rank order, each by
 //            descending score.
+#include <atomic>
 #include <cuda_fp16.h>
 
 #include "common.h"
@@ -441,7 +442,9 @@ cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shap
 namespace {
 __device__ __align__(256) unsigned char g_select_scratch[kSelectStaticBytes];
 constexpr int kMaxScratchDevices = 64;
-void* g_select_scratch_ptr[kMaxScratchDevices] = {nullptr};
+// Device address of the array per device.  Atomic, so that host threads whose
+// first calls on a device overlap do not race (each stores the same value).
+std::atomic<void*> g_select_scratch_ptr[kMaxScratchDevices];
 }  // namespace
 
 // Host code must not pass `g_select_scratch` itself to a kernel: on the host
@@ -452,13 +455,13 @@ cudaError_t select_static_scratch(void** ptr) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
-  if (!g_select_scratch_ptr[dev]) {
-    void* p = nullptr;
+  void* p = g_select_scratch_ptr[dev].load(std::memory_order_relaxed);
+  if (!p) {
     e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return e;
-    g_select_scratch_ptr[dev] = p;
+    g_select_scratch_ptr[dev].store(p, std::memory_order_relaxed);
   }
-  *ptr = g_select_scratch_ptr[dev];
+  *ptr = p;
   return cudaSuccess;
 }
 

@@ -1,14 +1,17 @@
-// Measurement helper, not part of the method's path: the sustained issue and
-// execution rate of the two tcgen05 MMA kinds the attention kernels use, so the
-// FP4 and FP16 tensor peaks of the blended roofline can be checked on the
-// machine at hand.  One CTA per SM allocates tensor memory, zeroes its shared-
+// Measurement helper, not part of the method's path and not part of
+// libthrift.so: a separate library (libthrift_probe.so) that the benchmark's
+// sweep loads to time the sustained issue and execution rate of the two
+// tcgen05 MMA kinds the attention kernels use, so the FP4 and FP16 tensor
+// peaks of the blended roofline can be checked on the machine at hand.  One CTA per SM allocates tensor memory, zeroes its shared-
 // memory operands (so every product is exactly zero), and issues `iters`
 // back-to-back M = 128, N = 256 products into one accumulator:
 //   kind 0: .kind::mxf4nvf4.block_scale.scale_vec::4X, K = 64 (E2M1, UE4M3 scales)
 //   kind 1: .kind::f16 (fp16 operands, fp32 accumulator), K = 16
 // The caller times the launch; the work is iters x 2 x 128 x 256 x K flop per CTA.
-#include "common.h"
-#include "ptx.cuh"
+#include <cuda_runtime.h>
+
+#include "../csrc/common.h"
+#include "../csrc/ptx.cuh"
 
 namespace thrift {
 namespace {
@@ -71,7 +74,8 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint32_t* e
   }
 }
 
-}  // namespace
+// The probe's own device error word (bounded-wait timeouts).
+__device__ uint32_t g_probe_error;
 
 cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaStream_t st) {
   const size_t smem = sizeof(RateSmem) + 1024;
@@ -88,4 +92,38 @@ cudaError_t launch_mma_rate(int kind, int iters, int ctas, uint32_t* err, cudaSt
   return cudaGetLastError();
 }
 
+}  // namespace
 }  // namespace thrift
+
+#define PROBE_API extern "C" __attribute__((visibility("default")))
+
+// Launch one CTA per SM of the current device, each issuing `iters`
+// back-to-back M = 128, N = 256 products of `kind` (0: NVFP4 K = 64, 1: fp16
+// K = 16), asynchronously on `stream`.  Returns 0, 1 for kind not in {0, 1} or
+// iters not in [1, 2^24] (checked before any launch), 3 for a CUDA error.
+PROBE_API int thrift_probe_mma_rate(int kind, int iters, void* stream) {
+  if (kind < 0 || kind > 1 || iters <= 0 || iters > (1 << 24)) return 1;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 3;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 3;
+  void* err = nullptr;
+  if (cudaGetSymbolAddress(&err, thrift::g_probe_error) != cudaSuccess) return 3;
+  return thrift::launch_mma_rate(kind, iters, nsm, static_cast<uint32_t*>(err), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? 0
+             : 3;
+}
+
+// Synchronise `stream`, read and clear the probe's error word: 0, or 4 if a
+// probe kernel gave up its bounded wait; 3 for a CUDA error.
+PROBE_API int thrift_probe_last_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return 3;
+  void* err = nullptr;
+  if (cudaGetSymbolAddress(&err, thrift::g_probe_error) != cudaSuccess) return 3;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return 3;
+  if (v == 0) return 0;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return 3;
+  return 4;
+}

@@ -194,7 +194,11 @@ THRIFT_API thrift_status thrift_select_blocks_vertical_window(const void* Q, con
  *     any stream capture;
  *   - every call shares the array and it keeps the last call's contents
  *     (nothing needs clearing: the kernels overwrite all they read); calls
- *     whose kernels overlap on the GPU, e.g. on two streams, race on it.
+ *     whose kernels overlap on the GPU, e.g. on two streams, race on it;
+ *   - the looked-up address is kept for the life of the process, so a
+ *     device reset (cudaDeviceReset) invalidates it, as it invalidates the
+ *     device error word's (thrift_last_device_error): do not call the
+ *     library on a device after resetting it.
  * Arguments and the mask output are as for thrift_select_blocks. */
 #define THRIFT_SELECT_STATIC_BYTES ((size_t)16 << 20)
 THRIFT_API thrift_status thrift_select_blocks_static(const void* Q, const void* K, const thrift_shape* shape,
@@ -310,21 +314,6 @@ THRIFT_API thrift_status thrift_decode_step(const void* q, const void* K, const 
  * cannot compute; THRIFT_ERR_CUDA if the synchronisation failed.  The word
  * keeps the first error recorded. */
 THRIFT_API thrift_status thrift_last_device_error(void* stream);
-
-/* Measurement helper, not part of the method (the pages have no counterpart):
- * launches one CTA per SM, each issuing `iters` back-to-back M = 128, N = 256
- * tcgen05 products from zeroed shared-memory operands into one tensor-memory
- * accumulator, so the caller can time the tensor pipe's rate for the two MMA
- * kinds the attention kernels use.
- *   kind 0: NVFP4 block-scaled (.kind::mxf4nvf4, scale_vec::4X), K = 64 per
- *           product: 2 * 128 * 256 * 64 flop.
- *   kind 1: fp16 (.kind::f16, fp32 accumulator), K = 16 per product:
- *           2 * 128 * 256 * 16 flop.
- * Work per launch = (number of SMs) * iters * flop per product.  Asynchronous
- * on `stream`; nothing is read or written in global memory except the device
- * error word on a bounded-wait timeout.  Returns THRIFT_ERR_INVALID_ARG for
- * kind not in {0, 1} or iters not in [1, 2^24]. */
-THRIFT_API thrift_status thrift_mma_rate_probe(int kind, int iters, void* stream);
 
 /* Static, human-readable name of a status. */
 THRIFT_API const char* thrift_strerror(thrift_status status);

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import fp16_block_attention_b200 as thrift
 
@@ -87,12 +88,14 @@ def test_null_pointers_and_bad_rho_are_rejected_before_launch():
     assert lib.thrift_attention_fused(fake, fake, fake, sh, 0.05, fake, fake, 8, None) == 5
 
 
-def test_mma_rate_probe_rejects_bad_arguments_before_launch():
-    lib = thrift.lib()
-    assert lib.thrift_mma_rate_probe(2, 10, None) == 1
-    assert lib.thrift_mma_rate_probe(-1, 10, None) == 1
-    assert lib.thrift_mma_rate_probe(0, 0, None) == 1
-    assert lib.thrift_mma_rate_probe(1, (1 << 24) + 1, None) == 1
+def test_mma_rate_probe_lives_outside_the_library_and_rejects_bad_arguments():
+    from fp16_block_attention_b200 import probe
+    assert not hasattr(thrift.lib(), "thrift_mma_rate_probe")
+    lib = probe.lib()
+    assert lib.thrift_probe_mma_rate(2, 10, None) == 1
+    assert lib.thrift_probe_mma_rate(-1, 10, None) == 1
+    assert lib.thrift_probe_mma_rate(0, 0, None) == 1
+    assert lib.thrift_probe_mma_rate(1, (1 << 24) + 1, None) == 1
 
 
 def test_workspace_sizes_cover_the_parts():
@@ -140,3 +143,43 @@ def test_decode_arguments_are_rejected_before_launch():
     assert lib.thrift_decode_attention(*args, fake, sh, fake, fake, 16, None) == 5       # workspace too small
     assert lib.thrift_decode_step(*args, fake, sh, -0.1, fake, fake, 1 << 30, None) == 1
     assert lib.thrift_decode_step(*args, fake, sh, 0.05, fake, None, 0, None) == 5
+
+
+class _FakeCuda:
+    """Stand-in for a CUDA tensor (no GPU here): what the binding's checks read."""
+
+    def __init__(self, numel, dtype=torch.float16, device="cuda:0", contiguous=True):
+        self._n, self.dtype, self.device, self._c = numel, dtype, torch.device(device), contiguous
+        self.is_cuda = True
+
+    def numel(self):
+        return self._n
+
+    def element_size(self):
+        return torch.empty(0, dtype=self.dtype).element_size()
+
+    def is_contiguous(self):
+        return self._c
+
+
+def test_binding_checks_sizes_and_devices_before_calling_the_library():
+    sh = thrift.Shape(1, 4, 2, 256, 64, 64, True)
+    nq, nk, nm = 4 * 256 * 64, 2 * 256 * 64, 4 * 4 * 4
+    ok = [(_FakeCuda(nq), "Q", torch.float16, nq, "n"), (_FakeCuda(nk), "K", torch.float16, nk, "n"),
+          (_FakeCuda(nm, torch.uint8), "mask", torch.uint8, nm, "n")]
+    assert thrift._guard(*ok) == torch.device("cuda:0")
+    assert thrift._counts(sh) == (nq, nk, nm)
+    with pytest.raises(ValueError, match="elements"):  # an undersized Q
+        thrift._guard((_FakeCuda(nq - 1), "Q", torch.float16, nq, "n"), *ok[1:])
+    with pytest.raises(ValueError, match="cuda:1"):  # K on another device
+        thrift._guard(ok[0], (_FakeCuda(nk, device="cuda:1"), "K", torch.float16, nk, "n"))
+    with pytest.raises(ValueError, match="bytes"):  # a workspace smaller than the shape needs
+        thrift._guard(ok[0], (_FakeCuda(100, torch.uint8), "ws", None, 101, "b"))
+    # a float32 workspace counts bytes, not elements
+    assert thrift._guard((_FakeCuda(26, torch.float32), "ws", None, 101, "b")) == torch.device("cuda:0")
+    with pytest.raises(ValueError, match="float16"):
+        thrift._guard((_FakeCuda(nq, torch.float32), "Q", torch.float16, nq, "n"))
+    with pytest.raises(ValueError, match="contiguous"):
+        thrift._guard((_FakeCuda(nq, contiguous=False), "Q", torch.float16, nq, "n"))
+    with pytest.raises(ValueError, match="CUDA"):
+        thrift.attention_fused(torch.zeros(nq, dtype=torch.float16), None, None, sh, 0.05)

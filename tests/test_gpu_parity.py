@@ -188,6 +188,7 @@ def test_gap_recovered_agrees_with_oracle():
 
 
 def test_mma_rate_probe_runs_without_error():
-    thrift.mma_rate_probe(0, 64)
-    thrift.mma_rate_probe(1, 64)
-    assert thrift.last_device_error() == 0
+    from fp16_block_attention_b200 import probe
+    probe.mma_rate(0, 64)
+    probe.mma_rate(1, 64)
+    assert probe.last_error() == 0
