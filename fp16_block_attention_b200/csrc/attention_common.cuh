@@ -53,18 +53,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // inline.  All warp roles' loops run at once on an SM and share its
 // instruction caches, so where a kernel's waits sit decides how often its
 // warps stall on instruction fetch; a kernel picks the form per role by
-// measurement.
+// measurement.  TAG makes separate copies of the slow path: a kernel whose
+// warpgroups run with different register counts (setmaxnreg) gives each
+// count its own copy, since one function cannot be allocated for both.
+template <int TAG>
 static __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                        uint32_t* err, uint32_t code) {
   return wait_or_abort(bar, parity, abort, err, code);
 }
 
-template <bool OUT_OF_LINE>
+template <bool OUT_OF_LINE, int TAG = 0>
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
                                              uint32_t code) {
   if constexpr (OUT_OF_LINE) {
     if (mbar_try_wait(bar, parity)) return true;
-    return wait_or_abort_slow(bar, parity, abort, err, code);
+    return wait_or_abort_slow<TAG>(bar, parity, abort, err, code);
   } else {
     return wait_or_abort(bar, parity, abort, err, code);
   }
@@ -86,6 +89,12 @@ __device__ __forceinline__ bool softmax_bar_or(bool flag) {
   return r != 0;
 }
 
+
+// Barrier of all `count` threads of the CTA that warps may reach from
+// different places in the code (barrier 2, not the aligned __syncthreads).
+__device__ __forceinline__ void cta_barrier_all(uint32_t count) {
+  asm volatile("barrier.sync 2, %0;" ::"r"(count) : "memory");
+}
 
 // Named barriers among a subset of the CTA's warps (count = threads taking part).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {

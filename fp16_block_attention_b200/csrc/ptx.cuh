@@ -237,6 +237,18 @@ __device__ __forceinline__ void mma_mxf8_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Move registers between the warpgroups of a CTA (executed by all threads of
+// a warpgroup).  The sum over warpgroups must stay within the registers the
+// CTA was launched with, or the increase waits for ever.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread
 // has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
