@@ -551,7 +551,37 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       if (failed) continue;
       const int kt = tile_of(it);
       const bool fp16 = fp16_of(it), eight = eight_of(it);
+      // All of the tile's waits come first, so that everything from the S
+      // load to the P stores is one stretch of code the compiler can
+      // interleave.  S of this tile:
       failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_s_full[grp], j & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      // this group's P buffers (the shared-memory P4 codes and the tensor-
+      // memory P4 scales) and its O are free once its previous tile's P V
+      // product is done;
+      if (!failed && j > 0)
+        failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (j - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      // the tensor-memory P region is taken in processing order: the P V
+      // product of its previous user must have been issued (a counter, so no
+      // barrier phase can be mistaken for another) and be complete.
+      if (!failed && (fp16 || (EIGHT && eight)) && pt_before > 0) {
+        if (ms.pt_issued < pt_before) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ms.pt_issued < pt_before) {
+            if (ms.abort) {
+              failed = true;
+              break;
+            }
+            if (globaltimer_ns() - t0 > kWaitNs) {
+              record_error(p.err, DEV_TIMEOUT_OTHER);
+              ms.abort = 1;
+              failed = true;
+              break;
+            }
+          }
+        }
+        if (!failed)
+          failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_pt_free, (pt_before - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      }
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) continue;
       tc_fence_after();
@@ -615,39 +645,6 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           sfw[g >> 2] |= sbyte << (8 * (g & 3));
         }
       }
-
-      // This group's P buffers (the shared-memory P4 codes and the tensor-
-      // memory P4 scales) and its O are free once its previous tile's P V
-      // product is done.
-      if (j > 0) {
-        failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (j - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
-        failed = __any_sync(0xffffffffu, failed);
-        if (failed) continue;
-      }
-      // The tensor-memory P region is taken in processing order: the P V
-      // product of its previous user must have been issued (a counter, so no
-      // barrier phase can be mistaken for another) and be complete.
-      if (fp16 || (EIGHT && eight)) {
-        if (pt_before > 0) {
-          bool ok = true;
-          if (ms.pt_issued < pt_before) {
-            const uint64_t t0 = globaltimer_ns();
-            while (ms.pt_issued < pt_before) {
-              if (ms.abort) { ok = false; break; }
-              if (globaltimer_ns() - t0 > kWaitNs) {
-                record_error(p.err, DEV_TIMEOUT_OTHER);
-                ms.abort = 1;
-                ok = false;
-                break;
-              }
-            }
-          }
-          if (ok) ok = bounded_wait<kOolSoftmax, 2>(&ms.bar_pt_free, (pt_before - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
-          failed = __any_sync(0xffffffffu, !ok);
-          if (failed) continue;
-        }
-      }
-      tc_fence_after();
 
       // P * 2^11 = 2^(S*c + 11 - M) for the row's 128 keys, encoded as fp16
       // or as NVFP4 (each group folds 1/scale into the exponent).
