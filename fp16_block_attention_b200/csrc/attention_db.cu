@@ -32,8 +32,9 @@
 // thread's row maximum.
 //
 // Tensor memory (512 columns): S (128), O_0 and O_1 (128 each), the fp16 /
-// 8-bit P operand (64), the scale factors of Q4, K4, V4 and of each group's
-// P4, and the MXFP8 scales of the 8-bit instantiation.  The S buffer is
+// 8-bit P operand (64), the scale factors of Q4, of K4 (two buffers, so the
+// next tile's are copied while the S buffer is still in use), of V4 and of
+// each group's P4, and the MXFP8 scales of the 8-bit instantiation.  The S buffer is
 // single: the S issuer computes S of the next key tile as soon as the
 // previous tile's group has loaded its S into registers, early in that
 // group's iteration.  The fp16 / 8-bit P region is shared by both groups in
@@ -82,13 +83,15 @@ constexpr uint32_t kDColS = 0;      // S of the key tile being handed to a group
 constexpr uint32_t kDColO = 128;    // O of group g at 128 + 128 g, D columns
 constexpr uint32_t kDColP = 384;    // fp16 P (64 columns) or P8 (32 columns), shared in processing order
 constexpr uint32_t kDColSFQ = 448;  // Q4 scales, 4 columns per 64-wide chunk of D
-constexpr uint32_t kDColSFK = 456;  // K4 scales of the key tile being multiplied
+constexpr uint32_t kDColSFK = 456;  // K4 scales of even processed key tiles (odd ones at kDColSFK1)
 constexpr uint32_t kDColSFV = 464;  // V4 scales of the key tile being multiplied
 constexpr uint32_t kDColSFP = 472;  // P4 scales of group g at 8 g: 64-key chunk c of row r at 4 c + r / 32
                                     // (P8: byte k of that column for keys 64 c + 32 k ..)
 constexpr uint32_t kDColSFQ8 = 488;  // Q8 scales (byte g: channels 32 g ..)
-constexpr uint32_t kDColSFK8 = 492;  // K8 scales of the key tile being multiplied
+constexpr uint32_t kDColSFK8 = 492;  // K8 scales of even processed key tiles (odd ones at kDColSFK81)
 constexpr uint32_t kDColSFV8 = 496;  // V8 scales (byte g: keys 32 g ..)
+constexpr uint32_t kDColSFK81 = 500;  // K8 scales of odd processed key tiles
+constexpr uint32_t kDColSFK1 = 504;   // K4 scales of odd processed key tiles
 
 template <int D, bool EIGHT>
 struct SmemDB {
@@ -375,21 +378,28 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
           ++uk16;
         }
+        // The K scales go to tensor memory before the wait for the S buffer,
+        // into the buffer of this tile's parity (the product two tiles back,
+        // which read it, precedes the copy in this thread's tcgen05 order), so
+        // only the products themselves follow the S buffer's release.
+        tc_fence_after();
+        const uint32_t sfk = tm + ((it & 1) ? kDColSFK1 : kDColSFK);
+        const uint32_t sfk8 = tm + ((it & 1) ? kDColSFK81 : kDColSFK8);
+        if (EIGHT && eight) {
+          tmem_cp_32x128b_x4(sfk8, make_sdesc(sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK8Bytes, 16, 128,
+                                              LAYOUT_NONE));
+        } else if (!fp16) {
+          const uint32_t ksf = sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK4Bytes + L::kV4Bytes;
+          for (int c = 0; c < D / 64; ++c)
+            tmem_cp_32x128b_x4(sfk + 4 * c, make_sdesc(ksf + 512 * c, 16, 128, LAYOUT_NONE));
+        }
         // The one S buffer: the group of the previous key tile must have
         // loaded its S.  (Barriers and phases count processed tiles, it.)
         if (it >= 1) {
           const int pv = it - 1;
           if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_s_free[pv & 1], (pv >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
             break;
-        }
-        tc_fence_after();
-        if (EIGHT && eight) {
-          tmem_cp_32x128b_x4(tm + kDColSFK8, make_sdesc(sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK8Bytes, 16,
-                                                        128, LAYOUT_NONE));
-        } else if (!fp16) {
-          const uint32_t ksf = sbase + L::kSlot4 + slot * L::kSlot4Bytes + L::kK4Bytes + L::kV4Bytes;
-          for (int c = 0; c < D / 64; ++c)
-            tmem_cp_32x128b_x4(tm + kDColSFK + 4 * c, make_sdesc(ksf + 512 * c, 16, 128, LAYOUT_NONE));
+          tc_fence_after();
         }
         const uint32_t dS = tm + kDColS;
         if (EIGHT && eight) {
@@ -400,14 +410,14 @@ __global__ void __launch_bounds__(kDBThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
             mma_mxf8(dS, make_sdesc(q8 + 32 * kk, 16, sbo8, sw8), make_sdesc(k8 + 32 * kk, 16, sbo8, sw8),
-                     idesc_mxf8(128, 128, kk, kk), tm + kDColSFQ8, tm + kDColSFK8, kk > 0);
+                     idesc_mxf8(128, 128, kk, kk), tm + kDColSFQ8, sfk8, kk > 0);
         } else if (!fp16) {
           const uint32_t q4 = sbase + L::kQ4;
           const uint32_t k4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
             mma_nvf4(dS, make_sdesc(q4 + 32 * c, 16, sbo4, sw4), make_sdesc(k4 + 32 * c, 16, sbo4, sw4),
-                     idesc_nvf4(128, 128), tm + kDColSFQ + 4 * c, tm + kDColSFK + 4 * c, c > 0);
+                     idesc_nvf4(128, 128), tm + kDColSFQ + 4 * c, sfk + 4 * c, c > 0);
         } else {
           const uint32_t q16 = sbase + L::kQ16, k16 = sbase + L::kSlot16;
 #pragma unroll
@@ -610,6 +620,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       const float smax = max128(s, gh);
       // t = fl32(S * sm_scale * log2 e) is monotone in S: max t = fl32(max S * c).
       const float Mn = fmaxf(M, ceilf(smax * c2));
+
       const float alpha = (M == -INFINITY) ? 0.f : exp2_int(M - Mn);
       const float Mx = (Mn == -INFINITY) ? 0.f : Mn;
       const float base = static_cast<float>(kPLog2) - Mx;  // exponent offset of P * 2^11
@@ -646,6 +657,10 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
       }
 
+      if (!fp16) {
+        tmem_st1(lane_base + kDColSFP + 8 * grp + quad, sfw[0]);
+        tmem_st1(lane_base + kDColSFP + 8 * grp + 4 + quad, sfw[1]);
+      }
       // P * 2^11 = 2^(S*c + 11 - M) for the row's 128 keys, encoded as fp16
       // or as NVFP4 (each group folds 1/scale into the exponent).
       float rs = 0.f;
@@ -697,11 +712,6 @@ __global__ void __launch_bounds__(kDBThreads, 1)
             *reinterpret_cast<uint4*>(d4 + sw64_off(r, c)) = w;
           }
         }
-        // Scale factors of a 128-row A operand: the MMA reads row r's four
-        // scales of 64-key chunk c from lane r, column base + 4c + r / 32
-        // (8-bit: byte k of that column for keys 64 c + 32 k ..).
-        tmem_st1(lane_base + kDColSFP + 8 * grp + quad, sfw[0]);
-        tmem_st1(lane_base + kDColSFP + 8 * grp + 4 + quad, sfw[1]);
       }
       l = l * alpha + rs;
       // Rescale this group's O when its maximum grew (rows with alpha = 1 are
