@@ -92,6 +92,7 @@ def _load():
         "thrift_decode_attention": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, vp, vp, sz, vp], st),
         "thrift_decode_step": ([vp, vp, vp, vp, vp, vp, vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_last_device_error": ([vp], st),
+        "thrift_set_wait_limit": ([ctypes.c_uint64], st),
         "thrift_strerror": ([st], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -112,7 +113,7 @@ EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quant8_bytes",
            "thrift_attention_fused", "thrift_fused_tiered_workspace_bytes", "thrift_attention_fused_tiered",
            "thrift_pool_keys", "thrift_decode_select", "thrift_decode_workspace_bytes",
            "thrift_decode_attention", "thrift_decode_step", "thrift_last_device_error",
-           "thrift_strerror")
+           "thrift_set_wait_limit", "thrift_strerror")
 
 
 def lib():
@@ -549,6 +550,15 @@ def last_device_error(stream=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if stream is None else stream.device
     with torch.cuda.device(dev):
         return int(_lib.thrift_last_device_error(_stream(stream, dev)))
+
+
+WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
+def set_wait_limit(ns: int):
+    """Bound (ns) of every wait inside the prefill attention kernels launched
+    from now on (process-wide; 2 s by default)."""
+    _check("thrift_set_wait_limit", _lib.thrift_set_wait_limit(int(ns)))
 
 
 def qk_scale_index(bh, n, g, NT, D):

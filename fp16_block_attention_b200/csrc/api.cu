@@ -3,6 +3,7 @@
 // memory.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 
 #include "common.h"
@@ -96,6 +97,20 @@ uint32_t* device_error_word() {
     g_err_ptr[dev].store(w, std::memory_order_relaxed);
   }
   return w;
+}
+
+namespace {
+std::atomic<uint64_t> g_wait_ns{kWaitNs};
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
+int test_withhold_tile() {
+  const char* v = std::getenv("THRIFT_TEST_WITHHOLD_TILE");
+  if (!v || !*v) return -1;
+  char* end = nullptr;
+  const long t = std::strtol(v, &end, 10);
+  return (end && *end == 0 && t >= 0 && t < (1L << 20)) ? static_cast<int>(t) : -1;
 }
 
 thrift_status check_shape(const thrift_shape* s) {
@@ -413,6 +428,12 @@ thrift_status thrift_last_device_error(void* stream) {
     if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return THRIFT_ERR_CUDA;
     return v == DEV_BAD_ARG ? THRIFT_ERR_INVALID_ARG : THRIFT_ERR_TIMEOUT;
   }
+  return THRIFT_OK;
+}
+
+thrift_status thrift_set_wait_limit(uint64_t ns) {
+  if (ns < 1000 || ns > 60000000000ull) return THRIFT_ERR_INVALID_ARG;
+  g_wait_ns.store(ns, std::memory_order_relaxed);
   return THRIFT_OK;
 }
 

@@ -194,29 +194,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       int u4 = 0, u16 = 0, u16k_only = 0;
       for (int kt = 0; kt < n_kt && !ms.abort; ++kt) {
         const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
+        // failure-detection test: this tile's slots are taken but its copies
+        // are never issued, so the waits of their consumers run out
+        const bool hold = kt == p.withhold;
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
-          if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (use > 0 && !wait_or_abort(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns))
             break;
-          uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
-          mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx4);
-          tma_load_3d(st, &mK4, &ms.bar_full4[slot], 0, kt * 128, bhk);
-          tma_load_3d(st + L::kK4Bytes, &mV4, &ms.bar_full4[slot], kt * 64, 0, bhk);
-          bulk_load(st + L::kK4Bytes + L::kV4Bytes, p.ks + (static_cast<size_t>(bhk) * p.NT + kt) * L::kKSFBytes,
-                    L::kKSFBytes, &ms.bar_full4[slot]);
-          bulk_load(st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes,
-                    p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * kt) * 512, L::kVSFBytes, &ms.bar_full4[slot]);
+          if (!hold) {
+            uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
+            mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx4);
+            tma_load_3d(st, &mK4, &ms.bar_full4[slot], 0, kt * 128, bhk);
+            tma_load_3d(st + L::kK4Bytes, &mV4, &ms.bar_full4[slot], kt * 64, 0, bhk);
+            bulk_load(st + L::kK4Bytes + L::kV4Bytes, p.ks + (static_cast<size_t>(bhk) * p.NT + kt) * L::kKSFBytes,
+                      L::kKSFBytes, &ms.bar_full4[slot]);
+            bulk_load(st + L::kK4Bytes + L::kV4Bytes + L::kKSFBytes,
+                      p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * kt) * 512, L::kVSFBytes, &ms.bar_full4[slot]);
+          }
           ++u4;
         }
         if (c != 0u) {
           // K16 and V16 have separate slots: K16 frees when S is done, V16 when P V is done.
           uint8_t* st = sm + L::kSlot16;
-          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns))
             break;
+          if (hold) {
+            ++u16;
+            continue;
+          }
           mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
           for (int pnl = 0; pnl < D / 64; ++pnl)
             tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
-          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
+          if (u16 > 0 && !wait_or_abort(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)) {
             ++u16k_only;
             break;
           }
@@ -227,11 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Let every copy this thread issued land before the CTA can exit.
-      mbar_wait(&ms.bar_q, 0, kWaitNs);
+      mbar_wait(&ms.bar_q, 0, p.wait_ns);
       for (int s = 0; s < kNS4; ++s)
-        if (u4 > s) mbar_wait(&ms.bar_full4[s], ((u4 - 1 - s) / kNS4) & 1, kWaitNs);
-      if (u16 + u16k_only > 0) mbar_wait(&ms.bar_full_k16, (u16 + u16k_only - 1) & 1, kWaitNs);
-      if (u16 > 0) mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, kWaitNs);
+        if (u4 > s) mbar_wait(&ms.bar_full4[s], ((u4 - 1 - s) / kNS4) & 1, p.wait_ns);
+      if (u16 + u16k_only > 0) mbar_wait(&ms.bar_full_k16, (u16 + u16k_only - 1) & 1, p.wait_ns);
+      if (u16 > 0) mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t p16 = sbase + L::kP16, p4 = sbase + L::kP4, psf = sbase + L::kPSF;
       constexpr uint32_t sbo4 = (D == 128) ? 512u : 256u;
       constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
-      bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
+      bool ok = wait_or_abort(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns);
       tc_fence_after();
       if (ok)
         for (int c = 0; c < D / 64; ++c)
@@ -280,12 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         if (c != 0xFu) {
           const int slot = u4 % kNS4, use = u4 / kNS4;
-          if (!wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
+          if (!wait_or_abort(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns)) return false;
           slot4_of[kt & 1] = slot;
           ++u4;
         }
         if (c != 0u) {
-          if (!wait_or_abort(&ms.bar_full_k16, u16k & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
+          if (!wait_or_abort(&ms.bar_full_k16, u16k & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns)) return false;
           ++u16k;
         }
         tc_fence_after();
@@ -296,11 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; ok && kt < n_kt; ++kt) {
         if (kt + 1 < n_kt) {
           if (!wait_loads(kt + 1)) break;
-          if (!wait_or_abort(&ms.bar_s_free, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) break;
+          if (!wait_or_abort(&ms.bar_s_free, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)) break;
           tc_fence_after();
           issue_s(kt + 1);
         }
-        if (!wait_or_abort(&ms.bar_p_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) break;
+        if (!wait_or_abort(&ms.bar_p_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
         const uint32_t sfset = tm + kColSF + 24 * (kt & 1);
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (c != 0u) {
-          if (!wait_or_abort(&ms.bar_full_v16, u16v & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) break;
+          if (!wait_or_abort(&ms.bar_full_v16, u16v & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns)) break;
           ++u16v;
           tc_fence_after();
           const uint32_t v16 = sbase + L::kSlot16 + L::kK16Bytes;
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // drain: every tensor-core operation of this CTA completes before exit
       mma_commit(&ms.bar_drain);
-      mbar_wait(&ms.bar_drain, 0, kWaitNs);
+      mbar_wait(&ms.bar_drain, 0, p.wait_ns);
     }
     __syncwarp();
   } else {
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t c = SKIP ? (ms.cls[kt] & 0xFu) : ms.cls[kt];  // FP16 flags
       const bool fp16 = (c >> (a * 2 + kh)) & 1u;
       const bool need16 = c != 0u, need4 = c != 0xFu;
-      if (!failed) failed = !wait_or_abort(&ms.bar_s_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (!failed) failed = !wait_or_abort(&ms.bar_s_full, kt & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       tc_fence_after();
       float s[kKPT];
@@ -443,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (kt > 0) {
         failed = __any_sync(0xffffffffu,
-                            !wait_or_abort(&ms.bar_o_done, (kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA));
+                            !wait_or_abort(&ms.bar_o_done, (kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns));
         if (failed) continue;  // the next joint barrier ends the loop for every softmax thread
         tc_fence_after();
       }
@@ -517,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- epilogue: O / l -> fp16 (both carry the 2^11 pre-scale) ----
-    if (!failed) failed = !wait_or_abort(&ms.bar_o_done, (n_kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+    if (!failed) failed = !wait_or_abort(&ms.bar_o_done, (n_kt - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
     failed = __any_sync(0xffffffffu, failed);
     ms.red_l[part][r] = l;
     if (!softmax_bar_or<kSoftmaxThreads>(failed)) {
@@ -602,6 +611,8 @@ cudaError_t launch_d(const void* Q, const void* K, const void* V, const uint8_t*
   prm.ks8 = eight ? static_cast<const uint8_t*>(eight->ks8) : nullptr;
   prm.vs8 = eight ? static_cast<const uint8_t*>(eight->vs8) : nullptr;
   prm.eight = eight ? 1 : 0;
+  prm.wait_ns = wait_limit_ns();
+  prm.withhold = test_withhold_tile();
   if (s.blk == 128) return launch_attention_db<D>(mQ16, mK16, mV16, mQ4, mK4, mV4, mQ8, mK8, mV8, prm, st);
   if (eight) return cudaErrorInvalidValue;  // the entry point rejects this shape first
   const unsigned grid = static_cast<unsigned>(BHq * prm.NT);

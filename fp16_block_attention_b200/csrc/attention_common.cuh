@@ -26,17 +26,20 @@ struct Params {
   const uint8_t* ks8;
   const uint8_t* vs8;
   int eight;  // the MXFP8 copies are present: the 8-bit instantiation
+  uint64_t wait_ns;  // bound of every wait in the kernel (thrift_set_wait_limit)
+  int withhold;      // failure-detection test only: the processed key tile whose copies the producer
+                     // does not issue (its consumers' waits then run out), or -1
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
-                                              uint32_t code) {
+                                              uint32_t code, uint64_t limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < (1u << 30); ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 63u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_error(err, code);
         *abort = 1;
         return false;
@@ -58,18 +61,18 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // count its own copy, since one function cannot be allocated for both.
 template <int TAG>
 static __device__ __noinline__ bool wait_or_abort_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                       uint32_t* err, uint32_t code) {
-  return wait_or_abort(bar, parity, abort, err, code);
+                                                       uint32_t* err, uint32_t code, uint64_t limit_ns) {
+  return wait_or_abort(bar, parity, abort, err, code, limit_ns);
 }
 
 template <bool OUT_OF_LINE, int TAG = 0>
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
-                                             uint32_t code) {
+                                             uint32_t code, uint64_t limit_ns) {
   if constexpr (OUT_OF_LINE) {
     if (mbar_try_wait(bar, parity)) return true;
-    return wait_or_abort_slow<TAG>(bar, parity, abort, err, code);
+    return wait_or_abort_slow<TAG>(bar, parity, abort, err, code, limit_ns);
   } else {
-    return wait_or_abort(bar, parity, abort, err, code);
+    return wait_or_abort(bar, parity, abort, err, code, limit_ns);
   }
 }
 

@@ -287,10 +287,17 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       int u4 = 0, u16 = 0;
       for (int it = 0; it < np && !ms.abort; ++it) {
         const int kt = tile_of(it);
+        // failure-detection test: this tile's slots are taken but its copies
+        // are never issued, so the waits of their consumers run out
+        const bool hold = it == p.withhold;
         if (!fp16_of(it) && !eight_of(it)) {
           const int slot = u4 % L::kNS, use = u4 / L::kNS;
-          if (use > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (use > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns))
             break;
+          if (hold) {
+            ++u4;
+            continue;
+          }
           uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
           mbar_arrive_expect_tx(&ms.bar_full4[slot], L::kTx4);
           tma_load_3d(st, &mK4, &ms.bar_full4[slot], 0, kt * 128, bhk);
@@ -305,9 +312,13 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           bool stop = false;
           for (int part = 0; part < 2; ++part) {
             const int slot = u4 % L::kNS, use = u4 / L::kNS;
-            if (use > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
+            if (use > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)) {
               stop = true;
               break;
+            }
+            if (hold) {
+              ++u4;
+              continue;
             }
             uint8_t* st = sm + L::kSlot4 + slot * L::kSlot4Bytes;
             const size_t sc = (static_cast<size_t>(bhk) * p.NT + kt) * 512;
@@ -324,13 +335,17 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           if (stop) break;
         } else {
           uint8_t* st = sm + L::kSlot16;
-          if (u16 > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
+          if (u16 > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty_k16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns))
             break;
+          if (hold) {
+            ++u16;
+            continue;
+          }
           mbar_arrive_expect_tx(&ms.bar_full_k16, L::kTx16);
           for (int pnl = 0; pnl < D / 64; ++pnl)
             tma_load_3d(st + pnl * 16384, &mK16, &ms.bar_full_k16, pnl * 64, kt * 128, bhk);
-          if (u16 > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) {
-            mbar_wait(&ms.bar_full_k16, u16 & 1, kWaitNs);  // the K16 copy of this tile is in flight
+          if (u16 > 0 && !bounded_wait<kOolRoles, 1>(&ms.bar_empty_v16, (u16 - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)) {
+            mbar_wait(&ms.bar_full_k16, u16 & 1, p.wait_ns);  // the K16 copy of this tile is in flight
             break;
           }
           mbar_arrive_expect_tx(&ms.bar_full_v16, L::kTx16);
@@ -340,12 +355,12 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
       }
       // Let every copy this thread issued land before the CTA can exit.
-      mbar_wait(&ms.bar_q, 0, kWaitNs);
+      mbar_wait(&ms.bar_q, 0, p.wait_ns);
       for (int s = 0; s < L::kNS; ++s)
-        if (u4 > s) mbar_wait(&ms.bar_full4[s], ((u4 - 1 - s) / L::kNS) & 1, kWaitNs);
+        if (u4 > s) mbar_wait(&ms.bar_full4[s], ((u4 - 1 - s) / L::kNS) & 1, p.wait_ns);
       if (u16 > 0) {
-        mbar_wait(&ms.bar_full_k16, (u16 - 1) & 1, kWaitNs);
-        mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, kWaitNs);
+        mbar_wait(&ms.bar_full_k16, (u16 - 1) & 1, p.wait_ns);
+        mbar_wait(&ms.bar_full_v16, (u16 - 1) & 1, p.wait_ns);
       }
     }
     __syncwarp();
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     if (lane == 0) {
       constexpr uint32_t sbo4 = (D == 128) ? 512u : 256u;
       constexpr uint32_t sw4 = (D == 128) ? LAYOUT_SW64 : LAYOUT_SW32;
-      bool ok = bounded_wait<kOolRoles, 1>(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD);
+      bool ok = bounded_wait<kOolRoles, 1>(&ms.bar_q, 0, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns);
       tc_fence_after();
       if (ok) {
         for (int c = 0; c < D / 64; ++c)
@@ -368,14 +383,14 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         if (EIGHT && eight) {
           // K8 in ring slot u4 (V8, in u4 + 1, is the P V issuer's)
           slot = u4 % L::kNS;
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           u4 += 2;
         } else if (!fp16) {
           slot = u4 % L::kNS;
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], (u4 / L::kNS) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           ++u4;
         } else {
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full_k16, uk16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           ++uk16;
         }
         // The K scales go to tensor memory before the wait for the S buffer,
@@ -397,7 +412,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         // loaded its S.  (Barriers and phases count processed tiles, it.)
         if (it >= 1) {
           const int pv = it - 1;
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_s_free[pv & 1], (pv >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)))
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_s_free[pv & 1], (pv >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns)))
             break;
           tc_fence_after();
         }
@@ -442,7 +457,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       }
       // drain: every tensor-core operation this thread issued completes before exit
       mma_commit(&ms.bar_drain[0]);
-      mbar_wait(&ms.bar_drain[0], 0, kWaitNs);
+      mbar_wait(&ms.bar_drain[0], 0, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == kDBMmaPV) {
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           slot = (u4 + 1) % L::kNS;
           const int use = (u4 + 1) / L::kNS;
           u4 += 2;
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           tc_fence_after();
           v4 = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
           tmem_cp_32x128b_x4(tm + kDColSFV8, make_sdesc(v4 + L::kV8Bytes, 16, 128, LAYOUT_NONE));
@@ -475,7 +490,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           // V4 landed with K4 in one barrier phase; wait on it here too so that
           // this thread observes the copy itself.  The producer cannot refill the
           // slot before this thread releases it.
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full4[slot], use & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           tc_fence_after();
           const uint32_t st = sbase + L::kSlot4 + slot * L::kSlot4Bytes;
           v4 = st + L::kK4Bytes;
@@ -483,10 +498,10 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           for (int c = 0; c < 2; ++c)
             tmem_cp_32x128b_x4(tm + kDColSFV + 4 * c, make_sdesc(vsf + 512 * c, 16, 128, LAYOUT_NONE));
         } else {
-          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))) break;
+          if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_full_v16, uv16 & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, p.wait_ns))) break;
           ++uv16;
         }
-        if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_p_full[g], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))) break;
+        if (!(ok = bounded_wait<kOolRoles, 1>(&ms.bar_p_full[g], (it >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, p.wait_ns))) break;
         const bool pt = fp16 || (EIGHT && eight);
         if (pt) ms.pt_issued = ++upt;  // the next user of the P region may wait on its barrier now
         tc_fence_after();
@@ -532,7 +547,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
         }
       }
       mma_commit(&ms.bar_drain[1]);
-      mbar_wait(&ms.bar_drain[1], 0, kWaitNs);
+      mbar_wait(&ms.bar_drain[1], 0, p.wait_ns);
     }
     __syncwarp();
   }
@@ -564,12 +579,12 @@ __global__ void __launch_bounds__(kDBThreads, 1)
       // All of the tile's waits come first, so that everything from the S
       // load to the P stores is one stretch of code the compiler can
       // interleave.  S of this tile:
-      failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_s_full[grp], j & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_s_full[grp], j & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
       // this group's P buffers (the shared-memory P4 codes and the tensor-
       // memory P4 scales) and its O are free once its previous tile's P V
       // product is done;
       if (!failed && j > 0)
-        failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (j - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+        failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (j - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
       // the tensor-memory P region is taken in processing order: the P V
       // product of its previous user must have been issued (a counter, so no
       // barrier phase can be mistaken for another) and be complete.
@@ -581,7 +596,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
               failed = true;
               break;
             }
-            if (globaltimer_ns() - t0 > kWaitNs) {
+            if (globaltimer_ns() - t0 > p.wait_ns) {
               record_error(p.err, DEV_TIMEOUT_OTHER);
               ms.abort = 1;
               failed = true;
@@ -590,7 +605,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
           }
         }
         if (!failed)
-          failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_pt_free, (pt_before - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+          failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_pt_free, (pt_before - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
       }
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       if (failed) continue;
@@ -746,7 +761,7 @@ __global__ void __launch_bounds__(kDBThreads, 1)
     const int n0 = (np + 1) / 2, n1 = np / 2;  // tiles of each group
     const int nmine = grp ? n1 : n0;
     if (!failed && nmine > 0)
-      failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (nmine - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      failed = !bounded_wait<kOolSoftmax, 2>(&ms.bar_o_done[grp], (nmine - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, p.wait_ns);
     ms.mrow[grp][r] = M;
     ms.lrow[grp][r] = l;
     // every softmax thread takes the same exit decision (and sees both groups' M and l)

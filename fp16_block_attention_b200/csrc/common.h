@@ -31,6 +31,16 @@ __host__ __device__ inline size_t v_scale_index(size_t bh, int d, int n, int NT)
 // Device error word of the current device (allocated statically in the library).
 uint32_t* device_error_word();
 
+// Bound of every wait inside the attention kernels launched from now on, in
+// nanoseconds (thrift_set_wait_limit; kWaitNs by default).
+uint64_t wait_limit_ns();
+
+// Failure-detection tests only: the processed key tile whose copies the
+// attention kernels' producer does not issue, from the environment variable
+// THRIFT_TEST_WITHHOLD_TILE read at each launch; -1 (the default) withholds
+// nothing.
+int test_withhold_tile();
+
 // ---- launchers (return cudaError_t of the launch) --------------------------
 cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* codes, void* scales,
                                cudaStream_t st);

@@ -315,6 +315,18 @@ THRIFT_API thrift_status thrift_decode_step(const void* q, const void* K, const 
  * keeps the first error recorded. */
 THRIFT_API thrift_status thrift_last_device_error(void* stream);
 
+/* Bound, in nanoseconds, of every wait inside the prefill attention kernels
+ * (thrift_attention, thrift_attention_tiered and the fused entries) launched
+ * after this call, process-wide; 2 s by default.  A kernel whose wait runs
+ * out records THRIFT_ERR_TIMEOUT in the device error word
+ * (thrift_last_device_error), raises an abort flag that makes every role of
+ * its CTA leave its loop, drains its copies and tensor-core work, and
+ * returns; the output of that launch is not written.  A shorter bound makes
+ * failure detection faster; it must stay well above a kernel's longest
+ * legitimate wait (microseconds on the supported shapes).  Returns
+ * THRIFT_ERR_INVALID_ARG outside [1 us, 60 s]. */
+THRIFT_API thrift_status thrift_set_wait_limit(uint64_t ns);
+
 /* Static, human-readable name of a status. */
 THRIFT_API const char* thrift_strerror(thrift_status status);
 
