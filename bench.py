@@ -747,6 +747,65 @@ def run_decode_sweep(args, dev, peaks):
     torch.cuda.empty_cache()
 
 
+def run_blk_sweep(args, dev, peaks, n_sm):
+    """Selection blocks of 128 x 128 against 64 x 64 on the D = 128 GQA
+    workloads at their rho: per block size, the time of quantise + select +
+    attention (the fused step) and of the attention kernel alone, effective
+    TFLOP/s and the blended roofline and MUFU fractions.  The gap-recovered
+    proxy at both block sizes is measured against the oracle in
+    tests/test_gpu_block_size.py."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    p16 = peaks["bf16_tflops"] * 1e12
+    p4 = FP4_OVER_BF16 * p16
+    stream = torch.cuda.current_stream(dev)
+    print("| workload | rho | blk | step ms (quantise + select + attention) | attention ms | "
+          "effective TFLOP/s (attention) | roofline frac | MUFU frac |")
+    print("|---|---:|---:|---:|---:|---:|---:|---:|")
+    for w0 in (synth.GQA_N32K, synth.BATCHED_GQA_N16K, synth.GQA_N128K):
+        Q, K, V = synth.generate(w0)
+        Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+        del Q, K, V
+        for blk in (128, 64):
+            w = w0.with_(blk=blk)
+            sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+            Od = torch.empty_like(Qd)
+            ws = torch.empty(thrift.fused_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+            qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+            mask = thrift.select_blocks(Qd, Kd, sh, w.rho)
+
+            def timed(fn, n):
+                for _ in range(args.warmup):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(n):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) / n
+
+            n = 3 if w.N > 65536 else 10
+            step_ms = timed(lambda: thrift.attention_fused(Qd, Kd, Vd, sh, w.rho, Od, ws, stream), n)
+            attn_ms = timed(lambda: thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od, stream), n)
+            if thrift.last_device_error(stream) != 0:
+                raise RuntimeError(f"a kernel reported a bounded-wait timeout on {w.name} (blk {blk})")
+            m = mask.cpu().numpy()
+            f16, f4 = flop_split(w, m)
+            t_bound = max(f16 / p16 + f4 / p4, attention_bytes(w, m) / (peaks["hbm_gbs"] * 1e9))
+            mufu = mufu_ceiling(w, m, attn_ms, 1965.0, n_sm)
+            print(f"| {w.name} | {w.rho:g} | {blk} | {step_ms:.4f} | {attn_ms:.4f} | "
+                  f"{w.flops() / (attn_ms * 1e-3) / 1e12:.1f} | {t_bound * 1e3 / attn_ms:.4f} | {mufu['frac']:.4f} |",
+                  flush=True)
+            del Od, ws, qz, mask
+            torch.cuda.empty_cache()
+        del Qd, Kd, Vd
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -762,11 +821,18 @@ def main(argv=None):
                     help="time the decode step on the GQA and batched caches (markdown table), then exit")
     ap.add_argument("--tier-sweep", action="store_true",
                     help="time attention with skipped and with 8-bit pairs (markdown tables), then exit")
+    ap.add_argument("--blk-sweep", action="store_true",
+                    help="time the GQA workloads with 128- and 64-key selection blocks (markdown table), then exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.sweep:
         run_sweep(args)
+    elif args.blk_sweep:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_blk_sweep(args, dev, load_peaks()[0], torch.cuda.get_device_properties(dev).multi_processor_count)
     elif args.decode_sweep or args.tier_sweep:
         import torch
         dev = torch.device("cuda", 0)
