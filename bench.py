@@ -806,6 +806,43 @@ def run_blk_sweep(args, dev, peaks, n_sm):
         torch.cuda.empty_cache()
 
 
+def run_ncu_case(args, dev):
+    """Small, fixed launch sequences on the 32k GQA workload for ncu captures
+    (the commands in profiles/ run these):
+      attention: quantise and select once at --rho, then the attention
+                 kernel 3 times (warm-up) and once more (the captured launch:
+                 -k regex:thrift_attention -s 3 -c 1);
+      stages:    the quantisers of Q, K, V and the selection at --rho, twice
+                 in the same order (capture the second round)."""
+    import torch
+
+    import fp16_block_attention_b200 as thrift
+
+    w = synth.GQA_N32K
+    rho = w.rho if args.rho is None else args.rho
+    Q, K, V = synth.generate(w)
+    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+    sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
+    qz = thrift.quantize_all(Qd, Kd, Vd, sh)
+    mask = thrift.select_blocks(Qd, Kd, sh, rho)
+    torch.cuda.synchronize()
+    if args.ncu_case == "attention":
+        Od = torch.empty_like(Qd)
+        for _ in range(4):
+            thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od)
+    else:
+        ws = torch.empty(thrift.select_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs)
+            thrift.quantize_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks)
+            thrift.quantize_nvfp4(Vd, thrift.V, sh, qz.v4, qz.vs)
+            thrift.select_blocks(Qd, Kd, sh, rho, mask, ws)
+    torch.cuda.synchronize()
+    if thrift.last_device_error() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout")
+    print(f"ncu case {args.ncu_case} on {w.name}, rho {rho:g}: done")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -821,6 +858,9 @@ def main(argv=None):
                     help="time the decode step on the GQA and batched caches (markdown table), then exit")
     ap.add_argument("--tier-sweep", action="store_true",
                     help="time attention with skipped and with 8-bit pairs (markdown tables), then exit")
+    ap.add_argument("--ncu-case", choices=["attention", "stages"],
+                    help="run a short fixed launch sequence on the 32k GQA workload for an ncu capture, then exit")
+    ap.add_argument("--rho", type=float, default=None, help="FP16 budget of --ncu-case (default: the workload's)")
     ap.add_argument("--blk-sweep", action="store_true",
                     help="time the GQA workloads with 128- and 64-key selection blocks (markdown table), then exit")
     args = ap.parse_args(argv)
@@ -828,6 +868,11 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.sweep:
         run_sweep(args)
+    elif args.ncu_case:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_ncu_case(args, dev)
     elif args.blk_sweep:
         import torch
         dev = torch.device("cuda", 0)
