@@ -71,6 +71,8 @@ def _load():
     sig = {
         "thrift_quant_bytes": ([psh, st, ctypes.POINTER(sz), ctypes.POINTER(sz)], st),
         "thrift_quantize_nvfp4": ([vp, st, psh, vp, vp, vp], st),
+        "thrift_quantize_pool_nvfp4": ([vp, st, psh, vp, vp, vp, vp], st),
+        "thrift_select_blocks_pooled": ([vp, vp, psh, ctypes.c_double, vp, vp, sz, vp], st),
         "thrift_quant8_bytes": ([psh, st, ctypes.POINTER(sz), ctypes.POINTER(sz)], st),
         "thrift_quantize_mxfp8": ([vp, st, psh, vp, vp, vp], st),
         "thrift_select_workspace_bytes": ([psh, ctypes.POINTER(sz)], st),
@@ -105,7 +107,8 @@ def _load():
 _lib = _load()
 
 # C-ABI symbols the header declares (checked by the tests).
-EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quant8_bytes", "thrift_quantize_mxfp8",
+EXPORTS = ("thrift_quant_bytes", "thrift_quantize_nvfp4", "thrift_quantize_pool_nvfp4", "thrift_quant8_bytes",
+           "thrift_quantize_mxfp8", "thrift_select_blocks_pooled",
            "thrift_select_workspace_bytes", "thrift_select_blocks",
            "thrift_select_blocks_static", "thrift_select_blocks_vertical_window", "thrift_select_blocks_tiered",
            "thrift_attention", "thrift_attention_tiered",
@@ -213,6 +216,29 @@ def quantize_nvfp4(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=No
     return codes, scales
 
 
+def quantize_pool_nvfp4(x: torch.Tensor, op: int, shape: Shape, codes=None, scales=None, means=None, stream=None):
+    """NVFP4 copy of Q or K (as quantize_nvfp4) and its FP32 block means
+    [B, H, nb, D] in one pass: (codes, scales, means)."""
+    if op not in (Q, K):
+        raise ValueError("quantize_pool_nvfp4 takes Q or K")
+    nq, nk, _ = _counts(shape)
+    nc, ns = quant_bytes(shape, op)
+    H = shape.Hq if op == Q else shape.Hkv
+    nm = shape.B * H * shape.nb * shape.D
+    dev = _guard((x, "x", torch.float16, nq if op == Q else nk, "n"), (codes, "codes", None, nc, "b"),
+                 (scales, "scales", None, ns, "b"), (means, "means", torch.float32, nm, "n"))
+    if codes is None:
+        codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(ns, dtype=torch.uint8, device=dev)
+    if means is None:
+        means = torch.empty((shape.B, H, shape.nb, shape.D), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_quantize_pool_nvfp4", _lib.thrift_quantize_pool_nvfp4(
+            _ptr(x), op, ctypes.byref(shape.c()), _ptr(codes), _ptr(scales), _ptr(means), _stream(stream, dev)))
+    return codes, scales, means
+
+
 def quant8_bytes(shape: Shape, op: int):
     c, s = ctypes.c_size_t(), ctypes.c_size_t()
     _check("thrift_quant8_bytes", _lib.thrift_quant8_bytes(ctypes.byref(shape.c()), op, ctypes.byref(c),
@@ -300,6 +326,25 @@ def select_blocks_vertical_window(Qt: torch.Tensor, Kt: torch.Tensor, shape: Sha
     with torch.cuda.device(dev):
         _check("thrift_select_blocks_vertical_window", _lib.thrift_select_blocks_vertical_window(
             _ptr(Qt), _ptr(Kt), ctypes.byref(shape.c()), float(rho), int(window), _ptr(mask), _ptr(ws), _nbytes(ws),
+            _stream(stream, dev)))
+    return mask
+
+
+def select_blocks_pooled(qm: torch.Tensor, km: torch.Tensor, shape: Shape, rho: float, mask=None, ws=None,
+                         stream=None):
+    """select_blocks from precomputed FP32 block means (quantize_pool_nvfp4)."""
+    _, _, nmask = _counts(shape)
+    need = select_workspace_bytes(shape)
+    dev = _guard((qm, "qm", torch.float32, shape.B * shape.Hq * shape.nb * shape.D, "n"),
+                 (km, "km", torch.float32, shape.B * shape.Hkv * shape.nb * shape.D, "n"),
+                 (mask, "mask", torch.uint8, nmask, "n"), (ws, "ws", None, need, "b"))
+    if mask is None:
+        mask = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), dtype=torch.uint8, device=dev)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("thrift_select_blocks_pooled", _lib.thrift_select_blocks_pooled(
+            _ptr(qm), _ptr(km), ctypes.byref(shape.c()), float(rho), _ptr(mask), _ptr(ws), _nbytes(ws),
             _stream(stream, dev)))
     return mask
 

@@ -160,6 +160,20 @@ thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thri
   return from_cuda(launch_quantize_qk(x, BH * s.N, s.N, s.D, codes, scales, cs));
 }
 
+thrift_status thrift_quantize_pool_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
+                                         void* scales, float* means, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (op != THRIFT_Q && op != THRIFT_K) return THRIFT_ERR_INVALID_ARG;
+  if (!x || !codes || !scales || !means) return THRIFT_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(means) & 3u))
+    return THRIFT_ERR_INVALID_ARG;
+  const thrift_shape& s = *shape;
+  const size_t BH = static_cast<size_t>(s.B) * ((op == THRIFT_Q) ? s.Hq : s.Hkv);
+  return from_cuda(
+      launch_quantize_pool_qk(x, BH, s.N, s.D, s.blk, codes, scales, means, static_cast<cudaStream_t>(stream)));
+}
+
 thrift_status thrift_quant8_bytes(const thrift_shape* shape, thrift_operand op, size_t* codes_bytes,
                                   size_t* scales_bytes) {
   thrift_status st = check_shape(shape);
@@ -197,6 +211,16 @@ thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_sh
   if (!aligned16(Q) || !aligned16(K)) return THRIFT_ERR_INVALID_ARG;
   if (!ws || ws_bytes < select_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
   return from_cuda(launch_select(Q, K, *shape, rho, mask, ws, static_cast<cudaStream_t>(stream)));
+}
+
+thrift_status thrift_select_blocks_pooled(const float* qm, const float* km, const thrift_shape* shape, double rho,
+                                          uint8_t* mask, void* ws, size_t ws_bytes, void* stream) {
+  thrift_status st = check_shape(shape);
+  if (st != THRIFT_OK) return st;
+  if (!qm || !km || !mask || !(rho >= 0.0 && rho <= 1.0)) return THRIFT_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(qm) & 3u) || (reinterpret_cast<uintptr_t>(km) & 3u)) return THRIFT_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < select_workspace_bytes(*shape) || !aligned16(ws)) return THRIFT_ERR_WORKSPACE;
+  return from_cuda(launch_select_pooled(qm, km, *shape, rho, mask, ws, static_cast<cudaStream_t>(stream)));
 }
 
 thrift_status thrift_select_blocks_tiered(const void* Q, const void* K, const thrift_shape* shape, double rho,
@@ -296,13 +320,17 @@ thrift_status thrift_attention_fused(const void* Q, const void* K, const void* V
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint32_t* err = device_error_word();
   if (!err) return THRIFT_ERR_CUDA;
-  if (launch_quantize_qk(Q, static_cast<size_t>(s.B) * s.Hq * s.N, s.N, s.D, w.q4, w.qs, cs) != cudaSuccess)
+  // Q and K are read once: quantised and pooled in one pass (the block means
+  // go straight into the selection workspace)
+  float *qm = nullptr, *km = nullptr;
+  select_means(w.sel, s, &qm, &km);
+  if (launch_quantize_pool_qk(Q, static_cast<size_t>(s.B) * s.Hq, s.N, s.D, s.blk, w.q4, w.qs, qm, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
-  if (launch_quantize_qk(K, static_cast<size_t>(s.B) * s.Hkv * s.N, s.N, s.D, w.k4, w.ks, cs) != cudaSuccess)
+  if (launch_quantize_pool_qk(K, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, s.blk, w.k4, w.ks, km, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
-  if (launch_select(Q, K, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (launch_select_pooled(nullptr, nullptr, s, rho, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
   return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, false, nullptr, err, cs));
 }
 
@@ -332,9 +360,11 @@ thrift_status thrift_attention_fused_tiered(const void* Q, const void* K, const 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint32_t* err = device_error_word();
   if (!err) return THRIFT_ERR_CUDA;
-  if (launch_quantize_qk(Q, static_cast<size_t>(s.B) * s.Hq * s.N, s.N, s.D, w.q4, w.qs, cs) != cudaSuccess)
+  float *qm = nullptr, *km = nullptr;  // Q and K quantised and pooled in one pass
+  select_means(w.sel, s, &qm, &km);
+  if (launch_quantize_pool_qk(Q, static_cast<size_t>(s.B) * s.Hq, s.N, s.D, s.blk, w.q4, w.qs, qm, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
-  if (launch_quantize_qk(K, static_cast<size_t>(s.B) * s.Hkv * s.N, s.N, s.D, w.k4, w.ks, cs) != cudaSuccess)
+  if (launch_quantize_pool_qk(K, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, s.blk, w.k4, w.ks, km, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
   if (launch_quantize_v(V, static_cast<size_t>(s.B) * s.Hkv, s.N, s.D, w.v4, w.vs, cs) != cudaSuccess)
     return THRIFT_ERR_CUDA;
@@ -344,7 +374,7 @@ thrift_status thrift_attention_fused_tiered(const void* Q, const void* K, const 
     if (launch_quantize_mx8(K, THRIFT_K, s, w.k8, w.ks8, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
     if (launch_quantize_mx8(V, THRIFT_V, s, w.v8, w.vs8, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
   }
-  if (launch_select_tiered(Q, K, s, rho, rho8, sigma, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
+  if (launch_select_tiered_pooled(s, rho, rho8, sigma, w.mask, w.sel, cs) != cudaSuccess) return THRIFT_ERR_CUDA;
   return from_cuda(launch_attention(Q, K, V, w.mask, w.q4, w.qs, w.k4, w.ks, w.v4, w.vs, s, O, true,
                                     eight ? &copies : nullptr, err, cs));
 }

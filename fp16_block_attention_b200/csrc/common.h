@@ -45,6 +45,11 @@ int test_withhold_tile();
 cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* codes, void* scales,
                                cudaStream_t st);
 cudaError_t launch_quantize_v(const void* v, size_t bh, int N, int D, void* codes, void* scales, cudaStream_t st);
+// Q or K quantised along D and pooled in one pass: the NVFP4 copy as
+// launch_quantize_qk writes it, and the FP32 block means [bh][N/blk][D] of
+// the selection (quantize.cu).
+cudaError_t launch_quantize_pool_qk(const void* x, size_t bh_count, int N, int D, int blk, void* codes, void* scales,
+                                    float* means, cudaStream_t st);
 
 // MXFP8 copies (quantize8.cu).
 size_t mx8_codes_bytes(const thrift_shape& s, thrift_operand op);
@@ -59,6 +64,14 @@ cudaError_t launch_select_static(const void* Q, const void* K, const thrift_shap
                                  cudaStream_t st);
 cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
                           cudaStream_t st);
+// The block means in a selection workspace (launch_quantize_pool_qk writes
+// them), and the selection from those means (no pooling pass).
+void select_means(void* ws, const thrift_shape& s, float** qm, float** km);
+// qm / km: the block means, or null for those already in the workspace.
+cudaError_t launch_select_pooled(const float* qm, const float* km, const thrift_shape& s, double rho, uint8_t* mask,
+                                 void* ws, cudaStream_t st);
+cudaError_t launch_select_tiered_pooled(const thrift_shape& s, double rho, double rho8, double sigma, uint8_t* mask,
+                                        void* ws, cudaStream_t st);
 // Tiered selection (select.cu): mask 1 FP16, 3 MXFP8, 0 NVFP4, 2 skipped.
 cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
                                  double sigma, uint8_t* mask, void* ws, cudaStream_t st);

@@ -131,7 +131,105 @@ __global__ void __launch_bounds__(kVThreads) quantize_v_kernel(const __half* __r
   }
 }
 
+// Q or K encoded along D and pooled in one pass (the fused entry points):
+// one CTA per (selection block of blk rows, bh), 256 threads.  Thread t takes
+// group g = t % (D/16) of rows t / (D/16), + 256 / (D/16), ... with all its
+// 16-byte loads in flight, encodes each group exactly as quantize_qk_kernel
+// does, and adds the group's values to 16 FP64 column sums.  The row slots'
+// sums meet by shuffles within a warp and through shared memory across
+// warps; the block mean is the sum / blk rounded once to FP32, as pool_kernel
+// computes it.  FP64 sums of up to 8192 fp16 values are exact in any order
+// (every partial sum is a multiple of 2^-24 below 2^29), so the means equal
+// pool_kernel's bit for bit and the tensor is read from HBM once.
+template <int D>
+__global__ void __launch_bounds__(256) quantize_pool_qk_kernel(const __half* __restrict__ x, int N, int blk,
+                                                               uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ scales,
+                                                               float* __restrict__ means) {
+  constexpr int G = D / 16;          // groups per row
+  constexpr int kSlots = 256 / G;    // row slots
+  constexpr int kMaxRows = 128 / kSlots;  // rows per thread for blk = 128 (4 for D = 128, 2 for D = 64)
+  __shared__ double part[8][D];      // per warp, per channel
+  const size_t bh = blockIdx.y;
+  const int i = blockIdx.x, nb = N / blk;
+  const int NT = num_tiles(N);
+  const int g = threadIdx.x % G, slot = threadIdx.x / G;
+  const int rows = blk / kSlots;     // rows of this thread (blk / kSlots <= kMaxRows)
+  const size_t row0 = bh * N + static_cast<size_t>(i) * blk;
+  uint4 a[kMaxRows], b[kMaxRows];
+#pragma unroll
+  for (int q = 0; q < kMaxRows; ++q) {
+    if (q < rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (row0 + slot + q * kSlots) * D + g * 16);
+      a[q] = __ldg(src);
+      b[q] = __ldg(src + 1);
+    }
+  }
+  double acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.0;
+#pragma unroll
+  for (int q = 0; q < kMaxRows; ++q) {
+    if (q < rows) {
+      float v[16];
+      const __half2* ha = reinterpret_cast<const __half2*>(&a[q]);
+      const __half2* hb = reinterpret_cast<const __half2*>(&b[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __half22float2(ha[e]), fb = __half22float2(hb[e]);
+        v[2 * e] = fa.x;
+        v[2 * e + 1] = fa.y;
+        v[8 + 2 * e] = fb.x;
+        v[8 + 2 * e + 1] = fb.y;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] += static_cast<double>(v[e]);
+      const Group16 enc = encode16(v);
+      const size_t row = row0 + slot + q * kSlots;
+      *reinterpret_cast<uint2*>(codes + row * (D / 2) + g * 8) = make_uint2(enc.lo, enc.hi);
+      const int n = i * blk + slot + q * kSlots;
+      scales[qk_scale_index(bh, n, g, NT, D)] = static_cast<uint8_t>(enc.scale);
+    }
+  }
+  // lanes with the same group: lane ^ G, lane ^ 2G, ... within the warp
+#pragma unroll
+  for (int off = G; off < 32; off *= 2)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (lane < G)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) part[warp][16 * lane + e] = acc[e];
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += 256) {
+    double sum = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += part[w][d];
+    means[(bh * nb + i) * D + d] = static_cast<float>(sum / blk);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_pool_qk(const void* x, size_t bh_count, int N, int D, int blk, void* codes, void* scales,
+                                    float* means, cudaStream_t st) {
+  const dim3 grid(N / blk, static_cast<unsigned>(bh_count));
+  if (D == 128)
+    quantize_pool_qk_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), N, blk,
+                                                       static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                                                       means);
+  else
+    quantize_pool_qk_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), N, blk,
+                                                      static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                                                      means);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (N % kTile) {
+    zero_qk_scale_padding<<<148, 256, 0, st>>>(bh_count, N, D, static_cast<uint8_t*>(scales));
+    e = cudaGetLastError();
+  }
+  return e;
+}
 
 cudaError_t launch_quantize_qk(const void* x, size_t rows, int N, int D, void* codes, void* scales,
                                cudaStream_t st) {

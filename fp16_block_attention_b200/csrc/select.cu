@@ -32,6 +32,7 @@
 //            causal mask) first, then whole columns in rank order, each by
 //            descending score.
 #include <atomic>
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "common.h"
@@ -113,8 +114,11 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __half* __rest
 __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qm, const float* __restrict__ km,
                                                     int Hq, int Hkv, int nb, int D, int causal, float sm_scale,
                                                     float* __restrict__ scores) {
-  __shared__ float qs[32][129];
-  __shared__ float ks[32][129];
+  // The two 32-row slices of block means, widened to FP64 once (exact) as
+  // they are staged, so the inner loop is loads and FP64 FMAs only.
+  extern __shared__ double score_smem[];
+  double* qs = score_smem;               // [32][D + 1]
+  double* ks = score_smem + 32 * (D + 1);
   const int bi = blockIdx.y * 32, bj = blockIdx.x * 32;
   if (causal && bj > bi + 31) return;
   const size_t bh = blockIdx.z;
@@ -122,14 +126,18 @@ __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qm
   const size_t bhk = b * Hkv + hq / (Hq / Hkv);
   for (int t = threadIdx.x; t < 32 * D; t += blockDim.x) {
     const int r = t / D, d = t % D;
-    qs[r][d] = (bi + r < nb) ? qm[(bh * nb + bi + r) * D + d] : 0.0f;
-    ks[r][d] = (bj + r < nb) ? km[(bhk * nb + bj + r) * D + d] : 0.0f;
+    qs[r * (D + 1) + d] = (bi + r < nb) ? static_cast<double>(qm[(bh * nb + bi + r) * D + d]) : 0.0;
+    ks[r * (D + 1) + d] = (bj + r < nb) ? static_cast<double>(km[(bhk * nb + bj + r) * D + d]) : 0.0;
   }
   __syncthreads();
   const int ti = (threadIdx.x / 16) * 2, tj = (threadIdx.x % 16) * 2;
+  const double* q0p = qs + ti * (D + 1);
+  const double* q1p = q0p + (D + 1);
+  const double* k0p = ks + tj * (D + 1);
+  const double* k1p = k0p + (D + 1);
   double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
   for (int d = 0; d < D; ++d) {
-    const double q0 = qs[ti][d], q1 = qs[ti + 1][d], k0 = ks[tj][d], k1 = ks[tj + 1][d];  // exact widening
+    const double q0 = q0p[d], q1 = q1p[d], k0 = k0p[d], k1 = k1p[d];
     acc[0][0] = fma(q0, k0, acc[0][0]);
     acc[0][1] = fma(q0, k1, acc[0][1]);
     acc[1][0] = fma(q1, k0, acc[1][0]);
@@ -216,17 +224,29 @@ __global__ void __launch_bounds__(1024) column_rank_kernel(const float* __restri
 // (8-bit); with keep < #valid the pairs after the first `keep` are marked 2
 // (skipped; the caller keeps them clear of forced, FP16 and 8-bit pairs), the
 // rest 0.
+// A head's selection runs on a cluster of kTopkCluster CTAs: CTA c of the
+// cluster takes rows c, c + kTopkCluster, ... (balanced under the causal
+// triangle).  Each radix pass, every CTA histograms its rows into its own
+// shared memory; after a cluster barrier, warp 0 of every CTA sums all the
+// cluster's histograms through distributed shared memory and finds the same
+// digit (the sum is the same everywhere, so no CTA has to broadcast it); a
+// second barrier keeps any histogram from being cleared, or its CTA from
+// exiting, while another CTA still reads it.
+constexpr int kTopkCluster = 4;
+
 template <int VW>
-__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int nb, int causal,
-                                                    long long k, long long k8end, long long keep,
-                                                    uint8_t* __restrict__ mask,
-                                                    const int* __restrict__ rank, int window) {
+__global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(1024)
+    topk_kernel(const float* __restrict__ scores, int nb, int causal, long long k, long long k8end, long long keep,
+                uint8_t* __restrict__ mask, const int* __restrict__ rank, int window) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ long long s_remaining;
   __shared__ int s_done;
   __shared__ int s_rank[VW ? kMaxVWBlocks : 1];
-  const size_t bh = blockIdx.x;
+  const size_t bh = blockIdx.x / kTopkCluster;
   if (VW) {
     for (int j = threadIdx.x; j < nb; j += blockDim.x) s_rank[j] = rank[bh * nb + j];
     __syncthreads();
@@ -261,7 +281,7 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
       for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
       __syncthreads();
       const uint64_t prefix = s_prefix;
-      for (int i = warp; i < nb; i += nwarps) {
+      for (int i = crank + kTopkCluster * warp; i < nb; i += kTopkCluster * nwarps) {
         const int ncol = causal ? i + 1 : nb;
         const float* row = sc + static_cast<size_t>(i) * nb;
         for (int j0 = 0; j0 < ncol; j0 += 128) {  // four column chunks, loads first
@@ -286,15 +306,19 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
           }
         }
       }
-      __syncthreads();
+      cluster.sync();  // every CTA's histogram of this pass is complete
       if (warp == 0) {
-        // lane l holds bins 255 - 8 l .. 248 - 8 l, highest first
+        // lane l holds bins 255 - 8 l .. 248 - 8 l, highest first, summed over the cluster
         uint32_t c[8], tot = 0;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          c[t] = hist[255 - 8 * lane - t];
-          tot += c[t];
+        for (int t = 0; t < 8; ++t) c[t] = 0;
+        for (int rk = 0; rk < kTopkCluster; ++rk) {
+          const unsigned int* h = cluster.map_shared_rank(hist, rk);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) c[t] += h[255 - 8 * lane - t];
         }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) tot += c[t];
         uint32_t incl = tot;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -321,7 +345,7 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
           s_done = (cnt == rem - cum);
         }
       }
-      __syncthreads();
+      cluster.sync();  // the digit is known everywhere; no histogram is read any more
       pmask |= 255ull << shift;
       if (s_done) break;
     }
@@ -334,8 +358,11 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
   const uint64_t eight_from = (eight_any && !eight_all) ? kth_largest(k8end) : 0ull;  // 8-bit: key >= eight_from
   const bool skip_any = keep < valid;
   const uint64_t keep_from = (skip_any && keep > 0) ? kth_largest(keep) : 0ull;  // skipped: key < keep_from
-  for (size_t idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int i = static_cast<int>(idx / nb), j = static_cast<int>(idx % nb);
+  // this CTA's rows of the mask
+  const int my_rows = (nb - crank + kTopkCluster - 1) / kTopkCluster;
+  for (size_t t = threadIdx.x; t < static_cast<size_t>(my_rows) * nb; t += blockDim.x) {
+    const int i = crank + kTopkCluster * static_cast<int>(t / nb), j = static_cast<int>(t % nb);
+    const size_t idx = static_cast<size_t>(i) * nb + j;
     uint8_t v = 0;
     if (!(causal && j > i)) {
       const uint64_t key = key_of(sc[idx], i, j);
@@ -372,13 +399,19 @@ long long budget_pairs(const thrift_shape& s, double rho) {
   return static_cast<long long>(kk);
 }
 
-void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s, const SelectWs& w, cudaStream_t st) {
+// pooled: the block means are already in the workspace (launch_quantize_pool_qk)
+void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s, const SelectWs& w, cudaStream_t st,
+                            bool pooled = false) {
   const int nb = s.N / s.blk;
-  pool_kernel<<<dim3(nb, s.B * s.Hq), kPoolThreads, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
-  pool_kernel<<<dim3(nb, s.B * s.Hkv), kPoolThreads, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
+  if (!pooled) {
+    pool_kernel<<<dim3(nb, s.B * s.Hq), kPoolThreads, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
+    pool_kernel<<<dim3(nb, s.B * s.Hkv), kPoolThreads, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
+  }
   const int tiles = (nb + 31) / 32;
-  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
-                                                               s.sm_scale, w.scores);
+  const int smem = 2 * 32 * (s.D + 1) * static_cast<int>(sizeof(double));
+  cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, smem, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
+                                                                  s.sm_scale, w.scores);
 }
 }  // namespace
 
@@ -395,25 +428,30 @@ cudaError_t launch_select_vertical_window(const void* Q, const void* K, const th
   launch_pool_and_scores(Q, K, s, w, st);
   column_rank_kernel<<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, w.rank);
   const long long k = budget_pairs(s, rho);
-  topk_kernel<1><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, w.rank, window);
+  topk_kernel<1><<<s.B * s.Hq * kTopkCluster, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, w.rank, window);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
-                          cudaStream_t st) {
+namespace {
+// pooled: the block means are given (qm / km, or those already in the
+// workspace when null) and no pooling pass runs
+cudaError_t select_impl(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
+                        cudaStream_t st, bool pooled, const float* qm = nullptr, const float* km = nullptr) {
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
-  launch_pool_and_scores(Q, K, s, w, st);
+  if (qm) w.qm = const_cast<float*>(qm);
+  if (km) w.km = const_cast<float*>(km);
+  launch_pool_and_scores(Q, K, s, w, st, pooled);
   const long long k = budget_pairs(s, rho);
-  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, nullptr, 0);
+  topk_kernel<0><<<s.B * s.Hq * kTopkCluster, 1024, 0, st>>>(w.scores, nb, s.causal, k, k, valid_pairs(s), mask, nullptr, 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
-                                 double sigma, uint8_t* mask, void* ws, cudaStream_t st) {
+cudaError_t select_tiered_impl(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
+                               double sigma, uint8_t* mask, void* ws, cudaStream_t st, bool pooled) {
   const int nb = s.N / s.blk;
   SelectWs w = carve(ws, s);
-  launch_pool_and_scores(Q, K, s, w, st);
+  launch_pool_and_scores(Q, K, s, w, st, pooled);
   // 8-bit pairs: the k8 after the FP16 ones; skipped pairs: the last ks of the
   // ranking, clear of the forced, FP16 and 8-bit pairs
   const long long n = valid_pairs(s), k16 = budget_pairs(s, rho);
@@ -424,8 +462,35 @@ cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shap
   const long long cap = n - (k16 + k8 > forced ? k16 + k8 : forced);
   if (ks > cap) ks = cap;
   if (ks < 0) ks = 0;
-  topk_kernel<0><<<s.B * s.Hq, 1024, 0, st>>>(w.scores, nb, s.causal, k16, k16 + k8, n - ks, mask, nullptr, 0);
+  topk_kernel<0><<<s.B * s.Hq * kTopkCluster, 1024, 0, st>>>(w.scores, nb, s.causal, k16, k16 + k8, n - ks, mask, nullptr, 0);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_select(const void* Q, const void* K, const thrift_shape& s, double rho, uint8_t* mask, void* ws,
+                          cudaStream_t st) {
+  return select_impl(Q, K, s, rho, mask, ws, st, false);
+}
+
+cudaError_t launch_select_pooled(const float* qm, const float* km, const thrift_shape& s, double rho, uint8_t* mask,
+                                 void* ws, cudaStream_t st) {
+  return select_impl(nullptr, nullptr, s, rho, mask, ws, st, true, qm, km);
+}
+
+void select_means(void* ws, const thrift_shape& s, float** qm, float** km) {
+  const SelectWs w = carve(ws, s);
+  *qm = w.qm;
+  *km = w.km;
+}
+
+cudaError_t launch_select_tiered(const void* Q, const void* K, const thrift_shape& s, double rho, double rho8,
+                                 double sigma, uint8_t* mask, void* ws, cudaStream_t st) {
+  return select_tiered_impl(Q, K, s, rho, rho8, sigma, mask, ws, st, false);
+}
+
+cudaError_t launch_select_tiered_pooled(const thrift_shape& s, double rho, double rho8, double sigma, uint8_t* mask,
+                                        void* ws, cudaStream_t st) {
+  return select_tiered_impl(nullptr, nullptr, s, rho, rho8, sigma, mask, ws, st, true);
 }
 
 // ---- selection without a caller-supplied workspace ------------------------

@@ -104,6 +104,18 @@ THRIFT_API thrift_status thrift_quant_bytes(const thrift_shape* shape, thrift_op
 THRIFT_API thrift_status thrift_quantize_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape, void* codes,
                                     void* scales, void* stream);
 
+/* Q or K quantised as thrift_quantize_nvfp4 does (identical codes and scales)
+ * and pooled in the same pass, so the fp16 tensor is read from HBM once:
+ * means [B][H][N/blk][D] FP32 receives the block means of the selection
+ * heuristic (ThriftAttention abstract: the cheap heuristic that picks the
+ * block pairs), each the FP64 sum of a block's blk rows divided by blk,
+ * rounded once to FP32, identical to what thrift_select_blocks computes
+ * internally.  op: THRIFT_Q (H = Hq) or THRIFT_K (H = Hkv); means 4-byte
+ * aligned.  Feed the means to thrift_select_blocks_pooled.  Errors as for
+ * thrift_quantize_nvfp4; INVALID_ARG for op V. */
+THRIFT_API thrift_status thrift_quantize_pool_nvfp4(const void* x, thrift_operand op, const thrift_shape* shape,
+                                                    void* codes, void* scales, float* means, void* stream);
+
 /* MXFP8 copies for 8-bit block pairs (mask value 3 of the tiered selection),
  * after TriAttention's 8-bit precision (abstract on the paper page of arXiv
  * 2611.07256): the OCP microscaling format with E4M3 elements and one E8M0
@@ -132,6 +144,14 @@ THRIFT_API thrift_status thrift_select_workspace_bytes(const thrift_shape* shape
  * thrift_select_workspace_bytes() bytes (contents need not be initialised). */
 THRIFT_API thrift_status thrift_select_blocks(const void* Q, const void* K, const thrift_shape* shape, double rho,
                                    uint8_t* mask, void* ws, size_t ws_bytes, void* stream);
+
+/* thrift_select_blocks from precomputed block means (qm [B][Hq][nb][D],
+ * km [B][Hkv][nb][D], FP32, as thrift_quantize_pool_nvfp4 writes them): the
+ * same scores, budget and mask, without a pooling pass.  ws as for
+ * thrift_select_blocks (the block-mean part of it is not used). */
+THRIFT_API thrift_status thrift_select_blocks_pooled(const float* qm, const float* km, const thrift_shape* shape,
+                                                     double rho, uint8_t* mask, void* ws, size_t ws_bytes,
+                                                     void* stream);
 
 /* Stage 1 with two more classes, 8-bit and skipped pairs, after
  * TriAttention's tile precisions (abstract on the paper page of arXiv

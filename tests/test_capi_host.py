@@ -183,3 +183,14 @@ def test_binding_checks_sizes_and_devices_before_calling_the_library():
         thrift._guard((_FakeCuda(nq, contiguous=False), "Q", torch.float16, nq, "n"))
     with pytest.raises(ValueError, match="CUDA"):
         thrift.attention_fused(torch.zeros(nq, dtype=torch.float16), None, None, sh, 0.05)
+
+
+def test_pooled_entry_points_check_their_arguments_before_launch():
+    lib = thrift.lib()
+    sh = ctypes.byref(_c(blk=64))
+    fake = ctypes.c_void_p(256)
+    assert lib.thrift_quantize_pool_nvfp4(fake, 2, sh, fake, fake, fake, None) == 1     # V cannot be pooled
+    assert lib.thrift_quantize_pool_nvfp4(None, 0, sh, fake, fake, fake, None) == 1
+    assert lib.thrift_quantize_pool_nvfp4(fake, 0, sh, fake, fake, ctypes.c_void_p(258), None) == 1  # misaligned means
+    assert lib.thrift_select_blocks_pooled(fake, fake, sh, 1.5, fake, fake, 1 << 30, None) == 1
+    assert lib.thrift_select_blocks_pooled(fake, fake, sh, 0.05, fake, fake, 8, None) == 5
