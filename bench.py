@@ -7,11 +7,14 @@ GQA prefill, B=1, Hq=32, Hkv=8, N=32768, D=128, fp16 inputs, 128x128
 selection blocks.  Inputs (Q alone is 268 MB) are larger than the 126 MB L2,
 so no flush is needed between steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--split heads]
 
 Prints one JSON line on rank 0.  For N > 1 (torchrun) every rank runs its own
-independent problem (weak scaling, no data-path collective); the timed
-region is bracketed by a barrier and the slowest rank's time is reported.
+independent problem (weak scaling, no data-path collective); with
+`--split heads` the ranks share one problem instead, rank r taking kv heads
+[r*Hkv/N, (r+1)*Hkv/N) and their query heads (strong scaling, no data-path
+collective either).  The timed region is bracketed by a barrier and the
+slowest rank's time is reported.
 `--impl reference` times the CPU oracle on a bounded row sample instead.
 """
 from __future__ import annotations
@@ -71,6 +74,36 @@ def rank_workload(w, rank: int, world: int):
 def whole_job_tflops(flops_per_rank: float, ms_per_step: float, world: int) -> float:
     """Whole-job throughput: every rank's work over the slowest rank's time."""
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def rank_heads(w, rank: int, world: int):
+    """kv-head split of one problem: rank `rank` of `world` runs kv heads
+    [rank*Hkv/world, (rank+1)*Hkv/world) and the Hq/Hkv query heads that share
+    each of them.  A query head reads one kv head only and the block selection
+    ranks each query head's pairs on their own, so every rank's output is the
+    slice of the whole problem's output: no data-path collective.  Returns
+    ((hk0, hk1), (hq0, hq1))."""
+    if not 1 <= world <= w.Hkv:
+        raise ValueError(f"a kv-head split needs 1 <= world ({world}) <= Hkv ({w.Hkv})")
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    G = w.Hq // w.Hkv
+    hk0, hk1 = rank * w.Hkv // world, (rank + 1) * w.Hkv // world
+    return (hk0, hk1), (hk0 * G, hk1 * G)
+
+
+def head_workload(w, rank: int, world: int):
+    """The shapes of rank `rank`'s share of a kv-head split (its data are slices
+    of the whole problem's, not a problem of their own)."""
+    (hk0, hk1), (hq0, hq1) = rank_heads(w, rank, world)
+    return w.with_(Hq=hq1 - hq0, Hkv=hk1 - hk0)
+
+
+def job_flops(w, world: int, split: str) -> float:
+    """Effective FLOPs of the whole job per step: `world` independent problems
+    (split "problems", weak scaling) or the one problem whose kv heads the ranks
+    share (split "heads", strong scaling)."""
+    return w.flops() if split == "heads" else world * w.flops()
 
 
 def load_peaks():
@@ -205,10 +238,26 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
-    w = rank_workload(WORKLOAD, rank, world)
-    Q, K, V = synth.generate(w)
+    if args.split == "heads":
+        # one problem; this rank's kv heads and their query heads are views of it
+        # (pointer offsets into the whole tensors; contiguous for B = 1)
+        (hk0, hk1), (hq0, hq1) = rank_heads(WORKLOAD, rank, world)
+        w = head_workload(WORKLOAD, rank, world)
+        Qa, Ka, Va = synth.generate(WORKLOAD)
+        Qf, Kf, Vf = (torch.from_numpy(a).to(dev) for a in (Qa, Ka, Va))
+        Qd, Kd, Vd = (t[:, lo:hi] for t, lo, hi in ((Qf, hq0, hq1), (Kf, hk0, hk1), (Vf, hk0, hk1)))
+        if not all(t.is_contiguous() for t in (Qd, Kd, Vd)):
+            Qd, Kd, Vd = (t.contiguous() for t in (Qd, Kd, Vd))
+        Q, K, V = (np.ascontiguousarray(a[:, lo:hi]) for a, lo, hi in ((Qa, hq0, hq1), (Ka, hk0, hk1),
+                                                                        (Va, hk0, hk1)))
+        del Qa, Ka, Va
+        share = f"kv heads [{hk0}, {hk1}) and query heads [{hq0}, {hq1}) on rank {rank}"
+    else:
+        w = rank_workload(WORKLOAD, rank, world)
+        Q, K, V = synth.generate(w)
+        Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
+        share = "the whole problem on every rank"
     sh = thrift.Shape(w.B, w.Hq, w.Hkv, w.N, w.D, w.blk, w.causal, w.sm_scale)
-    Qd, Kd, Vd = (torch.from_numpy(a).to(dev) for a in (Q, K, V))
     Od = torch.empty_like(Qd)
     ws = torch.empty(thrift.fused_workspace_bytes(sh), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -324,7 +373,7 @@ def run_gpu(args):
     p16 = peaks["bf16_tflops"] * 1e12
     p4 = FP4_OVER_BF16 * p16
     f16, f4 = flop_split(w, mask.cpu().numpy())
-    flops = w.flops()
+    flops = w.flops()                                 # this rank's launch
     t_tensor = f16 / p16 + f4 / p4
     bytes_alg = attention_bytes(w, mask.cpu().numpy())
     t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
@@ -332,15 +381,21 @@ def run_gpu(args):
     blended_peak = flops / t_bound / 1e12
     achieved = flops / (attn_ms * 1e-3) / 1e12
     n = world
-    value = whole_job_tflops(flops, ms_step, n)
+    jflops = job_flops(WORKLOAD if args.split == "heads" else w, n, args.split)
+    value = jflops / (ms_step * 1e-3) / 1e12
     clocks = clk.summary()
+    parallelism = (f"kv-head split x{n}: rank r runs kv heads [r*Hkv/{n}, (r+1)*Hkv/{n}) of one problem with "
+                   "their query heads, by pointer offsets, no data-path collective" if args.split == "heads"
+                   else f"independent problem per GPU x{n}")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": n, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "strong" if args.split == "heads" else "weak",
         "vs_baseline": None, "dtype": "nvfp4+fp16 (fp32 accum)", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "D": w.D, "causal": w.causal,
+        "config": {"workload": WORKLOAD.name, "B": WORKLOAD.B, "Hq": WORKLOAD.Hq, "Hkv": WORKLOAD.Hkv,
+                   "N": w.N, "D": w.D, "causal": w.causal,
                    "rho": w.rho, "blk": w.blk, "l2": "inputs larger than L2 (Q alone 268 MB), no flush",
-                   "parallelism": f"independent problem per GPU x{n}",
+                   "parallelism": parallelism, "rank0_share": share,
                    "step": "quantise-and-pool Q,K + quantise V + select from the pooled means + attention (C ABI; the fused entry point's launches)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(blended_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / blended_peak, 4), "traffic": profiled_traffic(),
@@ -352,7 +407,7 @@ def run_gpu(args):
         "clocks": clocks,
         "mufu_ceiling": mufu_ceiling(w, mask.cpu().numpy(), attn_ms, clocks.get("sm_mhz") or 1965.0,
                                      torch.cuda.get_device_properties(dev).multi_processor_count),
-        "e2e": {"value": round(whole_job_tflops(flops, e2e_ms, n), 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(jflops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
                 "api": "attention_fused (quantise + select + attend) per step",
                 "overlap": "two buffer sets, three streams: step i+1's upload and step i-1's download "
@@ -361,7 +416,7 @@ def run_gpu(args):
                 "d2h_bytes_per_step": int(Oh.numel() * 2)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -857,6 +912,9 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", default="problems", choices=["problems", "heads"],
+                    help="N > 1: an independent problem per rank (weak scaling, the default) or one problem "
+                         "whose kv heads the ranks share (strong scaling)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the attention kernel on every workload and rho (markdown table), then exit")
     ap.add_argument("--decode-sweep", action="store_true",
