@@ -93,6 +93,21 @@ __device__ __forceinline__ bool softmax_bar_or(bool flag) {
 }
 
 
+// The same on named barrier ID (ID != 0, 1 if another use of barrier 1 could interleave).
+template <int ID, int NT>
+__device__ __forceinline__ bool bar_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(flag)), "n"(ID), "n"(NT)
+      : "memory");
+  return r != 0;
+}
+
 // Barrier of all `count` threads of the CTA that warps may reach from
 // different places in the code (barrier 2, not the aligned __syncthreads).
 __device__ __forceinline__ void cta_barrier_all(uint32_t count) {

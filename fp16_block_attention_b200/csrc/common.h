@@ -84,16 +84,21 @@ cudaError_t launch_select_vertical_window(const void* Q, const void* K, const th
 // Block means of K for the decode selection: km [B][Hkv][nb][D] FP32 (select.cu).
 cudaError_t launch_pool_keys(const void* K, const thrift_shape& s, float* km, cudaStream_t st);
 struct DecodePlan {
-  int tiles_per_cta;  // key tiles of one chunk (<= 8)
-  int chunks;         // chunks per (batch, kv head)
-  int grid;           // persistent CTAs (at most one per SM)
+  int grid16;  // persistent CTAs of the FP16 pass (one per SM unless its chunk tables need more)
+  int ch16;    // FP16 chunk slots per (batch, kv head)
+  int C;       // key tiles per NVFP4 chunk
+  int cpu;     // NVFP4 chunks per (batch, kv head)
+  int grid4;   // persistent CTAs of the NVFP4 pass
 };
 DecodePlan decode_plan(const thrift_shape& s);
 struct DecodeWs {
-  uint8_t* mask;  // [B][Hq][nb] (thrift_decode_step)
-  float* part_o;  // [B][Hq][chunks][D]
-  float* part_l;  // [B][Hq][chunks]
-  float* part_m;  // [B][Hq][chunks]
+  uint8_t* mask;     // [B][Hq][nb] (thrift_decode_step)
+  float* part_o;     // [B][Hq][slots][D]
+  float* part_l;     // [B][Hq][slots]
+  float* part_m;     // [B][Hq][slots]
+  uint16_t* hbits;   // [B][Hkv][nb]: FP16 bits of the group's query heads per key tile
+  uint32_t* list16;  // [B][Hkv][nb]: the tiles some head keeps in FP16
+  int* n16;          // [B][Hkv]
 };
 size_t decode_workspace_bytes(const thrift_shape& s);
 DecodeWs decode_carve(void* ws, const thrift_shape& s);

@@ -17,30 +17,37 @@
 // Kernels:
 //   decode_select     one CTA per (batch, query head): the nb scores, then the
 //                     top k by rank of a unique 64-bit key.
-//   decode_attention  persistent, one CTA per SM walking chunks of <= 8 key
-//                     tiles of one (batch, kv head) with all its G query
-//                     heads, keys on the 128 tensor-memory lanes:
-//                       S^T = K q^T    (M = 128 keys, N = 8 or 16 heads: NVFP4
-//                                       with the prefill's K codes, and fp16 for
-//                                       the tiles a head of the group keeps in FP16)
-//                       P per head and key, relative to the chunk's maximum
-//                       O^T += V^T P^T (M = 128 channels; NVFP4 with the
-//                                       prefill's V codes as A, fp16 V as an
-//                                       MN-major A)
-//                     Two passes per chunk: every S first, so each head has one
-//                     maximum per chunk and O is never rescaled; then P and the
-//                     P V products.  S, O, the query copies and the selection
-//                     bits are double-buffered across chunks, and the loads
-//                     stream through a 10-slot NVFP4 ring and a 3-slot fp16
-//                     ring, so one chunk's products overlap the next one's
-//                     loads.  Writes each chunk's unnormalised O, l and M.
+//   decode_compact    one CTA per (batch, kv head) "unit": per key tile the
+//                     bits of the group's query heads that keep it in FP16,
+//                     and the list of the tiles some head keeps, in order.
+//   decode_attention  two passes, each a persistent kernel (one CTA per SM)
+//                     walking chunks of one unit's key tiles with all its G
+//                     query heads, keys on the 128 tensor-memory lanes:
+//                       NVFP4 pass: chunks of <= 16 consecutive tiles;
+//                         S^T = K q^T from the prefill's K codes, then
+//                         O^T += V^T P^T from its V codes, every head whose
+//                         selection keeps the tile in FP16 masked out;
+//                       FP16 pass: chunks of <= 2 tiles of the unit's list;
+//                         the same products in fp16 (V as an MN-major A), the
+//                         heads that do not keep the tile masked out.
+//                     Every key of every head is computed in exactly one pass.
+//                     Within a chunk two sweeps: every S first (one integer
+//                     maximum per head and chunk, so O is never rescaled),
+//                     then P and the P V products.  S, O and the query copies
+//                     are double-buffered across chunks and the loads stream
+//                     through one ring per pass (23 NVFP4 slots of 9 KB, or 6
+//                     fp16 slots of 32 KB), so one chunk's products overlap the
+//                     next one's loads.  Each chunk writes its unnormalised O,
+//                     l and M per head.
 //   decode_combine    per (batch, query head) and 32 channels: O = sum_c
-//                     2^(M_c - M) O_c / sum_c 2^(M_c - M) l_c (exact
-//                     power-of-two rescales), chunks spread over eight warps.
+//                     2^(M_c - M) O_c / sum_c 2^(M_c - M) l_c over both passes'
+//                     chunks (exact power-of-two rescales).
 // The chunk's own maximum leaves every NVFP4 code of P as under the global
 // one while the group scales stay E4M3 normals (the prefill's argument for
 // its running maximum).
 #include <cuda_fp16.h>
+
+#include <utility>
 
 #include "attention_common.cuh"
 #include "common.h"
@@ -53,92 +60,105 @@ namespace {
 using namespace attn;
 
 constexpr int kDD = 128;         // head dimension
-constexpr int kDThreads = 192;   // warps 0-3 softmax, 4 producer, 5 MMA issuer
+constexpr int kDThreads = 256;   // warps 0-3 softmax, 4 K producer, 5 S issuer, 6 V producer, 7 P V issuer
 constexpr int kDSoftmax = 128;
-constexpr int kDProducer = 4;
-constexpr int kDMma = 5;
-constexpr int kDRing4 = 10;      // NVFP4 slots: K4 + K scales, or V4 + V scales (9 KB)
-constexpr int kDRing16 = 3;      // fp16 slots: one K or V tile (32 KB)
+constexpr int kDProdK = 4;
+constexpr int kDIssueS = 5;      // also owns the tensor memory
+constexpr int kDProdV = 6;
+constexpr int kDIssuePV = 7;
 constexpr int kDMaxChunks = 64;  // chunks one CTA takes (the host plan keeps to it)
 constexpr int kDPBuf = 4;        // P buffers: the softmax threads run up to 4 tiles ahead of P V
-constexpr int kDMaxTiles = 8;    // key tiles of one chunk
+constexpr int kDMaxTiles = 16;   // key tiles of one chunk
+constexpr int kDTiles16 = 2;     // key tiles of one chunk of the FP16 pass
+constexpr int kDMaxSlots = 12;   // slots of one ring
 constexpr uint32_t kDTmemCols = 512;
+constexpr uint32_t kBarPsf = 3;  // named barrier: every softmax warp has written a tile's P scales
 
-// Key tiles per chunk for N = NH query-head columns: two S regions of
-// tiles x 2 NH columns (S4^T then S16^T per tile) fill columns 0-255.
-__host__ __device__ constexpr int decode_chunk_tiles(int NH) { return NH == 8 ? 8 : 4; }
+enum DecodePass : int { kPassFp4 = 0, kPassFp16 = 1 };
+
+// Key tiles per NVFP4 chunk for NH query-head columns: two S regions of
+// tiles x NH columns fill columns 0-255.
+__host__ __device__ constexpr int decode_chunk_tiles(int NH) { return 256 / (2 * NH); }
 
 // Tensor-memory columns (S regions below 256).
 constexpr uint32_t kCO = 256;    // O^T region r at 256 + 16 r
 constexpr uint32_t kCSFK = 288;  // K scales (A of S^T), two 64-wide chunks of D
 constexpr uint32_t kCSFQ = 296;  // q scales of query slot r at 296 + 8 r
 constexpr uint32_t kCSFV = 312;  // V scales (A of O^T), two 64-key chunks
-constexpr uint32_t kCSFP = 320;  // P scales (B of O^T)
+constexpr uint32_t kCSFP = 320;  // P scales of P buffer b (B of O^T) at 320 + 8 b
 
-struct DSmem {
-  // Query copies, two slots (chunk parity): fp16 rows (two SW128 panels of
-  // 16 rows x 128 B), NVFP4 rows (16 x 64 B, SW64), and their scale chunks.
-  static constexpr uint32_t kQSlot = 6144;
-  static constexpr uint32_t kQ16 = 0, kQ4 = 4096, kQSF = 5120;  // within a slot
-  static constexpr uint32_t kP4 = 2 * kQSlot;                // P codes: kDPBuf buffers of 16 x 64 B, SW64
-  static constexpr uint32_t kPSF = kP4 + kDPBuf * 1024;      // P scales: buffers of two 512-byte chunks
-  static constexpr uint32_t kP16 = kPSF + kDPBuf * 1024;     // fp16 P: buffers of two SW128 panels of 2 KB
-  static constexpr uint32_t kSlot4 = 9216;                   // 8 KB codes + 1 KB scales
-  static constexpr uint32_t kRing4 = kP16 + kDPBuf * 4096;
-  static constexpr uint32_t kRing16 = kRing4 + kDRing4 * kSlot4;
-  static constexpr uint32_t kMisc = kRing16 + kDRing16 * 32768;
-  static constexpr uint32_t kSel = kMisc + 1024;   // selection bits of the CTA's chunks
-  static constexpr uint32_t kBytes = kSel + kDMaxChunks * kDMaxTiles * 4;
-  static_assert(kQSlot % 1024 == 0 && kP16 % 1024 == 0 && kRing4 % 1024 == 0 && kRing16 % 1024 == 0,
+// Shared memory of one pass.  Query slots (chunk parity): NVFP4 rows (16 x 64
+// B, SW64) and their two scale chunks, or fp16 rows (two SW128 panels of 16
+// rows x 128 B).  P buffers: NVFP4 codes (16 x 64 B, SW64) and two 512-byte
+// scale chunks, or fp16 P (two SW128 panels).  Ring slots: an NVFP4 K or V tile
+// with its scales (8 KB + 1 KB), or an fp16 K or V tile (two 16 KB panels); K
+// and V have a ring each.
+template <int PASS>
+struct DLayout {
+  static constexpr uint32_t kQSlot = PASS == kPassFp4 ? 2048 : 4096;
+  static constexpr uint32_t kPBuf = PASS == kPassFp4 ? 2048 : 4096;
+  static constexpr uint32_t kSlot = PASS == kPassFp4 ? 9216 : 32768;
+  static constexpr int kSlotsK = PASS == kPassFp4 ? 12 : 3;
+  static constexpr int kSlotsV = PASS == kPassFp4 ? 11 : 3;
+  static constexpr uint32_t kP = 2 * kQSlot;
+  static constexpr uint32_t kRingK = kP + kDPBuf * kPBuf;
+  static constexpr uint32_t kRingV = kRingK + kSlotsK * kSlot;
+  static constexpr uint32_t kMisc = kRingV + kSlotsV * kSlot;
+  static constexpr uint32_t kInfo = kMisc + 2048;               // chunk table (CInfo)
+  static constexpr uint32_t kEntry = kInfo + kDMaxChunks * 16;  // [chunk][i]: tile | FP16 head bits << 16
+  static constexpr uint32_t kBytes = kEntry + kDMaxChunks * kDMaxTiles * 4;
+  static_assert(kSlotsK <= kDMaxSlots && kSlotsV <= kDMaxSlots, "ring barriers");
+  static_assert(kP % 1024 == 0 && kPBuf % 1024 == 0 && kRingK % 1024 == 0 && kSlot % 1024 == 0,
                 "swizzled tiles need 1 KB alignment");
   static_assert(kBytes + 1024 <= 232448, "shared memory above the 227 KB per-CTA limit");
 };
 
 struct DMisc {
   uint64_t bar_q[2];                  // query slot r staged (128 arrivals)
-  uint64_t full4[kDRing4], empty4[kDRing4];
-  uint64_t full16[kDRing16], empty16[kDRing16];
+  uint64_t full_k[kDMaxSlots], empty_k[kDMaxSlots];
+  uint64_t full_v[kDMaxSlots], empty_v[kDMaxSlots];
   uint64_t bar_s[2], s_free[2];       // S region r written / read by the softmax threads (128)
   uint64_t bar_o[2], o_free[2];       // O region r complete / read by the softmax threads (128)
   uint64_t bar_p[kDPBuf], bar_pv[kDPBuf];  // P buffer b written (128) / multiplied into O^T
-  uint64_t bar_drain;
+  uint64_t drain_s, drain_pv;
   uint32_t tmem;
   volatile int abort;
+  int nk;                             // chunks of this CTA
   float red[4][16];                   // per-warp maxima of S
   float lred[4][16];                  // per-warp sums of P
 };
-static_assert(sizeof(DMisc) <= 1024, "barriers must fit their shared-memory slice");
+static_assert(sizeof(DMisc) <= 2048, "barriers must fit their shared-memory slice");
+
+struct CInfo {
+  int unit;   // b * Hkv + kv head
+  int slot;   // partial-result slot of the chunk
+  int nt;     // key tiles
+  int first;  // NVFP4: first tile; FP16: first entry of the unit's list
+};
 
 struct DParams {
-  const __half* q;       // [B][Hq][D]
-  const uint8_t* mask;   // [B][Hq][nb], 1 = FP16 block
-  const uint8_t* ks;     // K scales, prefill layout
-  const uint8_t* vs;     // V scales, prefill layout
-  float* part_o;         // [B][Hq][cpu][D]
-  float* part_l;         // [B][Hq][cpu]
-  float* part_m;         // [B][Hq][cpu]
+  const __half* q;         // [B][Hq][D]
+  const uint16_t* hbits;   // [B * Hkv][NT]: bit g = query head g of the group keeps the tile in FP16
+  const uint32_t* list16;  // [B * Hkv][NT]: the tiles some head keeps, tile | bits << 16, ascending
+  const int* n16;          // [B * Hkv]: entries of each list
+  const uint8_t* ks;       // K scales, prefill layout
+  const uint8_t* vs;       // V scales, prefill layout
+  float* part_o;           // [B][Hq][cap][D]
+  float* part_l;           // [B][Hq][cap]
+  float* part_m;           // [B][Hq][cap]
   uint32_t* err;
+  uint64_t wait_ns;
   int Hq, Hkv, NT, G;
-  int chunk_tiles;       // key tiles per chunk (the last chunk of a unit may be shorter)
-  int cpu;               // chunks per (batch, kv head)
-  int W;                 // chunks in all
-  float c2;              // fl32(sm_scale * log2 e)
+  int units;               // B * Hkv
+  int C;                   // key tiles per NVFP4 chunk (a unit's last chunk may be shorter)
+  int cpu;                 // NVFP4 chunks per unit (partial slots 0 .. cpu - 1)
+  int cap;                 // partial slots per head: NT NVFP4 slots, then ceil(NT / kDTiles16) FP16 slots
+  int grid16;              // CTAs of the FP16 pass (the first of the grid; the rest run the NVFP4 pass)
+  float c2;                // fl32(sm_scale * log2 e)
 };
 
-struct Chunk {
-  int unit, c, t0, nt;
-  size_t head0;
-};
-
-__device__ __forceinline__ Chunk chunk_of(const DParams& p, int w) {
-  Chunk ch;
-  ch.unit = w / p.cpu;
-  ch.c = w % p.cpu;
-  ch.t0 = ch.c * p.chunk_tiles;
-  ch.nt = min(p.chunk_tiles, p.NT - ch.t0);
-  const int b = ch.unit / p.Hkv, hkv = ch.unit % p.Hkv;
-  ch.head0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(hkv) * p.G;
-  return ch;
+__device__ __forceinline__ size_t head0_of(const DParams& p, int unit) {
+  return static_cast<size_t>(unit / p.Hkv) * p.Hq + static_cast<size_t>(unit % p.Hkv) * p.G;
 }
 
 // Thread t's part of a chunk's query rows: 16-element group j = t % 8 of head
@@ -154,80 +174,91 @@ __device__ __forceinline__ void load_query(const DParams& p, size_t head0, int t
   }
 }
 
-// ... into query slot r: fp16 (SW128) and NVFP4 (SW64 codes; scale chunk
-// byte g * 16 + j % 4).
+// ... into query slot r: fp16 rows (SW128) for the FP16 pass; NVFP4 rows
+// (SW64 codes at 0, scale chunk byte g * 16 + j % 4 at 1024) for the other.
+template <int PASS>
 __device__ __forceinline__ void stage_query(uint8_t* sm, int r, int t, const uint4& a, const uint4& c) {
-  uint8_t* slot = sm + r * DSmem::kQSlot;
+  uint8_t* slot = sm + r * DLayout<PASS>::kQSlot;
   const int g = t / 8, j = t % 8;
-  uint8_t* q16 = slot + DSmem::kQ16 + (j / 4) * 2048;
-  *reinterpret_cast<uint4*>(q16 + sw128_off(g, 2 * (j % 4))) = a;
-  *reinterpret_cast<uint4*>(q16 + sw128_off(g, 2 * (j % 4) + 1)) = c;
-  float v[16];
-  const __half2* ha = reinterpret_cast<const __half2*>(&a);
-  const __half2* hc = reinterpret_cast<const __half2*>(&c);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 fa = __half22float2(ha[i]), fc = __half22float2(hc[i]);
-    v[2 * i] = fa.x;
-    v[2 * i + 1] = fa.y;
-    v[8 + 2 * i] = fc.x;
-    v[8 + 2 * i + 1] = fc.y;
-  }
-  const Group16 e = encode16(v);
-  *reinterpret_cast<uint2*>(slot + DSmem::kQ4 + sw64_off(g, j / 2) + 8 * (j % 2)) = make_uint2(e.lo, e.hi);
-  slot[DSmem::kQSF + (j / 4) * 512 + g * 16 + (j % 4)] = static_cast<uint8_t>(e.scale);
-  // rows 16-31 of both scale chunks are never read; keep them zero
-  *reinterpret_cast<uint32_t*>(slot + DSmem::kQSF + (t / 64) * 512 + 256 + (t % 64) * 4) = 0u;
-}
-
-// S4^T and S16^T of tile i from S region address `sreg` (this warp's lanes).
-template <int NH>
-__device__ __forceinline__ void load_s(uint32_t sreg, int i, uint32_t (&s4)[NH], uint32_t (&s16)[NH]) {
-  if constexpr (NH == 8) {
-    uint32_t v[16];
-    tmem_ld16(sreg + 16 * i, v);
-    tmem_ld_wait();
-    tmem_ld_fence(v);
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      s4[g] = v[g];
-      s16[g] = v[8 + g];
-    }
+  if constexpr (PASS == kPassFp16) {
+    uint8_t* q16 = slot + (j / 4) * 2048;
+    *reinterpret_cast<uint4*>(q16 + sw128_off(g, 2 * (j % 4))) = a;
+    *reinterpret_cast<uint4*>(q16 + sw128_off(g, 2 * (j % 4) + 1)) = c;
   } else {
-    tmem_ld16(sreg + 32 * i, s4);
-    tmem_ld16(sreg + 32 * i + 16, s16);
-    tmem_ld_wait();
-    tmem_ld_fence(s4);
-    tmem_ld_fence(s16);
+    float v[16];
+    const __half2* ha = reinterpret_cast<const __half2*>(&a);
+    const __half2* hc = reinterpret_cast<const __half2*>(&c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa = __half22float2(ha[i]), fc = __half22float2(hc[i]);
+      v[2 * i] = fa.x;
+      v[2 * i + 1] = fa.y;
+      v[8 + 2 * i] = fc.x;
+      v[8 + 2 * i + 1] = fc.y;
+    }
+    const Group16 e = encode16(v);
+    *reinterpret_cast<uint2*>(slot + sw64_off(g, j / 2) + 8 * (j % 2)) = make_uint2(e.lo, e.hi);
+    slot[1024 + (j / 4) * 512 + g * 16 + (j % 4)] = static_cast<uint8_t>(e.scale);
+    // rows 16-31 of both scale chunks are never read; keep them zero
+    *reinterpret_cast<uint32_t*>(slot + 1024 + (t / 64) * 512 + 256 + (t % 64) * 4) = 0u;
   }
 }
 
-// Persistent: one CTA per SM takes chunks w = blockIdx.x, + gridDim.x, ...
-// (at most kDMaxChunks).  NH = 8 or 16 query-head columns (G <= NH).  The
-// MMA issuer runs one chunk ahead: S(0), then S(k + 1) before P V(k), so the
-// softmax threads find the next chunk's S ready when they finish a chunk.
+// The NH columns at `addr` (this warp's lanes).
 template <int NH>
-__global__ void __launch_bounds__(kDThreads, 1)
-    thrift_decode_kernel(const __grid_constant__ CUtensorMap mK16, const __grid_constant__ CUtensorMap mV16,
-                         const __grid_constant__ CUtensorMap mK4, const __grid_constant__ CUtensorMap mV4,
-                         const DParams p) {
-  constexpr int kTiles = decode_chunk_tiles(NH);
-  constexpr uint32_t kSRegion = kTiles * 2 * NH;  // S region r at r * kSRegion
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  DMisc& ms = *reinterpret_cast<DMisc*>(sm + DSmem::kMisc);
-  uint32_t* selb = reinterpret_cast<uint32_t*>(sm + DSmem::kSel);  // [chunk][tile]: bit g = head g in FP16
+__device__ __forceinline__ void load_cols(uint32_t addr, uint32_t (&s)[NH]) {
+  if constexpr (NH == 8)
+    tmem_ld8(addr, s);
+  else
+    tmem_ld16(addr, s);
+  tmem_ld_wait();
+  tmem_ld_fence(s);
+}
+
+// Tiles i and i + 1: 2 NH columns at `addr`.
+template <int NH>
+__device__ __forceinline__ void load_pair(uint32_t addr, uint32_t (&s)[2 * NH]) {
+  if constexpr (NH == 8) {
+    tmem_ld16(addr, s);
+    tmem_ld_wait();
+    tmem_ld_fence(s);
+  } else {
+    uint32_t (&a)[16] = *reinterpret_cast<uint32_t(*)[16]>(&s[0]);
+    uint32_t (&b)[16] = *reinterpret_cast<uint32_t(*)[16]>(&s[16]);
+    tmem_ld16(addr, a);
+    tmem_ld16(addr + 16, b);
+    tmem_ld_wait();
+    tmem_ld_fence(a);
+    tmem_ld_fence(b);
+  }
+}
+
+// One CTA of a pass, persistent: CTA x of X takes the chunks w = x, x + X, ...
+// (at most kDMaxChunks; in the FP16 pass the empty ones are dropped).  NG =
+// 4, 8 or 16 query heads the softmax threads compute (G <= NG), NH = max(NG,
+// 8) head columns of the products.  Two producers (K tiles, V tiles) and two
+// tensor-core issuers (S^T = K q^T, O^T += V^T P^T), so the S products of the
+// next chunk run while the softmax threads finish this one and the P V
+// products follow them tile by tile.
+template <int PASS, int NG>
+__device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtensorMap* mV, const DParams& p,
+                                            uint8_t* sm, int x, int X) {
+  using L = DLayout<PASS>;
+  constexpr int NH = NG < 8 ? 8 : NG;
+  constexpr int kTiles = PASS == kPassFp4 ? decode_chunk_tiles(NH) : kDTiles16;
+  constexpr uint32_t kSRegion = kTiles * NH;  // S region r at r * kSRegion
+  static_assert(2 * kSRegion <= kCO, "S regions below the O regions");
+  DMisc& ms = *reinterpret_cast<DMisc*>(sm + L::kMisc);
+  CInfo* info = reinterpret_cast<CInfo*>(sm + L::kInfo);
+  uint32_t* entry = reinterpret_cast<uint32_t*>(sm + L::kEntry);
   const uint32_t sbase = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int G = p.G;
-  const int x = static_cast<int>(blockIdx.x), X = static_cast<int>(gridDim.x);
-  const int nk = x < p.W ? (p.W - x + X - 1) / X : 0;  // chunks of this CTA (<= kDMaxChunks)
 
-  if (warp == kDMma) {
+  if (warp == kDIssueS) {
     tmem_alloc(&ms.tmem, kDTmemCols);
     tmem_relinquish();
   }
-  if (tid == kDProducer * 32) {
+  if (tid == kDProdK * 32) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.bar_q[i], kDSoftmax);
       mbar_init(&ms.bar_s[i], 1);
@@ -239,214 +270,249 @@ __global__ void __launch_bounds__(kDThreads, 1)
       mbar_init(&ms.bar_p[i], kDSoftmax);
       mbar_init(&ms.bar_pv[i], 1);
     }
-    for (int i = 0; i < kDRing4; ++i) {
-      mbar_init(&ms.full4[i], 1);
-      mbar_init(&ms.empty4[i], 1);
+    for (int i = 0; i < L::kSlotsK; ++i) {
+      mbar_init(&ms.full_k[i], 1);
+      mbar_init(&ms.empty_k[i], 1);
     }
-    for (int i = 0; i < kDRing16; ++i) {
-      mbar_init(&ms.full16[i], 1);
-      mbar_init(&ms.empty16[i], 1);
+    for (int i = 0; i < L::kSlotsV; ++i) {
+      mbar_init(&ms.full_v[i], 1);
+      mbar_init(&ms.empty_v[i], 1);
     }
-    mbar_init(&ms.bar_drain, 1);
+    mbar_init(&ms.drain_s, 1);
+    mbar_init(&ms.drain_pv, 1);
     ms.abort = 0;
     fence_mbar_init();
   }
-  // Selection bits of every chunk of this CTA, all loads in flight at once.
+  // The chunk table.  NVFP4: chunk w = x, x + X, ... of the units x cpu chunks
+  // of C consecutive tiles.  FP16: the chunks of kDTiles16 listed tiles,
+  // numbered unit by unit (a running sum over the units' counts), and this CTA
+  // takes g = x, x + X, ... (at most kDMaxChunks: the host sizes X for a list
+  // holding every tile).
+  if (warp == 0) {
+    if constexpr (PASS == kPassFp4) {
+      const int W = p.units * p.cpu;
+      const int nk = x < W ? (W - x + X - 1) / X : 0;
+      for (int k = lane; k < nk; k += 32) {
+        const int w = x + k * X;
+        CInfo c;
+        c.unit = w / p.cpu;
+        c.slot = w % p.cpu;
+        c.first = c.slot * p.C;
+        c.nt = min(p.C, p.NT - c.first);
+        info[k] = c;
+      }
+      if (lane == 0) ms.nk = nk;
+    } else {
+      int run = 0;
+      for (int u0 = 0; u0 < p.units; u0 += 32) {
+        const int u = u0 + lane;
+        const int n = u < p.units ? p.n16[u] : 0;
+        const int nch = (n + kDTiles16 - 1) / kDTiles16;
+        int inc = nch;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += v;
+        }
+        const int P = run + inc - nch;  // first chunk of unit u
+        for (int g = P + ((x - P) % X + X) % X; g < P + nch; g += X) {
+          const int j = g - P;
+          CInfo c;
+          c.unit = u;
+          c.slot = p.NT + j;
+          c.first = j * kDTiles16;
+          c.nt = min(kDTiles16, n - c.first);
+          info[(g - x) / X] = c;
+        }
+        run += __shfl_sync(0xffffffffu, inc, 31);
+      }
+      if (lane == 0) ms.nk = run > x ? (run - x + X - 1) / X : 0;  // run: the chunks of all units
+    }
+  }
+  // P buffers start zero: the rows of heads NG .. 15 and scale rows 16-31 are never written.
+  for (int i = tid; i < kDPBuf * static_cast<int>(L::kPBuf) / 16; i += kDThreads)
+    reinterpret_cast<uint4*>(sm + L::kP)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  const int nk = ms.nk;
   for (int e = tid; e < nk * kDMaxTiles; e += kDThreads) {
     const int k = e / kDMaxTiles, i = e % kDMaxTiles;
-    const Chunk ch = chunk_of(p, x + k * X);
-    uint32_t bits = 0u;
-    if (i < ch.nt) {
-      uint8_t m[16];
-#pragma unroll
-      for (int g = 0; g < 16; ++g) m[g] = g < G ? p.mask[(ch.head0 + g) * p.NT + ch.t0 + i] : 0;
-#pragma unroll
-      for (int g = 0; g < 16; ++g) bits |= (m[g] ? 1u : 0u) << g;
+    const CInfo c = info[k];
+    uint32_t v = 0u;
+    if (i < c.nt) {
+      const size_t row = static_cast<size_t>(c.unit) * p.NT;
+      if constexpr (PASS == kPassFp4) {
+        const int tile = c.first + i;
+        v = static_cast<uint32_t>(tile) | (static_cast<uint32_t>(p.hbits[row + tile]) << 16);
+      } else {
+        v = p.list16[row + c.first + i];
+      }
     }
-    selb[e] = bits;
+    entry[e] = v;
   }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ms.tmem;
+  const uint64_t wns = p.wait_ns;
 
-  if (warp == kDProducer) {
-    // ======================== producer ========================
+  if (warp == kDProdK || warp == kDProdV) {
+    // ======================== producers: K tiles, V tiles ========================
+    const bool is_v = warp == kDProdV;
     if (lane == 0) {
-      prefetch_tensormap(&mK4);
-      prefetch_tensormap(&mV4);
-      int u4 = 0, u16 = 0;
-      auto fill4 = [&](bool is_v, int bhk, int tile) -> bool {
-        const int slot = u4 % kDRing4, use = u4 / kDRing4;
-        if (use > 0 && !wait_or_abort(&ms.empty4[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
-          return false;
-        uint8_t* st = sm + DSmem::kRing4 + slot * DSmem::kSlot4;
-        mbar_arrive_expect_tx(&ms.full4[slot], DSmem::kSlot4);
-        if (!is_v) {
-          tma_load_3d(st, &mK4, &ms.full4[slot], 0, tile * 128, bhk);
-          bulk_load(st + 8192, p.ks + (static_cast<size_t>(bhk) * p.NT + tile) * 1024, 1024, &ms.full4[slot]);
-        } else {
-          tma_load_3d(st, &mV4, &ms.full4[slot], tile * 64, 0, bhk);
-          bulk_load(st + 8192, p.vs + (static_cast<size_t>(bhk) * 2 * p.NT + 2 * tile) * 512, 1024,
-                    &ms.full4[slot]);
-        }
-        ++u4;
-        return true;
-      };
-      auto fill16 = [&](const CUtensorMap* map, int bhk, int tile) -> bool {
-        const int slot = u16 % kDRing16, use = u16 / kDRing16;
-        if (use > 0 && !wait_or_abort(&ms.empty16[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
-          return false;
-        uint8_t* st = sm + DSmem::kRing16 + slot * 32768;
-        mbar_arrive_expect_tx(&ms.full16[slot], 32768);
-        for (int pnl = 0; pnl < 2; ++pnl)
-          tma_load_3d(st + pnl * 16384, map, &ms.full16[slot], pnl * 64, tile * 128, bhk);
-        ++u16;
-        return true;
-      };
-      // The order the MMA issuer consumes: K4 then K16 of chunk k (its S),
-      // V4 (and V16) tile by tile (its P V), with S(k + 1) before P V(k).
-      auto fills_s = [&](int k) -> bool {
-        const Chunk ch = chunk_of(p, x + k * X);
-        for (int i = 0; i < ch.nt; ++i)
-          if (!fill4(false, ch.unit, ch.t0 + i)) return false;
-        for (int i = 0; i < ch.nt; ++i)
-          if (selb[k * kDMaxTiles + i] && !fill16(&mK16, ch.unit, ch.t0 + i)) return false;
-        return true;
-      };
-      auto fills_pv = [&](int k) -> bool {
-        const Chunk ch = chunk_of(p, x + k * X);
-        for (int i = 0; i < ch.nt; ++i) {
-          if (!fill4(true, ch.unit, ch.t0 + i)) return false;
-          if (selb[k * kDMaxTiles + i] && !fill16(&mV16, ch.unit, ch.t0 + i)) return false;
-        }
-        return true;
-      };
-      bool ok = nk == 0 || fills_s(0);
+      const CUtensorMap* map = is_v ? mV : mK;
+      prefetch_tensormap(map);
+      const int slots = is_v ? L::kSlotsV : L::kSlotsK;
+      uint64_t* full = is_v ? ms.full_v : ms.full_k;
+      uint64_t* empty = is_v ? ms.empty_v : ms.empty_k;
+      uint8_t* ring = sm + (is_v ? L::kRingV : L::kRingK);
+      int u = 0;
+      bool ok = true;
       for (int k = 0; ok && k < nk; ++k) {
-        if (k + 1 < nk) ok = fills_s(k + 1);
-        if (ok) ok = fills_pv(k);
+        const CInfo c = info[k];
+        for (int i = 0; ok && i < c.nt; ++i) {
+          const int tile = static_cast<int>(entry[k * kDMaxTiles + i] & 0xFFFFu);
+          const int slot = u % slots, use = u / slots;
+          if (use > 0 && !wait_or_abort(&empty[slot], (use - 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = ring + slot * L::kSlot;
+          mbar_arrive_expect_tx(&full[slot], L::kSlot);
+          if constexpr (PASS == kPassFp4) {
+            if (!is_v) {
+              tma_load_3d(st, map, &full[slot], 0, tile * 128, c.unit);
+              bulk_load(st + 8192, p.ks + (static_cast<size_t>(c.unit) * p.NT + tile) * 1024, 1024, &full[slot]);
+            } else {
+              tma_load_3d(st, map, &full[slot], tile * 64, 0, c.unit);
+              bulk_load(st + 8192, p.vs + (static_cast<size_t>(c.unit) * 2 * p.NT + 2 * tile) * 512, 1024,
+                        &full[slot]);
+            }
+          } else {
+            for (int pnl = 0; pnl < 2; ++pnl)
+              tma_load_3d(st + pnl * 16384, map, &full[slot], pnl * 64, tile * 128, c.unit);
+          }
+          ++u;
+        }
       }
       // Let every copy this thread issued land before the CTA can exit.
-      for (int s = 0; s < kDRing4; ++s)
-        if (u4 > s) mbar_wait(&ms.full4[s], ((u4 - 1 - s) / kDRing4) & 1, kWaitNs);
-      for (int s = 0; s < kDRing16; ++s)
-        if (u16 > s) mbar_wait(&ms.full16[s], ((u16 - 1 - s) / kDRing16) & 1, kWaitNs);
+      for (int s = 0; s < slots; ++s)
+        if (u > s) mbar_wait(&full[s], ((u - 1 - s) / slots) & 1, kWaitNs);
     }
     __syncwarp();
-  } else if (warp == kDMma) {
-    // ======================== MMA issuer ========================
+  } else if (warp == kDIssueS) {
+    // ======================== S issuer: S^T of every tile of chunk k into S region k % 2 ========================
     if (lane == 0) {
       constexpr uint32_t idS4 = idesc_nvf4(128, NH);
       constexpr uint32_t idS16 = idesc_f16(128, NH, false);
-      constexpr uint32_t idO16 = idesc_f16_mn(128, NH, true, false);
-      int u4 = 0, u16 = 0, gt = 0;
-      // S(k): S4^T of every tile, then S16^T of the tiles with an FP16 head, into S region k % 2.
-      auto issue_s = [&](int k) -> bool {
-        const Chunk ch = chunk_of(p, x + k * X);
+      int u = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < nk; ++k) {
+        const CInfo c = info[k];
         const int r = k & 1;
-        if (!wait_or_abort(&ms.bar_q[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) return false;
+        if (!wait_or_abort(&ms.bar_q[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns)) break;
         // S region r was last read by the softmax threads for chunk k - 2.
-        if (k >= 2 && !wait_or_abort(&ms.s_free[r], ((k - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
-          return false;
+        if (k >= 2 && !wait_or_abort(&ms.s_free[r], ((k - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns))
+          break;
         tc_fence_after();
-        const uint32_t qs = sbase + r * DSmem::kQSlot;
-        for (int c = 0; c < 2; ++c)
-          tmem_cp_32x128b_x4(tm + kCSFQ + 8 * r + 4 * c, make_sdesc(qs + DSmem::kQSF + 512 * c, 16, 128, LAYOUT_NONE));
+        const uint32_t qs = sbase + r * L::kQSlot;
+        if constexpr (PASS == kPassFp4)
+          for (int cc = 0; cc < 2; ++cc)
+            tmem_cp_32x128b_x4(tm + kCSFQ + 8 * r + 4 * cc, make_sdesc(qs + 1024 + 512 * cc, 16, 128, LAYOUT_NONE));
         const uint32_t sreg = tm + r * kSRegion;
 #pragma unroll 1
-        for (int i = 0; i < ch.nt; ++i) {
-          const int slot = u4 % kDRing4;
-          if (!wait_or_abort(&ms.full4[slot], (u4 / kDRing4) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
-          ++u4;
+        for (int i = 0; i < c.nt; ++i) {
+          const int slot = u % L::kSlotsK;
+          if (!wait_or_abort(&ms.full_k[slot], (u / L::kSlotsK) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, wns)) {
+            ok = false;
+            break;
+          }
+          ++u;
           tc_fence_after();
-          const uint32_t st = sbase + DSmem::kRing4 + slot * DSmem::kSlot4;
-          for (int c = 0; c < 2; ++c)
-            tmem_cp_32x128b_x4(tm + kCSFK + 4 * c, make_sdesc(st + 8192 + 512 * c, 16, 128, LAYOUT_NONE));
+          const uint32_t st = sbase + L::kRingK + slot * L::kSlot;
+          if constexpr (PASS == kPassFp4) {
+            // these copies follow the previous products in this thread's
+            // tcgen05 order, so they cannot overwrite scales those still read
+            for (int cc = 0; cc < 2; ++cc)
+              tmem_cp_32x128b_x4(tm + kCSFK + 4 * cc, make_sdesc(st + 8192 + 512 * cc, 16, 128, LAYOUT_NONE));
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-            mma_nvf4(sreg + 2 * NH * i, make_sdesc(st + 32 * c, 16, 512, LAYOUT_SW64),
-                     make_sdesc(qs + DSmem::kQ4 + 32 * c, 16, 512, LAYOUT_SW64), idS4, tm + kCSFK + 4 * c,
-                     tm + kCSFQ + 8 * r + 4 * c, c > 0);
-          mma_commit(&ms.empty4[slot]);
-        }
-#pragma unroll 1
-        for (int i = 0; i < ch.nt; ++i) {
-          if (!selb[k * kDMaxTiles + i]) continue;
-          const int slot = u16 % kDRing16;
-          if (!wait_or_abort(&ms.full16[slot], (u16 / kDRing16) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))
-            return false;
-          ++u16;
-          tc_fence_after();
-          const uint32_t k16 = sbase + DSmem::kRing16 + slot * 32768;
+            for (int cc = 0; cc < 2; ++cc)
+              mma_nvf4(sreg + NH * i, make_sdesc(st + 32 * cc, 16, 512, LAYOUT_SW64),
+                       make_sdesc(qs + 32 * cc, 16, 512, LAYOUT_SW64), idS4, tm + kCSFK + 4 * cc,
+                       tm + kCSFQ + 8 * r + 4 * cc, cc > 0);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < kDD / 16; ++kk)
-            mma_f16(sreg + 2 * NH * i + NH,
-                    make_sdesc(k16 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
-                    make_sdesc(qs + DSmem::kQ16 + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idS16,
-                    kk > 0);
-          mma_commit(&ms.empty16[slot]);
+            for (int kk = 0; kk < kDD / 16; ++kk)
+              mma_f16(sreg + NH * i, make_sdesc(st + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128),
+                      make_sdesc(qs + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idS16, kk > 0);
+          }
+          mma_commit(&ms.empty_k[slot]);
         }
+        if (!ok) break;
         mma_commit(&ms.bar_s[r]);
-        return true;
-      };
-      // P V(k): O^T += V^T P^T tile by tile into O region k % 2.
-      auto issue_pv = [&](int k) -> bool {
-        const Chunk ch = chunk_of(p, x + k * X);
+      }
+      // drain: every tensor-core operation this thread issued completes before exit
+      mma_commit(&ms.drain_s);
+      mbar_wait(&ms.drain_s, 0, kWaitNs);
+    }
+    __syncwarp();
+  } else if (warp == kDIssuePV) {
+    // ======================== P V issuer: O^T += V^T P^T tile by tile into O region k % 2 ========================
+    if (lane == 0) {
+      constexpr uint32_t idS4 = idesc_nvf4(128, NH);
+      constexpr uint32_t idO16 = idesc_f16_mn(128, NH, true, false);
+      int u = 0, gt = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < nk; ++k) {
+        const CInfo c = info[k];
         const int r = k & 1;
         // O region r was last read by the softmax threads for chunk k - 2.
-        if (k >= 2 && !wait_or_abort(&ms.o_free[r], ((k - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER))
-          return false;
+        if (k >= 2 && !wait_or_abort(&ms.o_free[r], ((k - 2) >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns))
+          break;
         tc_fence_after();
         const uint32_t oreg = tm + kCO + 16 * r;
 #pragma unroll 1
-        for (int i = 0; i < ch.nt; ++i, ++gt) {
+        for (int i = 0; i < c.nt; ++i, ++gt) {
           const int pb = gt % kDPBuf;
-          const int slot = u4 % kDRing4;
-          if (!wait_or_abort(&ms.full4[slot], (u4 / kDRing4) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD)) return false;
-          ++u4;
+          const int slot = u % L::kSlotsV;
+          if (!wait_or_abort(&ms.full_v[slot], (u / L::kSlotsV) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, wns)) {
+            ok = false;
+            break;
+          }
+          ++u;
           tc_fence_after();
-          const uint32_t st = sbase + DSmem::kRing4 + slot * DSmem::kSlot4;
-          // these copies follow the previous products in this thread's tcgen05
-          // order, so they cannot overwrite scales those still read
-          for (int c = 0; c < 2; ++c)
-            tmem_cp_32x128b_x4(tm + kCSFV + 4 * c, make_sdesc(st + 8192 + 512 * c, 16, 128, LAYOUT_NONE));
-          if (!wait_or_abort(&ms.bar_p[pb], (gt / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER)) return false;
+          const uint32_t st = sbase + L::kRingV + slot * L::kSlot;
+          if constexpr (PASS == kPassFp4)
+            for (int cc = 0; cc < 2; ++cc)
+              tmem_cp_32x128b_x4(tm + kCSFV + 4 * cc, make_sdesc(st + 8192 + 512 * cc, 16, 128, LAYOUT_NONE));
+          if (!wait_or_abort(&ms.bar_p[pb], (gt / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t p4 = sbase + DSmem::kP4 + pb * 1024, psf = sbase + DSmem::kPSF + pb * 1024;
-          for (int c = 0; c < 2; ++c)
-            tmem_cp_32x128b_x4(tm + kCSFP + 4 * c, make_sdesc(psf + 512 * c, 16, 128, LAYOUT_NONE));
+          const uint32_t pbuf = sbase + L::kP + pb * L::kPBuf;
+          if constexpr (PASS == kPassFp4) {
+            // the P scales of buffer pb were written to tensor memory by the softmax threads
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-            mma_nvf4(oreg, make_sdesc(st + 32 * c, 16, 512, LAYOUT_SW64), make_sdesc(p4 + 32 * c, 16, 512, LAYOUT_SW64),
-                     idS4, tm + kCSFV + 4 * c, tm + kCSFP + 4 * c, (i > 0 || c > 0) ? 1u : 0u);
-          if (selb[k * kDMaxTiles + i]) {
-            const int s16 = u16 % kDRing16;
-            if (!wait_or_abort(&ms.full16[s16], (u16 / kDRing16) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD))
-              return false;
-            ++u16;
-            tc_fence_after();
-            const uint32_t v16 = sbase + DSmem::kRing16 + s16 * 32768, p16 = sbase + DSmem::kP16 + pb * 4096;
+            for (int cc = 0; cc < 2; ++cc)
+              mma_nvf4(oreg, make_sdesc(st + 32 * cc, 16, 512, LAYOUT_SW64),
+                       make_sdesc(pbuf + 32 * cc, 16, 512, LAYOUT_SW64), idS4, tm + kCSFV + 4 * cc,
+                       tm + kCSFP + 8 * pb + 4 * cc, (i > 0 || cc > 0) ? 1u : 0u);
+          } else {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_f16(oreg, make_sdesc(v16 + kk * 2048, 16384, 1024, LAYOUT_SW128),
-                      make_sdesc(p16 + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idO16, 1u);
-            mma_commit(&ms.empty16[s16]);
+              mma_f16(oreg, make_sdesc(st + kk * 2048, 16384, 1024, LAYOUT_SW128),
+                      make_sdesc(pbuf + (kk / 4) * 2048 + (kk % 4) * 32, 16, 1024, LAYOUT_SW128), idO16,
+                      (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&ms.empty4[slot]);
+          mma_commit(&ms.empty_v[slot]);
           mma_commit(&ms.bar_pv[pb]);
         }
+        if (!ok) break;
         mma_commit(&ms.bar_o[r]);
-        return true;
-      };
-      bool ok = nk == 0 || issue_s(0);
-      for (int k = 0; ok && k < nk; ++k) {
-        if (k + 1 < nk) ok = issue_s(k + 1);
-        if (ok) ok = issue_pv(k);
       }
-      // drain: every tensor-core operation this thread issued completes before exit
-      mma_commit(&ms.bar_drain);
-      mbar_wait(&ms.bar_drain, 0, kWaitNs);
+      mma_commit(&ms.drain_pv);
+      mbar_wait(&ms.drain_pv, 0, kWaitNs);
     }
     __syncwarp();
   } else {
@@ -458,146 +524,214 @@ __global__ void __launch_bounds__(kDThreads, 1)
     int gt = 0;
     uint4 qa, qc;
     if (nk > 0) {
-      load_query(p, chunk_of(p, x).head0, t, qa, qc);
-      stage_query(sm, 0, t, qa, qc);
+      load_query(p, head0_of(p, info[0].unit), t, qa, qc);
+      stage_query<PASS>(sm, 0, t, qa, qc);
       fence_proxy_async_smem();
       mbar_arrive(&ms.bar_q[0]);
     }
     for (int k = 0; k < nk; ++k) {
-      const Chunk ch = chunk_of(p, x + k * X);
+      const CInfo c = info[k];
+      const size_t head0 = head0_of(p, c.unit);
       const int r = k & 1;
-      const uint32_t* sel = selb + k * kDMaxTiles;
+      const uint32_t* ent = entry + k * kDMaxTiles;
       // the next chunk's query rows, in flight while this chunk's S is read
-      if (k + 1 < nk) load_query(p, chunk_of(p, x + (k + 1) * X).head0, t, qa, qc);
-      // ---- pass 1: maximum of S per head over the chunk ----
-      float mx[NH];
+      if (k + 1 < nk) load_query(p, head0_of(p, info[k + 1].unit), t, qa, qc);
+      // ---- sweep 1: maximum of S per head over the keys this pass computes ----
+      float mx[NG];
 #pragma unroll
-      for (int g = 0; g < NH; ++g) mx[g] = -INFINITY;
-      if (!failed) failed = !wait_or_abort(&ms.bar_s[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      for (int g = 0; g < NG; ++g) mx[g] = -INFINITY;
+      if (!failed) failed = !wait_or_abort(&ms.bar_s[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, wns);
       failed = __any_sync(0xffffffffu, failed);  // tcgen05.ld is warp-collective
       const uint32_t sreg = lane_base + r * kSRegion;
       if (!failed) {
         tc_fence_after();
-        for (int i = 0; i < ch.nt; ++i) {
-          uint32_t s4[NH], s16[NH];
-          load_s<NH>(sreg, i, s4, s16);
-          const uint32_t si = sel[i];
+        // two tiles per load (the second, past the chunk's end, reads columns
+        // of the region that no head takes: mine = 0)
+        for (int i = 0; i < c.nt; i += 2) {
+          uint32_t s[2 * NH];
+          load_pair<NH>(sreg + NH * i, s);
 #pragma unroll
-          for (int g = 0; g < NH; ++g) mx[g] = fmaxf(mx[g], __uint_as_float(((si >> g) & 1u) ? s16[g] : s4[g]));
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t h16 = ent[i + j] >> 16;
+            const uint32_t mine = i + j >= c.nt ? 0u : PASS == kPassFp4 ? ~h16 : h16;  // heads this pass computes
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+              mx[g] = fmaxf(mx[g], ((mine >> g) & 1u) ? __uint_as_float(s[j * NH + g]) : -INFINITY);
+          }
         }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-        for (int g = 0; g < NH; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
+        for (int g = 0; g < NG; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
       if (lane == 0)
 #pragma unroll
-        for (int g = 0; g < NH; ++g) ms.red[warp][g] = mx[g];
+        for (int g = 0; g < NG; ++g) ms.red[warp][g] = mx[g];
       failed = softmax_bar_or<kDSoftmax>(failed);
-      // base_g = 11 - M_g, M_g = ceil(max t) = ceil(fl32(max S * c2)); thread g keeps its M for the epilogue
-      float base[NH];
-      float my_m = 0.f;
+      // base_g = 11 - M_g, M_g = ceil(max t) = ceil(fl32(max S * c2)); thread g
+      // keeps its M for the epilogue.  A head with no key in this chunk's pass
+      // has M = -inf: its P is zero, its l is zero and its M weighs nothing in
+      // the combine.
+      float base[NG];
+      float my_m = -INFINITY;
 #pragma unroll
-      for (int g = 0; g < NH; ++g) {
+      for (int g = 0; g < NG; ++g) {
         const float M = ceilf(fmaxf(fmaxf(ms.red[0][g], ms.red[1][g]), fmaxf(ms.red[2][g], ms.red[3][g])) * c2);
-        base[g] = static_cast<float>(kPLog2) - M;
+        base[g] = static_cast<float>(kPLog2) - (M == -INFINITY ? 0.f : M);
         if (t == g) my_m = M;
       }
       // The next chunk's query slot was last read by the S products of chunk
       // k - 1, which completed before this thread saw bar_s of chunk k - 1.
       if (!failed && k + 1 < nk) {
-        stage_query(sm, r ^ 1, t, qa, qc);
+        stage_query<PASS>(sm, r ^ 1, t, qa, qc);
         fence_proxy_async_smem();
         mbar_arrive(&ms.bar_q[r ^ 1]);
       }
-      // ---- pass 2: P per head and key, encoded into buffer gt % kDPBuf ----
-      float lsum[NH];
+      // ---- sweep 2: P per head and key, into buffer gt % kDPBuf ----
+      float lsum[NG];
 #pragma unroll
-      for (int g = 0; g < NH; ++g) lsum[g] = 0.f;
-      for (int i = 0; i < ch.nt && !failed; ++i, ++gt) {
-        const int pb = gt % kDPBuf;
-        if (gt >= kDPBuf)
-          failed = !wait_or_abort(&ms.bar_pv[pb], ((gt - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
-        failed = __any_sync(0xffffffffu, failed);
-        if (failed) break;
-        tc_fence_after();
-        const uint32_t si = sel[i];
-        uint32_t s4[NH], s16[NH];
-        load_s<NH>(sreg, i, s4, s16);
-        // Every head at once (independent chains): S in the head's precision,
-        // the group maximum over 16 consecutive keys (lanes), the group scale,
-        // P * 2^11 (divided by the scale for an NVFP4 head) and its code.
-        float sv[NH], gm[NH];
+      for (int g = 0; g < NG; ++g) lsum[g] = 0.f;
+      if constexpr (PASS == kPassFp4) {
+        // Two tiles at a time (two independent chains per warp).  failed is the
+        // same in every softmax warp here, and stays so at the end of every pair:
+        // the loop holds a barrier that every softmax warp reaches.
+        for (int i = 0; i < c.nt && !failed;) {
+          const bool two = i + 1 < c.nt;
+          const int pb0 = gt % kDPBuf, pb1 = (gt + 1) % kDPBuf;
+          if (gt >= kDPBuf)
+            failed = !wait_or_abort(&ms.bar_pv[pb0], ((gt - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err,
+                                    DEV_TIMEOUT_MMA, wns);
+          if (!failed && two && gt + 1 >= kDPBuf)
+            failed = !wait_or_abort(&ms.bar_pv[pb1], ((gt + 1 - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err,
+                                    DEV_TIMEOUT_MMA, wns);
+          failed = __any_sync(0xffffffffu, failed);
+          uint8_t* pbuf[2] = {sm + L::kP + pb0 * L::kPBuf, sm + L::kP + pb1 * L::kPBuf};
+          if (!failed) {
+            tc_fence_after();
+            uint32_t s[2 * NH];
+            load_pair<NH>(sreg + NH * i, s);
+            // Every head of both tiles at once: the group maximum over 16
+            // consecutive keys (lanes), the group scale, P * 2^11 / scale and
+            // its code; heads that keep the tile in FP16 get zero codes and
+            // scales.  (The second tile of an odd end is computed and dropped.)
+            uint32_t mine[2];
 #pragma unroll
-        for (int g = 0; g < NH; ++g) {
-          sv[g] = __uint_as_float(((si >> g) & 1u) ? s16[g] : s4[g]);
-          gm[g] = sv[g];
+            for (int j = 0; j < 2; ++j) mine[j] = ~(ent[i + j] >> 16);
+            float gm[2][NG];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int g = 0; g < NG; ++g) gm[j][g] = __uint_as_float(s[j * NH + g]);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int g = 0; g < NG; ++g) gm[j][g] = fmaxf(gm[j][g], __shfl_xor_sync(0xffffffffu, gm[j][g], o));
+            uint32_t wd[2][NG], sbyte[2][NG];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int g = 0; g < NG; ++g) {
+                const bool on = (mine[j] >> g) & 1u;
+                const float amax = ex2(fmaf(gm[j][g], c2, base[g]));  // max of P * 2^11 in the group
+                const uint32_t sb = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;
+                const float sc0 = e4m3_to_f32(sb);
+                const float sc = sc0 <= 0.f ? 1.0f : sc0;  // zero scale: the code rounds to 0, l keeps P
+                const float xv = ex2(fmaf(__uint_as_float(s[j * NH + g]), c2, base[g] - lg2(sc)));  // P 2^11 / scale
+                if (j == 0 || two) lsum[g] = fmaf(on ? xv : 0.f, sc, lsum[g]);
+                sbyte[j][g] = on ? sb : 0u;
+                wd[j][g] = on ? ((cvt_e2m1x2(xv, 0.f) & 0xFu) << (4 * (lane & 7))) : 0u;
+              }
+            // codes of keys 8m .. 8m + 7 in one word (key t at byte t / 2 of row g)
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int g = 0; g < NG; ++g) wd[j][g] |= __shfl_xor_sync(0xffffffffu, wd[j][g], o);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              if (j == 0 || two)
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                  if ((lane & 7) == 0)
+                    *reinterpret_cast<uint32_t*>(pbuf[j] + sw64_off(g, warp) + (lane >> 1)) = wd[j][g];
+                  if ((lane & 15) == 0)
+                    pbuf[j][1024 + (t / 64) * 512 + g * 16 + (t % 64) / 16] = static_cast<uint8_t>(sbyte[j][g]);
+                }
+          }
+          // The P scales into tensor memory, in the layout a 32x128b.warpx4
+          // copy of the two 512-byte scale chunks gives: row g of chunk cc at
+          // lane g of every 32-lane quarter, columns kCSFP + 8 pb + 4 cc ..
+          // + 3.  Each warp writes its own quarter once every warp's bytes are
+          // in; every softmax warp reaches this barrier on every pair, and
+          // leaves together with the others if any gave up a wait.
+          failed = bar_or<kBarPsf, kDSoftmax>(failed);
+          if (failed) break;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (j == 0 || two) {
+              const uint4 r0 = *reinterpret_cast<const uint4*>(pbuf[j] + 1024 + lane * 16);
+              const uint4 r1 = *reinterpret_cast<const uint4*>(pbuf[j] + 1536 + lane * 16);
+              const uint32_t sfw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+              tmem_st8(lane_base + kCSFP + 8 * (j == 0 ? pb0 : pb1), sfw);
+            }
+          tmem_st_wait();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&ms.bar_p[pb0]);
+          if (two) mbar_arrive(&ms.bar_p[pb1]);
+          i += two ? 2 : 1;
+          gt += two ? 2 : 1;
         }
+      } else {
+        for (int i = 0; i < c.nt && !failed; ++i, ++gt) {
+          const int pb = gt % kDPBuf;
+          if (gt >= kDPBuf)
+            failed = !wait_or_abort(&ms.bar_pv[pb], ((gt - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA,
+                                    wns);
+          failed = __any_sync(0xffffffffu, failed);
+          if (failed) break;
+          tc_fence_after();
+          const uint32_t mine = ent[i] >> 16;
+          uint32_t s[NH];
+          load_cols<NH>(sreg + NH * i, s);
+          uint8_t* pbuf = sm + L::kP + pb * L::kPBuf;
 #pragma unroll
-        for (int o = 1; o < 16; o <<= 1)
-#pragma unroll
-          for (int g = 0; g < NH; ++g) gm[g] = fmaxf(gm[g], __shfl_xor_sync(0xffffffffu, gm[g], o));
-        uint32_t wd[NH], sbyte[NH];
-        float x16[NH];
-        // Padding heads (g >= G) have zero query rows: their values are finite
-        // and only reach O^T columns nobody reads, so every head is computed
-        // (straight-line code, so the heads' latency chains overlap).
-#pragma unroll
-        for (int g = 0; g < NH; ++g) {
-          const bool h16 = (si >> g) & 1u;
-          const float amax = ex2(fmaf(gm[g], c2, base[g]));  // max of P * 2^11 in the group
-          const uint32_t sb = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.f) & 0xFFu;
-          const float sc0 = e4m3_to_f32(sb);
-          const float sc = (h16 || sc0 <= 0.f) ? 1.0f : sc0;  // zero scale: the code rounds to 0, l keeps P
-          const float xv = ex2(fmaf(sv[g], c2, base[g] - lg2(sc)));  // P * 2^11 / scale
-          lsum[g] = fmaf(xv, sc, lsum[g]);
-          x16[g] = h16 ? xv : 0.f;
-          sbyte[g] = h16 ? 0u : sb;
-          wd[g] = h16 ? 0u : ((cvt_e2m1x2(xv, 0.f) & 0xFu) << (4 * (lane & 7)));
+          for (int g = 0; g < NG; ++g) {
+            const bool on = (mine >> g) & 1u;
+            const float xv = on ? ex2(fmaf(__uint_as_float(s[g]), c2, base[g])) : 0.f;  // P * 2^11
+            lsum[g] += xv;
+            *reinterpret_cast<__half*>(pbuf + (t / 64) * 2048 + sw128_off(g, (t % 64) / 8) + (t % 8) * 2) =
+                __float2half_rn(xv);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&ms.bar_p[pb]);
         }
-        // codes of keys 8m .. 8m + 7 in one word (key t at byte t / 2 of row g)
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1)
-#pragma unroll
-          for (int g = 0; g < NH; ++g) wd[g] |= __shfl_xor_sync(0xffffffffu, wd[g], o);
-        uint8_t* p4 = sm + DSmem::kP4 + pb * 1024;
-        uint8_t* psf = sm + DSmem::kPSF + pb * 1024;
-        uint8_t* p16 = sm + DSmem::kP16 + pb * 4096;
-#pragma unroll
-        for (int g = 0; g < NH; ++g) {
-          if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(p4 + sw64_off(g, warp) + (lane >> 1)) = wd[g];
-          if ((lane & 15) == 0) psf[(t / 64) * 512 + g * 16 + (t % 64) / 16] = static_cast<uint8_t>(sbyte[g]);
-          if (si)
-            *reinterpret_cast<__half*>(p16 + (t / 64) * 2048 + sw128_off(g, (t % 64) / 8) + (t % 8) * 2) =
-                __float2half_rn(x16[g]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&ms.bar_p[pb]);
       }
       tc_fence_before();
       mbar_arrive(&ms.s_free[r]);
       // ---- epilogue: the chunk's O^T column g, l_g and M_g ----
-      if (!failed) failed = !wait_or_abort(&ms.bar_o[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA);
+      if (!failed) failed = !wait_or_abort(&ms.bar_o[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, wns);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-        for (int g = 0; g < NH; ++g) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], o);
+        for (int g = 0; g < NG; ++g) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], o);
       if (lane == 0)
 #pragma unroll
-        for (int g = 0; g < NH; ++g) ms.lred[warp][g] = lsum[g];
+        for (int g = 0; g < NG; ++g) ms.lred[warp][g] = lsum[g];
       failed = softmax_bar_or<kDSoftmax>(failed);
       if (failed) break;
       tc_fence_after();
-      uint32_t o[16];
-      tmem_ld16(lane_base + kCO + 16 * r, o);
-      tmem_ld_wait();
-      tmem_ld_fence(o);
+      uint32_t o[NH];
+      load_cols<NH>(lane_base + kCO + 16 * r, o);
 #pragma unroll
-      for (int g = 0; g < NH; ++g)
-        if (g < G) p.part_o[((ch.head0 + g) * p.cpu + ch.c) * kDD + t] = __uint_as_float(o[g]);
-      if (t < G) {
-        const size_t idx = (ch.head0 + t) * p.cpu + ch.c;
+      for (int g = 0; g < NG; ++g)
+        if (g < p.G) p.part_o[((head0 + g) * p.cap + c.slot) * kDD + t] = __uint_as_float(o[g]);
+      if (t < p.G) {
+        const size_t idx = (head0 + t) * p.cap + c.slot;
         p.part_l[idx] = (ms.lred[0][t] + ms.lred[1][t]) + (ms.lred[2][t] + ms.lred[3][t]);
         p.part_m[idx] = my_m;
       }
@@ -608,68 +742,142 @@ __global__ void __launch_bounds__(kDThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kDMma) {
+  if (warp == kDIssueS) {
     tc_fence_after();
     tmem_dealloc(tm, kDTmemCols);
   }
 }
 
-// O = sum_c 2^(M_c - M) O_c / sum_c 2^(M_c - M) l_c; both carry the 2^11
-// pre-scale.  Grid (B * Hq, D / 32), 256 threads: the CTA takes 32 channels of
-// one head; warp w sums chunks c = w, w + 8, ... (lanes over channels, so the
-// loads are coalesced and independent), then the eight partial sums are added
-// in a fixed order.  chunks <= 1024.
-__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
+// Both passes in one launch: CTAs 0 .. grid16 - 1 run the FP16 pass, the rest
+// the NVFP4 pass (which needs nothing from the FP16 pass), so NVFP4 CTAs start
+// on the SMs that FP16 CTAs leave.
+// Both passes in one launch: CTAs 0 .. grid16 - 1 run the FP16 pass, the rest
+// the NVFP4 pass (which needs nothing from the FP16 pass), so NVFP4 CTAs start
+// on the SMs that FP16 CTAs leave.
+template <int NG>
+__global__ void __launch_bounds__(kDThreads, 1)
+    thrift_decode_kernel(const __grid_constant__ CUtensorMap mK16, const __grid_constant__ CUtensorMap mV16,
+                         const __grid_constant__ CUtensorMap mK4, const __grid_constant__ CUtensorMap mV4,
+                         const DParams p) {
+  griddep_launch_dependents();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Everything below reads the tile bits, lists and counts of the compaction
+  // kernel and writes partial results the previous combine may still read.
+  griddep_wait();
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < p.grid16)
+    decode_pass<kPassFp16, NG>(&mK16, &mV16, p, sm, b, p.grid16);
+  else
+    decode_pass<kPassFp4, NG>(&mK4, &mV4, p, sm, b - p.grid16, static_cast<int>(gridDim.x) - p.grid16);
+}
+
+// Per unit (b, kv head): bit g of hbits[t] = query head g of the group keeps
+// key tile t in FP16; list16 = the tiles with any bit, ascending, as tile |
+// bits << 16; n16 = their number.  One thread per tile (NT <= 1024).
+__global__ void __launch_bounds__(1024) decode_compact_kernel(const uint8_t* __restrict__ mask, int Hq, int Hkv,
+                                                              int NT, uint16_t* __restrict__ hbits,
+                                                              uint32_t* __restrict__ list16, int* __restrict__ n16) {
+  __shared__ int wtot[32];
+  griddep_launch_dependents();
+  griddep_wait();  // the mask may come from the kernel before
+  const int unit = blockIdx.x, G = Hq / Hkv;
+  const size_t head0 = static_cast<size_t>(unit / Hkv) * Hq + static_cast<size_t>(unit % Hkv) * G;
+  const int t = threadIdx.x, warp = t / 32, lane = t % 32;
+  uint32_t bits = 0u;
+  if (t < NT) {
+    for (int g = 0; g < G; ++g) bits |= (mask[(head0 + g) * NT + t] ? 1u : 0u) << g;
+    hbits[static_cast<size_t>(unit) * NT + t] = static_cast<uint16_t>(bits);
+  }
+  const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
+  if (lane == 0) wtot[warp] = __popc(bal);
+  __syncthreads();
+  int off = 0;
+  for (int w = 0; w < warp; ++w) off += wtot[w];
+  if (bits) list16[static_cast<size_t>(unit) * NT + off + __popc(bal & ((1u << lane) - 1u))] =
+      static_cast<uint32_t>(t) | (bits << 16);
+  if (t == 0) {
+    int n = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x / 32); ++w) n += wtot[w];
+    n16[unit] = n;
+  }
+}
+
+// 2^e for an integer-valued e <= 0, exactly; 0 below 2^-126 and for e = -inf
+// or NaN (a difference of two infinite maxima: chunks that weigh nothing).
+__device__ __forceinline__ float pow2_weight(float e) { return e >= -126.0f ? exp2_int(e) : 0.f; }
+
+// O = sum_c 2^(M_c - M) O_c / sum_c 2^(M_c - M) l_c over the head's NVFP4
+// chunks (slots 0 .. cpu - 1) and FP16 chunks (slots NT ..); both carry the
+// 2^11 pre-scale; a chunk with M_c = -inf holds no key of the head and weighs
+// 0.  One CTA of 512 threads per (batch, query head), one pass over the
+// partial results: warp w merges chunks c = w, w + 16, ... into a running
+// (M, l, O) with lane j holding channels 4 j .. 4 j + 3 (one coalesced
+// 512-byte row per chunk); the maxima are integers, so every rescale is an
+// exact power of two.  Then warp 0 merges the sixteen warps in order.
+__global__ void __launch_bounds__(512) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_l,
-                                                             const float* __restrict__ part_m, int chunks,
-                                                             __half* __restrict__ O) {
-  __shared__ float wsm[1024];
-  __shared__ float red[8][33];
-  __shared__ float s_m, s_l;
+                                                             const float* __restrict__ part_m,
+                                                             const int* __restrict__ n16, int Hq, int Hkv, int NT,
+                                                             int cpu, int cap, __half* __restrict__ O) {
+  constexpr int kWarps = 16;
+  __shared__ float4 red4[kWarps][32];
+  __shared__ float redm[kWarps], redl[kWarps];
+  griddep_wait();  // the passes' partial results
   const size_t bh = blockIdx.x;
-  const int d0 = blockIdx.y * 32;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const float* pm = part_m + bh * chunks;
-  const float* pl = part_l + bh * chunks;
-  const float* po = part_o + bh * chunks * kDD;
-  float m = -INFINITY;
-  for (int c = tid; c < chunks; c += 256) m = fmaxf(m, pm[c]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp][0] = m;
-  __syncthreads();
-  if (tid == 0) {
-    float mm = red[0][0];
-    for (int w = 1; w < 8; ++w) mm = fmaxf(mm, red[w][0]);
-    s_m = mm;
-  }
-  __syncthreads();
-  const float M = s_m;
-  float l = 0.f;
-  for (int c = tid; c < chunks; c += 256) {
-    const float w = exp2_int(pm[c] - M);
-    wsm[c] = w;
-    l = fmaf(w, pl[c], l);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  __syncthreads();  // red[][0] was read above; wsm complete
-  if (lane == 0) red[warp][32] = l;
-  __syncthreads();
-  if (tid == 0) {
-    float ll = 0.f;
-    for (int w = 0; w < 8; ++w) ll += red[w][32];
-    s_l = ll;
-  }
-  float acc = 0.f;
+  const int G = Hq / Hkv;
+  const int unit = static_cast<int>(bh / Hq) * Hkv + static_cast<int>(bh % Hq) / G;
+  const int chunks = cpu + (n16[unit] + kDTiles16 - 1) / kDTiles16;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const float* pm = part_m + bh * cap;
+  const float* pl = part_l + bh * cap;
+  const float4* po = reinterpret_cast<const float4*>(part_o + bh * cap * kDD);
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-  for (int c = warp; c < chunks; c += 8) acc = fmaf(wsm[c], po[static_cast<size_t>(c) * kDD + d0 + lane], acc);
-  red[warp][lane] = acc;
+  for (int c = warp; c < chunks; c += kWarps) {
+    const int slot = c < cpu ? c : NT + (c - cpu);
+    const float mc = pm[slot], lc = pl[slot];
+    const float4 v = po[static_cast<size_t>(slot) * (kDD / 4) + lane];
+    if (mc > M) {  // a new maximum: rescale what is summed so far
+      const float f = pow2_weight(M - mc);
+      acc.x *= f;
+      acc.y *= f;
+      acc.z *= f;
+      acc.w *= f;
+      L *= f;
+      M = mc;
+    }
+    const float wgt = pow2_weight(mc - M);
+    acc.x = fmaf(wgt, v.x, acc.x);
+    acc.y = fmaf(wgt, v.y, acc.y);
+    acc.z = fmaf(wgt, v.z, acc.z);
+    acc.w = fmaf(wgt, v.w, acc.w);
+    L = fmaf(wgt, lc, L);
+  }
+  red4[warp][lane] = acc;
+  if (lane == 0) {
+    redm[warp] = M;
+    redl[warp] = L;
+  }
   __syncthreads();
-  if (tid < 32) {
-    float sum = 0.f;
-    for (int w = 0; w < 8; ++w) sum += red[w][tid];
-    O[bh * kDD + d0 + tid] = __float2half_rn(sum / s_l);
+  if (warp == 0) {
+    float Mt = redm[0];
+    for (int w = 1; w < kWarps; ++w) Mt = fmaxf(Mt, redm[w]);
+    float Lt = 0.f;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = pow2_weight(redm[w] - Mt);
+      const float4 v = red4[w][lane];
+      sum.x = fmaf(f, v.x, sum.x);
+      sum.y = fmaf(f, v.y, sum.y);
+      sum.z = fmaf(f, v.z, sum.z);
+      sum.w = fmaf(f, v.w, sum.w);
+      Lt = fmaf(f, redl[w], Lt);
+    }
+    __half2* out = reinterpret_cast<__half2*>(O + bh * kDD + 4 * lane);
+    out[0] = __floats2half2_rn(sum.x / Lt, sum.y / Lt);
+    out[1] = __floats2half2_rn(sum.z / Lt, sum.w / Lt);
   }
 }
 
@@ -693,6 +901,7 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(const __half* __res
                                                              float sm_scale, long long k, uint8_t* __restrict__ mask) {
   constexpr int kRows = 4;  // key blocks per warp and step, all loads in flight at once
   __shared__ unsigned long long keys[1024];
+  griddep_launch_dependents();
   const size_t bh = blockIdx.x;
   const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
   const int G = Hq / Hkv;
@@ -743,56 +952,122 @@ int sm_count() {
 }
 }  // namespace
 
-// Chunk size for one wave of persistent CTAs: the size (at most the TMEM
-// budget's) that minimises the most key tiles any CTA takes, counting half a
-// tile of per-chunk overhead; ties to the larger chunk.  A CTA takes at most
-// kDMaxChunks chunks (more CTAs than SMs beyond that).
+// The FP16 pass takes one CTA per SM (more if a list holding every tile would
+// give a CTA more than kDMaxChunks chunks); the NVFP4 pass as many again, with
+// the chunk size (at most the TMEM budget's) that minimises the most key tiles
+// any of its CTAs takes, counting half a tile of per-chunk overhead, ties to
+// the larger chunk.
 DecodePlan decode_plan(const thrift_shape& s) {
   const int NT = num_tiles(s.N);
-  const int units = s.B * s.Hkv;
+  const long long units = static_cast<long long>(s.B) * s.Hkv;
   const int NH = (s.Hq / s.Hkv) <= 8 ? 8 : 16;
   const int cmax = decode_chunk_tiles(NH);
-  const int nsm = sm_count();
-  DecodePlan best{1, NT, 1};
+  const long long nsm = sm_count();
+  DecodePlan pl;
+  pl.ch16 = (NT + kDTiles16 - 1) / kDTiles16;
+  const long long need16 = (units * pl.ch16 + kDMaxChunks - 1) / kDMaxChunks;
+  pl.grid16 = static_cast<int>(need16 > nsm ? need16 : nsm);
+  pl.C = cmax < NT ? cmax : NT;
+  pl.cpu = (NT + pl.C - 1) / pl.C;
+  pl.grid4 = static_cast<int>(nsm);
   double best_cost = 1e300;
   for (int C = 1; C <= cmax && C <= NT; ++C) {
-    const int cpu = (NT + C - 1) / C;
-    const long long W = static_cast<long long>(units) * cpu;
+    const long long cpu = (NT + C - 1) / C;
+    const long long W = units * cpu;
     long long grid = W < nsm ? W : nsm;
-    if (grid * kDMaxChunks < W) grid = (W + kDMaxChunks - 1) / kDMaxChunks;  // selection bits of <= 64 chunks
+    if (grid * kDMaxChunks < W) grid = (W + kDMaxChunks - 1) / kDMaxChunks;
     const double cost = static_cast<double>((W + grid - 1) / grid) * (C + 0.5);
     if (cost <= best_cost) {
       best_cost = cost;
-      best.tiles_per_cta = C;
-      best.chunks = cpu;
-      best.grid = static_cast<int>(grid);
+      pl.C = C;
+      pl.cpu = static_cast<int>(cpu);
+      pl.grid4 = static_cast<int>(grid);
     }
   }
-  return best;
+  return pl;
 }
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Sized for one-tile chunks (the most partial results any plan writes).
+// Partial results: NT NVFP4 slots (one-tile chunks, the most any plan makes)
+// and every FP16 chunk slot per head; then the per-unit tile bits, lists and
+// counts.
+static size_t decode_rows(const thrift_shape& s) {
+  const size_t NT = num_tiles(s.N);
+  return static_cast<size_t>(s.B) * s.Hq * (NT + (NT + kDTiles16 - 1) / kDTiles16);
+}
+
 size_t decode_workspace_bytes(const thrift_shape& s) {
-  const size_t rows = static_cast<size_t>(s.B) * s.Hq * num_tiles(s.N);
-  return align256(static_cast<size_t>(s.B) * s.Hq * num_tiles(s.N)) + align256(rows * kDD * sizeof(float)) +
-         2 * align256(rows * sizeof(float));
+  const size_t rows = decode_rows(s);
+  const size_t units = static_cast<size_t>(s.B) * s.Hkv, NT = num_tiles(s.N);
+  return align256(static_cast<size_t>(s.B) * s.Hq * NT) + align256(rows * kDD * sizeof(float)) +
+         2 * align256(rows * sizeof(float)) + align256(units * NT * sizeof(uint16_t)) +
+         align256(units * NT * sizeof(uint32_t)) + align256(units * sizeof(int));
 }
 
 DecodeWs decode_carve(void* ws, const thrift_shape& s) {
-  const size_t rows = static_cast<size_t>(s.B) * s.Hq * num_tiles(s.N);
+  const size_t rows = decode_rows(s);
+  const size_t units = static_cast<size_t>(s.B) * s.Hkv, NT = num_tiles(s.N);
   uint8_t* p = static_cast<uint8_t*>(ws);
   DecodeWs w;
   w.mask = p;
-  p += align256(static_cast<size_t>(s.B) * s.Hq * num_tiles(s.N));
+  p += align256(static_cast<size_t>(s.B) * s.Hq * NT);
   w.part_o = reinterpret_cast<float*>(p);
   p += align256(rows * kDD * sizeof(float));
   w.part_l = reinterpret_cast<float*>(p);
   p += align256(rows * sizeof(float));
   w.part_m = reinterpret_cast<float*>(p);
+  p += align256(rows * sizeof(float));
+  w.hbits = reinterpret_cast<uint16_t*>(p);
+  p += align256(units * NT * sizeof(uint16_t));
+  w.list16 = reinterpret_cast<uint32_t*>(p);
+  p += align256(units * NT * sizeof(uint32_t));
+  w.n16 = reinterpret_cast<int*>(p);
   return w;
 }
+
+namespace {
+// Launch on `st` with programmatic stream serialization: the kernel may start
+// while the one before it in the stream finishes, and waits for it
+// (griddepcontrol.wait) before touching what that one writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Every decode kernel asks for the largest shared-memory carveout, so that
+// consecutive kernels of a step do not make the SMs change their L1 / shared
+// split between them.
+template <typename K>
+cudaError_t max_carveout(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
+}
+
+template <int NG>
+cudaError_t launch_passes(const CUtensorMap (&maps)[4], const DParams& prm, const DecodePlan& pl, cudaStream_t st) {
+  const size_t smem = (DLayout<kPassFp4>::kBytes > DLayout<kPassFp16>::kBytes ? DLayout<kPassFp4>::kBytes
+                                                                                : DLayout<kPassFp16>::kBytes) +
+                      1024;
+  cudaError_t e = cudaFuncSetAttribute(thrift_decode_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if ((e = max_carveout(thrift_decode_kernel<NG>)) != cudaSuccess) return e;
+  return launch_dependent(thrift_decode_kernel<NG>, dim3(pl.grid16 + pl.grid4), dim3(kDThreads), smem, st, maps[0],
+                          maps[1], maps[2], maps[3], prm);
+}
+}  // namespace
 
 cudaError_t launch_decode_select(const void* q, const float* km, const thrift_shape& s, double rho, uint8_t* mask,
                                  cudaStream_t st) {
@@ -800,6 +1075,8 @@ cudaError_t launch_decode_select(const void* q, const float* km, const thrift_sh
   double kk = ceil(rho * static_cast<double>(nb) - 1e-9);
   if (kk < 0) kk = 0;
   if (kk > nb) kk = nb;
+  const cudaError_t e = max_carveout(decode_select_kernel);
+  if (e != cudaSuccess) return e;
   decode_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(static_cast<const __half*>(q), km, s.Hq, s.Hkv, nb, s.sm_scale,
                                                    static_cast<long long>(kk), mask);
   return cudaGetLastError();
@@ -808,52 +1085,58 @@ cudaError_t launch_decode_select(const void* q, const float* km, const thrift_sh
 cudaError_t launch_decode_attention(const void* q, const void* K, const void* V, const void* k4, const void* ks,
                                     const void* v4, const void* vs, const uint8_t* mask, const thrift_shape& s,
                                     void* O, const DecodeWs& w, uint32_t* err, cudaStream_t st) {
-  CUtensorMap mK16, mV16, mK4, mV4;
+  CUtensorMap maps[4];  // fp16 K, fp16 V, NVFP4 K, NVFP4 V
   const uint64_t BHk = static_cast<uint64_t>(s.B) * s.Hkv;
   bool ok = true;
-  ok &= make_tmap_3d(&mK16, K, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kDD, s.N, BHk, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_tmap_3d(&mV16, V, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kDD, s.N, BHk, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_tmap_3d(&mK4, k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kDD / 2, s.N, BHk, kDD / 2, 128,
+  ok &= make_tmap_3d(&maps[0], K, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kDD, s.N, BHk, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_tmap_3d(&maps[1], V, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kDD, s.N, BHk, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_tmap_3d(&maps[2], k4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kDD / 2, s.N, BHk, kDD / 2, 128,
                      CU_TENSOR_MAP_SWIZZLE_64B);
-  ok &= make_tmap_3d(&mV4, v4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.N / 2, kDD, BHk, 64, kDD, CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= make_tmap_3d(&maps[3], v4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.N / 2, kDD, BHk, 64, kDD,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
   if (!ok) return cudaErrorInvalidValue;
   const DecodePlan pl = decode_plan(s);
   const int G = s.Hq / s.Hkv;
+  const int NT = num_tiles(s.N);
+  cudaError_t e = max_carveout(decode_compact_kernel);
+  if (e != cudaSuccess) return e;
+  if ((e = max_carveout(decode_combine_kernel)) != cudaSuccess) return e;
+  e = launch_dependent(decode_compact_kernel, dim3(static_cast<unsigned>(BHk)), dim3(1024), 0, st, mask, s.Hq, s.Hkv,
+                       NT, w.hbits, w.list16, w.n16);
+  if (e != cudaSuccess) return e;
   DParams prm;
   prm.q = static_cast<const __half*>(q);
-  prm.mask = mask;
+  prm.hbits = w.hbits;
+  prm.list16 = w.list16;
+  prm.n16 = w.n16;
   prm.ks = static_cast<const uint8_t*>(ks);
   prm.vs = static_cast<const uint8_t*>(vs);
   prm.part_o = w.part_o;
   prm.part_l = w.part_l;
   prm.part_m = w.part_m;
   prm.err = err;
+  prm.wait_ns = wait_limit_ns();
   prm.Hq = s.Hq;
   prm.Hkv = s.Hkv;
-  prm.NT = num_tiles(s.N);
+  prm.NT = NT;
   prm.G = G;
-  prm.chunk_tiles = pl.tiles_per_cta;
-  prm.cpu = pl.chunks;
-  prm.W = static_cast<int>(BHk) * pl.chunks;
+  prm.units = static_cast<int>(BHk);
+  prm.C = pl.C;
+  prm.cpu = pl.cpu;
+  prm.cap = NT + pl.ch16;
+  prm.grid16 = pl.grid16;
   prm.c2 = static_cast<float>(static_cast<double>(s.sm_scale) * 1.4426950408889634073599246810019);
-  const size_t smem = DSmem::kBytes + 1024;
-  cudaError_t e;
-  if (G <= 8) {
-    e = cudaFuncSetAttribute(thrift_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    thrift_decode_kernel<8><<<pl.grid, kDThreads, smem, st>>>(mK16, mV16, mK4, mV4, prm);
-  } else {
-    e = cudaFuncSetAttribute(thrift_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    thrift_decode_kernel<16><<<pl.grid, kDThreads, smem, st>>>(mK16, mV16, mK4, mV4, prm);
-  }
-  e = cudaGetLastError();
+  if (G <= 4)
+    e = launch_passes<4>(maps, prm, pl, st);
+  else if (G <= 8)
+    e = launch_passes<8>(maps, prm, pl, st);
+  else
+    e = launch_passes<16>(maps, prm, pl, st);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(s.B * s.Hq, kDD / 32), 256, 0, st>>>(w.part_o, w.part_l, w.part_m, pl.chunks,
-                                                                     static_cast<__half*>(O));
-  return cudaGetLastError();
+  return launch_dependent(decode_combine_kernel, dim3(s.B * s.Hq), dim3(512), 0, st, w.part_o, w.part_l, w.part_m,
+                          w.n16, s.Hq, s.Hkv, NT, pl.cpu, prm.cap, static_cast<__half*>(O));
 }
 
 }  // namespace thrift
