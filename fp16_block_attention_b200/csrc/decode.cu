@@ -891,53 +891,86 @@ __device__ __forceinline__ uint64_t decode_key(float score, int j, int nb) {
   return (forced << 63) | (static_cast<uint64_t>(u) << 31) | (0x7FFFFFFFull - static_cast<uint64_t>(j));
 }
 
-// One CTA per (batch, query head); nb <= 1024, D = 128.  score_j =
-// fl32(sm_scale * fl32(q . kmean_j)): the products of the fp16 query and the
-// FP32 means are exact in FP64; the FP64 sum (a warp tree, one warp per key
-// block, lanes over channels) is rounded once.  Then the top k by rank of a
-// unique key.
+// One CTA of 1024 threads per (batch, query head); nb <= 1024, D = 128.
+// score_j = fl32(sm_scale * fl32(q . kmean_j)): the products of the fp16
+// query and the FP32 means are exact in FP64; their FP64 sum (one warp per key
+// block, lane l holding channels 4 l .. 4 l + 3 so that a block's 512 bytes
+// are one coalesced load, then a warp tree) is rounded once.  Then the top k
+// of the unique 64-bit keys: a bitonic sort into descending order (stages
+// across warps through shared memory, stages within a warp by shuffles), and
+// the first k sorted keys name the selected blocks.  The keys are unique, so
+// the set is the k largest, as a ranking would give.
 __global__ void __launch_bounds__(1024) decode_select_kernel(const __half* __restrict__ q,
                                                              const float* __restrict__ km, int Hq, int Hkv, int nb,
                                                              float sm_scale, long long k, uint8_t* __restrict__ mask) {
-  constexpr int kRows = 4;  // key blocks per warp and step, all loads in flight at once
+  constexpr int kRows = 8;  // key blocks per warp and step, all loads in flight at once
   __shared__ unsigned long long keys[1024];
+  __shared__ uint8_t sel[1024];
   griddep_launch_dependents();
   const size_t bh = blockIdx.x;
   const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
   const int G = Hq / Hkv;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
+  const int i = threadIdx.x, warp = i / 32, lane = i % 32;
   const float* kmh = km + (static_cast<size_t>(b) * Hkv + h / G) * nb * static_cast<size_t>(kDD);
-  double qd[kDD / 32];
-#pragma unroll
-  for (int i = 0; i < kDD / 32; ++i) qd[i] = static_cast<double>(__half2float(q[bh * kDD + lane + 32 * i]));
-  for (int j0 = warp * kRows; j0 < nb; j0 += nwarps * kRows) {
-    float v[kRows][kDD / 32];
+  double qd[4];
+  {
+    const uint2 qv = *reinterpret_cast<const uint2*>(q + bh * kDD + 4 * lane);
+    const float2 q01 = __half22float2(*reinterpret_cast<const __half2*>(&qv.x));
+    const float2 q23 = __half22float2(*reinterpret_cast<const __half2*>(&qv.y));
+    qd[0] = q01.x;
+    qd[1] = q01.y;
+    qd[2] = q23.x;
+    qd[3] = q23.y;
+  }
+  sel[i] = 0;
+  if (i >= nb) keys[i] = 0ull;  // padding past nb sorts last (blocks below nb are all written below)
+  for (int j0 = warp * kRows; j0 < nb; j0 += 32 * kRows) {
+    float4 v[kRows];
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
-#pragma unroll
-      for (int i = 0; i < kDD / 32; ++i)
-        v[r][i] = j0 + r < nb ? kmh[static_cast<size_t>(j0 + r) * kDD + lane + 32 * i] : 0.f;
+      v[r] = j0 + r < nb ? reinterpret_cast<const float4*>(kmh + static_cast<size_t>(j0 + r) * kDD)[lane]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    double dot[kRows];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
-      double dot = 0.0;
+      dot[r] = fma(qd[0], static_cast<double>(v[r].x), fma(qd[1], static_cast<double>(v[r].y),
+               fma(qd[2], static_cast<double>(v[r].z), qd[3] * static_cast<double>(v[r].w))));
+    }
 #pragma unroll
-      for (int i = 0; i < kDD / 32; ++i) dot = fma(qd[i], static_cast<double>(v[r][i]), dot);
+    for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      if (lane == 0 && j0 + r < nb) {
-        const float sc =
-            static_cast<float>(static_cast<double>(sm_scale) * static_cast<double>(static_cast<float>(dot)));
-        keys[j0 + r] = decode_key(sc, j0 + r, nb);
-      }
+      for (int r = 0; r < kRows; ++r) dot[r] += __shfl_xor_sync(0xffffffffu, dot[r], o);
+    if (lane < kRows && j0 + lane < nb) {
+      double d = dot[0];
+#pragma unroll
+      for (int r = 1; r < kRows; ++r) d = lane == r ? dot[r] : d;
+      const float sc = static_cast<float>(static_cast<double>(sm_scale) * static_cast<double>(static_cast<float>(d)));
+      keys[j0 + lane] = decode_key(sc, j0 + lane, nb);
     }
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
-    const unsigned long long kj = keys[j];
-    int rank = 0;
-    for (int jj = 0; jj < nb; ++jj) rank += keys[jj] > kj ? 1 : 0;
-    mask[bh * nb + j] = rank < k ? 1 : 0;
+  unsigned long long key = keys[i];
+  // bitonic sort of the 1024 keys, descending (element i held by thread i)
+  for (int kk = 2; kk <= 1024; kk <<= 1) {
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      unsigned long long other;
+      if (j >= 32) {
+        keys[i] = key;
+        __syncthreads();
+        other = keys[i ^ j];
+        __syncthreads();
+      } else {
+        other = __shfl_xor_sync(0xffffffffu, key, j);
+      }
+      // the pair (i, i ^ j) is ordered descending in blocks where (i & kk) == 0
+      const bool lower = (i & j) == 0, desc = (i & kk) == 0;
+      const bool take_max = lower == desc;
+      key = take_max ? (key > other ? key : other) : (key < other ? key : other);
+    }
   }
+  if (i < k) sel[0x7FFFFFFF - static_cast<int>(key & 0x7FFFFFFFull)] = 1;
+  __syncthreads();
+  if (i < nb) mask[bh * nb + i] = sel[i];
 }
 
 }  // namespace
