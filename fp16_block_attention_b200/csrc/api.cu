@@ -26,7 +26,15 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-thrift_status from_cuda(cudaError_t e) { return e == cudaSuccess ? THRIFT_OK : THRIFT_ERR_CUDA; }
+// A failed launch or call also leaves its error as the runtime's last error,
+// which the next launch's check would report again: read it here, so that one
+// failed call does not fail the next (an error that poisons the context
+// stays, as it must).
+thrift_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return THRIFT_OK;
+  cudaGetLastError();
+  return THRIFT_ERR_CUDA;
+}
 
 struct QuantSizes {
   size_t codes, scales;

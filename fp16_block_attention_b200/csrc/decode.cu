@@ -27,7 +27,7 @@
 //                         S^T = K q^T from the prefill's K codes, then
 //                         O^T += V^T P^T from its V codes, every head whose
 //                         selection keeps the tile in FP16 masked out;
-//                       FP16 pass: chunks of <= 2 tiles of the unit's list;
+//                       FP16 pass: chunks of <= 4 tiles of the unit's list;
 //                         the same products in fp16 (V as an MN-major A), the
 //                         heads that do not keep the tile masked out.
 //                     Every key of every head is computed in exactly one pass.
@@ -47,6 +47,7 @@
 // its running maximum).
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <utility>
 
 #include "attention_common.cuh"
@@ -60,19 +61,34 @@ namespace {
 using namespace attn;
 
 constexpr int kDD = 128;         // head dimension
-constexpr int kDThreads = 256;   // warps 0-3 softmax, 4 K producer, 5 S issuer, 6 V producer, 7 P V issuer
-constexpr int kDSoftmax = 128;
-constexpr int kDProdK = 4;
-constexpr int kDIssueS = 5;      // also owns the tensor memory
-constexpr int kDProdV = 6;
-constexpr int kDIssuePV = 7;
+// Warp roles: 4 softmax warps per softmax warpgroup (one or two), then the K
+// producer, the S issuer (which also owns the tensor memory), the V producer,
+// the P V issuer and, with at most 8 heads, a V scale copier.  The two-group
+// form (4 heads) alternates pairs of key tiles between the groups.  Registers
+// are granted to an SM's warps four at a time, so the register budget is
+// that of the thread count rounded up to 128: 16 heads need about 220
+// registers a thread and run without a copier (256 threads, its P V issuer
+// copies the V scales itself); 8 heads about 150 (288 threads, bounded as
+// 384); 4 heads about 110 (416 threads with two groups, bounded as 512).
+template <int NG>
+struct DCfg {
+  static constexpr int kGroups = NG == 4 ? 2 : 1;
+  static constexpr bool kCopier = NG < 16;
+  static constexpr int kSoftWarps = 4 * kGroups;
+  static constexpr int kSoft = 32 * kSoftWarps;  // softmax threads
+  static constexpr int kProdK = kSoftWarps, kIssueS = kSoftWarps + 1, kProdV = kSoftWarps + 2,
+                       kIssuePV = kSoftWarps + 3, kCopyV = kSoftWarps + 4;
+  static constexpr int kThreads = 32 * (kSoftWarps + 4 + (kCopier ? 1 : 0));
+  static constexpr int kBound = (kThreads + 127) / 128 * 128;
+};
+constexpr int kDGroup = 128;     // threads of one softmax warpgroup
 constexpr int kDMaxChunks = 64;  // chunks one CTA takes (the host plan keeps to it)
 constexpr int kDPBuf = 4;        // P buffers: the softmax threads run up to 4 tiles ahead of P V
 constexpr int kDMaxTiles = 16;   // key tiles of one chunk
-constexpr int kDTiles16 = 2;     // key tiles of one chunk of the FP16 pass
+constexpr int kDTiles16 = 4;     // key tiles of one chunk of the FP16 pass
 constexpr int kDMaxSlots = 12;   // slots of one ring
 constexpr uint32_t kDTmemCols = 512;
-constexpr uint32_t kBarPsf = 3;  // named barrier: every softmax warp has written a tile's P scales
+constexpr uint32_t kBarPsf = 3;  // named barriers 3, 4: a softmax group's warps have written a tile's P scales
 
 enum DecodePass : int { kPassFp4 = 0, kPassFp16 = 1 };
 
@@ -84,8 +100,8 @@ __host__ __device__ constexpr int decode_chunk_tiles(int NH) { return 256 / (2 *
 constexpr uint32_t kCO = 256;    // O^T region r at 256 + 16 r
 constexpr uint32_t kCSFK = 288;  // K scales (A of S^T), two 64-wide chunks of D
 constexpr uint32_t kCSFQ = 296;  // q scales of query slot r at 296 + 8 r
-constexpr uint32_t kCSFV = 312;  // V scales (A of O^T), two 64-key chunks
 constexpr uint32_t kCSFP = 320;  // P scales of P buffer b (B of O^T) at 320 + 8 b
+constexpr uint32_t kCSFV = 352;  // V scales of V ring slot s (A of O^T, two 64-key chunks) at 352 + 8 s
 
 // Shared memory of one pass.  Query slots (chunk parity): NVFP4 rows (16 x 64
 // B, SW64) and their two scale chunks, or fp16 rows (two SW128 panels of 16
@@ -120,12 +136,13 @@ struct DMisc {
   uint64_t bar_s[2], s_free[2];       // S region r written / read by the softmax threads (128)
   uint64_t bar_o[2], o_free[2];       // O region r complete / read by the softmax threads (128)
   uint64_t bar_p[kDPBuf], bar_pv[kDPBuf];  // P buffer b written (128) / multiplied into O^T
-  uint64_t drain_s, drain_pv;
+  uint64_t vsf_ready[kDMaxSlots];     // NVFP4 pass: V scales of ring slot s in tensor memory
+  uint64_t drain_s, drain_pv, drain_cp;
   uint32_t tmem;
   volatile int abort;
   int nk;                             // chunks of this CTA
-  float red[4][16];                   // per-warp maxima of S
-  float lred[4][16];                  // per-warp sums of P
+  float red[8][16];                   // per-warp maxima of S
+  float lred[8][16];                  // per-warp sums of P
 };
 static_assert(sizeof(DMisc) <= 2048, "barriers must fit their shared-memory slice");
 
@@ -244,6 +261,7 @@ template <int PASS, int NG>
 __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtensorMap* mV, const DParams& p,
                                             uint8_t* sm, int x, int X) {
   using L = DLayout<PASS>;
+  using Cfg = DCfg<NG>;
   constexpr int NH = NG < 8 ? 8 : NG;
   constexpr int kTiles = PASS == kPassFp4 ? decode_chunk_tiles(NH) : kDTiles16;
   constexpr uint32_t kSRegion = kTiles * NH;  // S region r at r * kSRegion
@@ -254,20 +272,20 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
   const uint32_t sbase = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
-  if (warp == kDIssueS) {
+  if (warp == Cfg::kIssueS) {
     tmem_alloc(&ms.tmem, kDTmemCols);
     tmem_relinquish();
   }
-  if (tid == kDProdK * 32) {
+  if (tid == Cfg::kProdK * 32) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ms.bar_q[i], kDSoftmax);
+      mbar_init(&ms.bar_q[i], kDGroup);        // staged by softmax group 0
       mbar_init(&ms.bar_s[i], 1);
-      mbar_init(&ms.s_free[i], kDSoftmax);
+      mbar_init(&ms.s_free[i], Cfg::kSoft);    // read by every softmax thread
       mbar_init(&ms.bar_o[i], 1);
-      mbar_init(&ms.o_free[i], kDSoftmax);
+      mbar_init(&ms.o_free[i], kDGroup);       // read by softmax group 0
     }
     for (int i = 0; i < kDPBuf; ++i) {
-      mbar_init(&ms.bar_p[i], kDSoftmax);
+      mbar_init(&ms.bar_p[i], kDGroup);        // each tile's P comes from one group
       mbar_init(&ms.bar_pv[i], 1);
     }
     for (int i = 0; i < L::kSlotsK; ++i) {
@@ -277,9 +295,11 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
     for (int i = 0; i < L::kSlotsV; ++i) {
       mbar_init(&ms.full_v[i], 1);
       mbar_init(&ms.empty_v[i], 1);
+      mbar_init(&ms.vsf_ready[i], 1);
     }
     mbar_init(&ms.drain_s, 1);
     mbar_init(&ms.drain_pv, 1);
+    mbar_init(&ms.drain_cp, 1);
     ms.abort = 0;
     fence_mbar_init();
   }
@@ -330,11 +350,11 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
     }
   }
   // P buffers start zero: the rows of heads NG .. 15 and scale rows 16-31 are never written.
-  for (int i = tid; i < kDPBuf * static_cast<int>(L::kPBuf) / 16; i += kDThreads)
+  for (int i = tid; i < kDPBuf * static_cast<int>(L::kPBuf) / 16; i += Cfg::kThreads)
     reinterpret_cast<uint4*>(sm + L::kP)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   const int nk = ms.nk;
-  for (int e = tid; e < nk * kDMaxTiles; e += kDThreads) {
+  for (int e = tid; e < nk * kDMaxTiles; e += Cfg::kThreads) {
     const int k = e / kDMaxTiles, i = e % kDMaxTiles;
     const CInfo c = info[k];
     uint32_t v = 0u;
@@ -356,9 +376,9 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
   const uint32_t tm = ms.tmem;
   const uint64_t wns = p.wait_ns;
 
-  if (warp == kDProdK || warp == kDProdV) {
+  if (warp == Cfg::kProdK || warp == Cfg::kProdV) {
     // ======================== producers: K tiles, V tiles ========================
-    const bool is_v = warp == kDProdV;
+    const bool is_v = warp == Cfg::kProdV;
     if (lane == 0) {
       const CUtensorMap* map = is_v ? mV : mK;
       prefetch_tensormap(map);
@@ -366,6 +386,9 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       uint64_t* full = is_v ? ms.full_v : ms.full_k;
       uint64_t* empty = is_v ? ms.empty_v : ms.empty_k;
       uint8_t* ring = sm + (is_v ? L::kRingV : L::kRingK);
+      // every cache tile is read once per step: let it leave L2 first (the
+      // partial results the combine reads stay)
+      const uint64_t pol = l2_evict_first_policy();
       int u = 0;
       bool ok = true;
       for (int k = 0; ok && k < nk; ++k) {
@@ -381,16 +404,17 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
           mbar_arrive_expect_tx(&full[slot], L::kSlot);
           if constexpr (PASS == kPassFp4) {
             if (!is_v) {
-              tma_load_3d(st, map, &full[slot], 0, tile * 128, c.unit);
-              bulk_load(st + 8192, p.ks + (static_cast<size_t>(c.unit) * p.NT + tile) * 1024, 1024, &full[slot]);
+              tma_load_3d_hint(st, map, &full[slot], 0, tile * 128, c.unit, pol);
+              bulk_load_hint(st + 8192, p.ks + (static_cast<size_t>(c.unit) * p.NT + tile) * 1024, 1024, &full[slot],
+                             pol);
             } else {
-              tma_load_3d(st, map, &full[slot], tile * 64, 0, c.unit);
-              bulk_load(st + 8192, p.vs + (static_cast<size_t>(c.unit) * 2 * p.NT + 2 * tile) * 512, 1024,
-                        &full[slot]);
+              tma_load_3d_hint(st, map, &full[slot], tile * 64, 0, c.unit, pol);
+              bulk_load_hint(st + 8192, p.vs + (static_cast<size_t>(c.unit) * 2 * p.NT + 2 * tile) * 512, 1024,
+                             &full[slot], pol);
             }
           } else {
             for (int pnl = 0; pnl < 2; ++pnl)
-              tma_load_3d(st + pnl * 16384, map, &full[slot], pnl * 64, tile * 128, c.unit);
+              tma_load_3d_hint(st + pnl * 16384, map, &full[slot], pnl * 64, tile * 128, c.unit, pol);
           }
           ++u;
         }
@@ -400,7 +424,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
         if (u > s) mbar_wait(&full[s], ((u - 1 - s) / slots) & 1, kWaitNs);
     }
     __syncwarp();
-  } else if (warp == kDIssueS) {
+  } else if (warp == Cfg::kIssueS) {
     // ======================== S issuer: S^T of every tile of chunk k into S region k % 2 ========================
     if (lane == 0) {
       constexpr uint32_t idS4 = idesc_nvf4(128, NH);
@@ -456,7 +480,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       mbar_wait(&ms.drain_s, 0, kWaitNs);
     }
     __syncwarp();
-  } else if (warp == kDIssuePV) {
+  } else if (warp == Cfg::kIssuePV) {
     // ======================== P V issuer: O^T += V^T P^T tile by tile into O region k % 2 ========================
     if (lane == 0) {
       constexpr uint32_t idS4 = idesc_nvf4(128, NH);
@@ -475,16 +499,22 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
         for (int i = 0; i < c.nt; ++i, ++gt) {
           const int pb = gt % kDPBuf;
           const int slot = u % L::kSlotsV;
-          if (!wait_or_abort(&ms.full_v[slot], (u / L::kSlotsV) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, wns)) {
+          // NVFP4 with a copier: it has put the slot's V scales into tensor
+          // memory (after the copy landed); otherwise the copy itself
+          constexpr bool kViaCopier = PASS == kPassFp4 && Cfg::kCopier;
+          if (!wait_or_abort(kViaCopier ? &ms.vsf_ready[slot] : &ms.full_v[slot], (u / L::kSlotsV) & 1, &ms.abort,
+                             p.err, DEV_TIMEOUT_LOAD, wns)) {
             ok = false;
             break;
           }
           ++u;
           tc_fence_after();
           const uint32_t st = sbase + L::kRingV + slot * L::kSlot;
-          if constexpr (PASS == kPassFp4)
+          // (this slot's columns were last read by products of this thread,
+          // which the copies follow in its tcgen05 order)
+          if constexpr (PASS == kPassFp4 && !kViaCopier)
             for (int cc = 0; cc < 2; ++cc)
-              tmem_cp_32x128b_x4(tm + kCSFV + 4 * cc, make_sdesc(st + 8192 + 512 * cc, 16, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4(tm + kCSFV + 8 * slot + 4 * cc, make_sdesc(st + 8192 + 512 * cc, 16, 128, LAYOUT_NONE));
           if (!wait_or_abort(&ms.bar_p[pb], (gt / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_OTHER, wns)) {
             ok = false;
             break;
@@ -496,7 +526,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
               mma_nvf4(oreg, make_sdesc(st + 32 * cc, 16, 512, LAYOUT_SW64),
-                       make_sdesc(pbuf + 32 * cc, 16, 512, LAYOUT_SW64), idS4, tm + kCSFV + 4 * cc,
+                       make_sdesc(pbuf + 32 * cc, 16, 512, LAYOUT_SW64), idS4, tm + kCSFV + 8 * slot + 4 * cc,
                        tm + kCSFP + 8 * pb + 4 * cc, (i > 0 || cc > 0) ? 1u : 0u);
           } else {
 #pragma unroll
@@ -515,17 +545,52 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       mbar_wait(&ms.drain_pv, 0, kWaitNs);
     }
     __syncwarp();
+  } else if (Cfg::kCopier && warp == Cfg::kCopyV) {
+    // ======================== V scale copier (NVFP4 pass) ========================
+    // Each V tile's scales into the tensor-memory columns of its ring slot, in
+    // the order the P V issuer takes the tiles.  A slot is refilled only after
+    // the products that read its columns completed (the producer waits for
+    // them), so the copy cannot overwrite scales still in use.
+    if constexpr (PASS == kPassFp4) {
+      if (lane == 0) {
+        int u = 0;
+        bool ok = true;
+        for (int k = 0; ok && k < nk; ++k) {
+          const int nt = info[k].nt;
+          for (int i = 0; i < nt; ++i) {
+            const int slot = u % L::kSlotsV;
+            if (!wait_or_abort(&ms.full_v[slot], (u / L::kSlotsV) & 1, &ms.abort, p.err, DEV_TIMEOUT_LOAD, wns)) {
+              ok = false;
+              break;
+            }
+            ++u;
+            tc_fence_after();
+            const uint32_t st = sbase + L::kRingV + slot * L::kSlot;
+            for (int cc = 0; cc < 2; ++cc)
+              tmem_cp_32x128b_x4(tm + kCSFV + 8 * slot + 4 * cc, make_sdesc(st + 8192 + 512 * cc, 16, 128,
+                                                                             LAYOUT_NONE));
+            mma_commit(&ms.vsf_ready[slot]);
+          }
+        }
+        mma_commit(&ms.drain_cp);
+        mbar_wait(&ms.drain_cp, 0, kWaitNs);
+      }
+    }
+    __syncwarp();
   } else {
     // ======= softmax threads: lane = key of a tile, then channel of O^T =======
-    const int t = tid;
+    // Group grp's thread tq takes key tq of its tiles (TMEM lane tq) and, in
+    // group 0, channel tq of O^T.  Group 0 stages the query rows and writes
+    // the chunk's results; the groups split each chunk's tiles by pairs.
+    const int grp = Cfg::kGroups == 1 ? 0 : warp / 4, tq = tid % kDGroup;
     const float c2 = p.c2;
-    const uint32_t lane_base = tm + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tm + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     bool failed = false;
-    int gt = 0;
+    int gt0 = 0;  // tiles of this CTA before the chunk (P buffer of tile i: (gt0 + i) % kDPBuf)
     uint4 qa, qc;
-    if (nk > 0) {
-      load_query(p, head0_of(p, info[0].unit), t, qa, qc);
-      stage_query<PASS>(sm, 0, t, qa, qc);
+    if (nk > 0 && grp == 0) {
+      load_query(p, head0_of(p, info[0].unit), tq, qa, qc);
+      stage_query<PASS>(sm, 0, tq, qa, qc);
       fence_proxy_async_smem();
       mbar_arrive(&ms.bar_q[0]);
     }
@@ -535,7 +600,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       const int r = k & 1;
       const uint32_t* ent = entry + k * kDMaxTiles;
       // the next chunk's query rows, in flight while this chunk's S is read
-      if (k + 1 < nk) load_query(p, head0_of(p, info[k + 1].unit), t, qa, qc);
+      if (grp == 0 && k + 1 < nk) load_query(p, head0_of(p, info[k + 1].unit), tq, qa, qc);
       // ---- sweep 1: maximum of S per head over the keys this pass computes ----
       float mx[NG];
 #pragma unroll
@@ -545,9 +610,9 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       const uint32_t sreg = lane_base + r * kSRegion;
       if (!failed) {
         tc_fence_after();
-        // two tiles per load (the second, past the chunk's end, reads columns
-        // of the region that no head takes: mine = 0)
-        for (int i = 0; i < c.nt; i += 2) {
+        // two tiles per load, every kGroups-th pair (the second tile, past the
+        // chunk's end, reads columns of the region that no head takes: mine = 0)
+        for (int i = 2 * grp; i < c.nt; i += 2 * Cfg::kGroups) {
           uint32_t s[2 * NH];
           load_pair<NH>(sreg + NH * i, s);
 #pragma unroll
@@ -567,7 +632,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       if (lane == 0)
 #pragma unroll
         for (int g = 0; g < NG; ++g) ms.red[warp][g] = mx[g];
-      failed = softmax_bar_or<kDSoftmax>(failed);
+      failed = softmax_bar_or<Cfg::kSoft>(failed);
       // base_g = 11 - M_g, M_g = ceil(max t) = ceil(fl32(max S * c2)); thread g
       // keeps its M for the epilogue.  A head with no key in this chunk's pass
       // has M = -inf: its P is zero, its l is zero and its M weighs nothing in
@@ -576,27 +641,32 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       float my_m = -INFINITY;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
-        const float M = ceilf(fmaxf(fmaxf(ms.red[0][g], ms.red[1][g]), fmaxf(ms.red[2][g], ms.red[3][g])) * c2);
+        float mw = ms.red[0][g];
+#pragma unroll
+        for (int w = 1; w < Cfg::kSoftWarps; ++w) mw = fmaxf(mw, ms.red[w][g]);
+        const float M = ceilf(mw * c2);
         base[g] = static_cast<float>(kPLog2) - (M == -INFINITY ? 0.f : M);
-        if (t == g) my_m = M;
+        if (tid == g) my_m = M;
       }
       // The next chunk's query slot was last read by the S products of chunk
       // k - 1, which completed before this thread saw bar_s of chunk k - 1.
-      if (!failed && k + 1 < nk) {
-        stage_query<PASS>(sm, r ^ 1, t, qa, qc);
+      if (!failed && grp == 0 && k + 1 < nk) {
+        stage_query<PASS>(sm, r ^ 1, tq, qa, qc);
         fence_proxy_async_smem();
         mbar_arrive(&ms.bar_q[r ^ 1]);
       }
-      // ---- sweep 2: P per head and key, into buffer gt % kDPBuf ----
+      // ---- sweep 2: P per head and key, tile i into buffer (gt0 + i) % kDPBuf ----
       float lsum[NG];
 #pragma unroll
       for (int g = 0; g < NG; ++g) lsum[g] = 0.f;
       if constexpr (PASS == kPassFp4) {
-        // Two tiles at a time (two independent chains per warp).  failed is the
-        // same in every softmax warp here, and stays so at the end of every pair:
-        // the loop holds a barrier that every softmax warp reaches.
-        for (int i = 0; i < c.nt && !failed;) {
+        // Two tiles at a time (two independent chains per warp), pairs
+        // alternating between the groups.  failed is the same in every softmax
+        // warp here, and stays the same within a group at the end of every
+        // pair: the loop holds a barrier that each of its warps reaches.
+        for (int i = 2 * grp; i < c.nt && !failed; i += 2 * Cfg::kGroups) {
           const bool two = i + 1 < c.nt;
+          const int gt = gt0 + i;
           const int pb0 = gt % kDPBuf, pb1 = (gt + 1) % kDPBuf;
           if (gt >= kDPBuf)
             failed = !wait_or_abort(&ms.bar_pv[pb0], ((gt - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err,
@@ -656,18 +726,21 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
 #pragma unroll
                 for (int g = 0; g < NG; ++g) {
                   if ((lane & 7) == 0)
-                    *reinterpret_cast<uint32_t*>(pbuf[j] + sw64_off(g, warp) + (lane >> 1)) = wd[j][g];
+                    *reinterpret_cast<uint32_t*>(pbuf[j] + sw64_off(g, warp % 4) + (lane >> 1)) = wd[j][g];
                   if ((lane & 15) == 0)
-                    pbuf[j][1024 + (t / 64) * 512 + g * 16 + (t % 64) / 16] = static_cast<uint8_t>(sbyte[j][g]);
+                    pbuf[j][1024 + (tq / 64) * 512 + g * 16 + (tq % 64) / 16] = static_cast<uint8_t>(sbyte[j][g]);
                 }
           }
           // The P scales into tensor memory, in the layout a 32x128b.warpx4
           // copy of the two 512-byte scale chunks gives: row g of chunk cc at
           // lane g of every 32-lane quarter, columns kCSFP + 8 pb + 4 cc ..
-          // + 3.  Each warp writes its own quarter once every warp's bytes are
-          // in; every softmax warp reaches this barrier on every pair, and
-          // leaves together with the others if any gave up a wait.
-          failed = bar_or<kBarPsf, kDSoftmax>(failed);
+          // + 3.  Each warp writes its own quarter once every warp of its group
+          // has written its bytes; every warp of the group reaches this barrier
+          // on every pair, and leaves with the others if any gave up a wait.
+          if (Cfg::kGroups == 1 || grp == 0)
+            failed = bar_or<kBarPsf, kDGroup>(failed);
+          else
+            failed = bar_or<kBarPsf + 1, kDGroup>(failed);
           if (failed) break;
 #pragma unroll
           for (int j = 0; j < 2; ++j)
@@ -682,11 +755,10 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
           tc_fence_before();
           mbar_arrive(&ms.bar_p[pb0]);
           if (two) mbar_arrive(&ms.bar_p[pb1]);
-          i += two ? 2 : 1;
-          gt += two ? 2 : 1;
         }
       } else {
-        for (int i = 0; i < c.nt && !failed; ++i, ++gt) {
+        for (int i = grp; i < c.nt && !failed; i += Cfg::kGroups) {
+          const int gt = gt0 + i;
           const int pb = gt % kDPBuf;
           if (gt >= kDPBuf)
             failed = !wait_or_abort(&ms.bar_pv[pb], ((gt - kDPBuf) / kDPBuf) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA,
@@ -703,7 +775,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
             const bool on = (mine >> g) & 1u;
             const float xv = on ? ex2(fmaf(__uint_as_float(s[g]), c2, base[g])) : 0.f;  // P * 2^11
             lsum[g] += xv;
-            *reinterpret_cast<__half*>(pbuf + (t / 64) * 2048 + sw128_off(g, (t % 64) / 8) + (t % 8) * 2) =
+            *reinterpret_cast<__half*>(pbuf + (tq / 64) * 2048 + sw128_off(g, (tq % 64) / 8) + (tq % 8) * 2) =
                 __float2half_rn(xv);
           }
           fence_proxy_async_smem();
@@ -711,10 +783,12 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
           mbar_arrive(&ms.bar_p[pb]);
         }
       }
+      gt0 += c.nt;
       tc_fence_before();
       mbar_arrive(&ms.s_free[r]);
-      // ---- epilogue: the chunk's O^T column g, l_g and M_g ----
-      if (!failed) failed = !wait_or_abort(&ms.bar_o[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, wns);
+      // ---- epilogue (group 0): the chunk's O^T column g, l_g and M_g ----
+      if (!failed && grp == 0)
+        failed = !wait_or_abort(&ms.bar_o[r], (k >> 1) & 1, &ms.abort, p.err, DEV_TIMEOUT_MMA, wns);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
@@ -722,27 +796,32 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       if (lane == 0)
 #pragma unroll
         for (int g = 0; g < NG; ++g) ms.lred[warp][g] = lsum[g];
-      failed = softmax_bar_or<kDSoftmax>(failed);
+      failed = softmax_bar_or<Cfg::kSoft>(failed);
       if (failed) break;
-      tc_fence_after();
-      uint32_t o[NH];
-      load_cols<NH>(lane_base + kCO + 16 * r, o);
+      if (grp == 0) {
+        tc_fence_after();
+        uint32_t o[NH];
+        load_cols<NH>(lane_base + kCO + 16 * r, o);
 #pragma unroll
-      for (int g = 0; g < NG; ++g)
-        if (g < p.G) p.part_o[((head0 + g) * p.cap + c.slot) * kDD + t] = __uint_as_float(o[g]);
-      if (t < p.G) {
-        const size_t idx = (head0 + t) * p.cap + c.slot;
-        p.part_l[idx] = (ms.lred[0][t] + ms.lred[1][t]) + (ms.lred[2][t] + ms.lred[3][t]);
-        p.part_m[idx] = my_m;
+        for (int g = 0; g < NG; ++g)
+          if (g < p.G) p.part_o[((head0 + g) * p.cap + c.slot) * kDD + tq] = __uint_as_float(o[g]);
+        if (tq < p.G) {
+          const size_t idx = (head0 + tq) * p.cap + c.slot;
+          float lt = 0.f;
+#pragma unroll
+          for (int w = 0; w < Cfg::kSoftWarps; ++w) lt += ms.lred[w][tq];
+          p.part_l[idx] = lt;
+          p.part_m[idx] = my_m;
+        }
+        tc_fence_before();
+        mbar_arrive(&ms.o_free[r]);
       }
-      tc_fence_before();
-      mbar_arrive(&ms.o_free[r]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kDIssueS) {
+  if (warp == Cfg::kIssueS) {
     tc_fence_after();
     tmem_dealloc(tm, kDTmemCols);
   }
@@ -755,7 +834,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
 // the NVFP4 pass (which needs nothing from the FP16 pass), so NVFP4 CTAs start
 // on the SMs that FP16 CTAs leave.
 template <int NG>
-__global__ void __launch_bounds__(kDThreads, 1)
+__global__ void __launch_bounds__(DCfg<NG>::kBound, 1)
     thrift_decode_kernel(const __grid_constant__ CUtensorMap mK16, const __grid_constant__ CUtensorMap mV16,
                          const __grid_constant__ CUtensorMap mK4, const __grid_constant__ CUtensorMap mV4,
                          const DParams p) {
@@ -811,10 +890,11 @@ __device__ __forceinline__ float pow2_weight(float e) { return e >= -126.0f ? ex
 // chunks (slots 0 .. cpu - 1) and FP16 chunks (slots NT ..); both carry the
 // 2^11 pre-scale; a chunk with M_c = -inf holds no key of the head and weighs
 // 0.  One CTA of 512 threads per (batch, query head), one pass over the
-// partial results: warp w merges chunks c = w, w + 16, ... into a running
-// (M, l, O) with lane j holding channels 4 j .. 4 j + 3 (one coalesced
-// 512-byte row per chunk); the maxima are integers, so every rescale is an
-// exact power of two.  Then warp 0 merges the sixteen warps in order.
+// partial results: warp w merges chunks c = w, w + 16, ... eight at a time
+// (all eight rows loaded before any is used) into a running (M, l, O), lane
+// j holding channels 4 j .. 4 j + 3 (one coalesced 512-byte row per chunk);
+// the maxima are integers, so every rescale is an exact power of two.  Then
+// warp 0 merges the sixteen warps in order.
 __global__ void __launch_bounds__(512) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_l,
                                                              const float* __restrict__ part_m,
@@ -832,28 +912,42 @@ __global__ void __launch_bounds__(512) decode_combine_kernel(const float* __rest
   const float* pm = part_m + bh * cap;
   const float* pl = part_l + bh * cap;
   const float4* po = reinterpret_cast<const float4*>(part_o + bh * cap * kDD);
+  constexpr int kBatch = 8;  // chunk rows a lane has in flight at once
   float M = -INFINITY, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int c = warp; c < chunks; c += kWarps) {
-    const int slot = c < cpu ? c : NT + (c - cpu);
-    const float mc = pm[slot], lc = pl[slot];
-    const float4 v = po[static_cast<size_t>(slot) * (kDD / 4) + lane];
-    if (mc > M) {  // a new maximum: rescale what is summed so far
-      const float f = pow2_weight(M - mc);
+  for (int c0 = warp; c0 < chunks; c0 += kWarps * kBatch) {
+    float mc[kBatch], lc[kBatch];
+    float4 v[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int c = c0 + r * kWarps;
+      const int slot = c < cpu ? c : NT + (c - cpu);
+      const bool in = c < chunks;
+      mc[r] = in ? pm[slot] : -INFINITY;
+      lc[r] = in ? pl[slot] : 0.f;
+      v[r] = in ? po[static_cast<size_t>(slot) * (kDD / 4) + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mb = mc[0];
+#pragma unroll
+    for (int r = 1; r < kBatch; ++r) mb = fmaxf(mb, mc[r]);
+    if (mb > M) {  // a new maximum: rescale what is summed so far
+      const float f = pow2_weight(M - mb);
       acc.x *= f;
       acc.y *= f;
       acc.z *= f;
       acc.w *= f;
       L *= f;
-      M = mc;
+      M = mb;
     }
-    const float wgt = pow2_weight(mc - M);
-    acc.x = fmaf(wgt, v.x, acc.x);
-    acc.y = fmaf(wgt, v.y, acc.y);
-    acc.z = fmaf(wgt, v.z, acc.z);
-    acc.w = fmaf(wgt, v.w, acc.w);
-    L = fmaf(wgt, lc, L);
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const float wgt = pow2_weight(mc[r] - M);
+      acc.x = fmaf(wgt, v[r].x, acc.x);
+      acc.y = fmaf(wgt, v[r].y, acc.y);
+      acc.z = fmaf(wgt, v[r].z, acc.z);
+      acc.w = fmaf(wgt, v[r].w, acc.w);
+      L = fmaf(wgt, lc[r], L);
+    }
   }
   red4[warp][lane] = acc;
   if (lane == 0) {
@@ -976,11 +1070,16 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(const __half* __res
 }  // namespace
 
 namespace {
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device, asked once per device.
 int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
-                                                cudaSuccess || n <= 0)
-    return 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 }  // namespace
@@ -1081,11 +1180,23 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 // Every decode kernel asks for the largest shared-memory carveout, so that
 // consecutive kernels of a step do not make the SMs change their L1 / shared
-// split between them.
+// split between them; `smem` > 0 also raises its dynamic shared-memory limit.
+// Function attributes are per device: each kernel sets them once per device
+// (a bit per device in `done`), not on every call.
 template <typename K>
-cudaError_t max_carveout(K kernel) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
+cudaError_t kernel_attributes(K kernel, std::atomic<uint32_t>& done, size_t smem = 0) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint32_t bit = dev >= 0 && dev < 32 ? (1u << dev) : 0u;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  if (smem > 0 && (e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(smem))) != cudaSuccess)
+    return e;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           static_cast<int>(cudaSharedmemCarveoutMaxShared));
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 template <int NG>
@@ -1093,12 +1204,20 @@ cudaError_t launch_passes(const CUtensorMap (&maps)[4], const DParams& prm, cons
   const size_t smem = (DLayout<kPassFp4>::kBytes > DLayout<kPassFp16>::kBytes ? DLayout<kPassFp4>::kBytes
                                                                                 : DLayout<kPassFp16>::kBytes) +
                       1024;
-  cudaError_t e = cudaFuncSetAttribute(thrift_decode_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static std::atomic<uint32_t> done{0};
+  cudaError_t e = kernel_attributes(thrift_decode_kernel<NG>, done, smem);
   if (e != cudaSuccess) return e;
-  if ((e = max_carveout(thrift_decode_kernel<NG>)) != cudaSuccess) return e;
-  return launch_dependent(thrift_decode_kernel<NG>, dim3(pl.grid16 + pl.grid4), dim3(kDThreads), smem, st, maps[0],
-                          maps[1], maps[2], maps[3], prm);
+  e = launch_dependent(thrift_decode_kernel<NG>, dim3(pl.grid16 + pl.grid4), dim3(DCfg<NG>::kThreads), smem, st, maps[0],
+                       maps[1], maps[2], maps[3], prm);
+  if (e == cudaErrorInvalidValue) {
+    // the attributes were set in a context that has since been reset: once more
+    cudaGetLastError();
+    done.store(0u, std::memory_order_release);
+    if ((e = kernel_attributes(thrift_decode_kernel<NG>, done, smem)) != cudaSuccess) return e;
+    e = launch_dependent(thrift_decode_kernel<NG>, dim3(pl.grid16 + pl.grid4), dim3(DCfg<NG>::kThreads), smem, st, maps[0],
+                         maps[1], maps[2], maps[3], prm);
+  }
+  return e;
 }
 }  // namespace
 
@@ -1108,7 +1227,8 @@ cudaError_t launch_decode_select(const void* q, const float* km, const thrift_sh
   double kk = ceil(rho * static_cast<double>(nb) - 1e-9);
   if (kk < 0) kk = 0;
   if (kk > nb) kk = nb;
-  const cudaError_t e = max_carveout(decode_select_kernel);
+  static std::atomic<uint32_t> done{0};
+  const cudaError_t e = kernel_attributes(decode_select_kernel, done);
   if (e != cudaSuccess) return e;
   decode_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(static_cast<const __half*>(q), km, s.Hq, s.Hkv, nb, s.sm_scale,
                                                    static_cast<long long>(kk), mask);
@@ -1133,9 +1253,10 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
   const DecodePlan pl = decode_plan(s);
   const int G = s.Hq / s.Hkv;
   const int NT = num_tiles(s.N);
-  cudaError_t e = max_carveout(decode_compact_kernel);
+  static std::atomic<uint32_t> done_compact{0}, done_combine{0};
+  cudaError_t e = kernel_attributes(decode_compact_kernel, done_compact);
   if (e != cudaSuccess) return e;
-  if ((e = max_carveout(decode_combine_kernel)) != cudaSuccess) return e;
+  if ((e = kernel_attributes(decode_combine_kernel, done_combine)) != cudaSuccess) return e;
   e = launch_dependent(decode_compact_kernel, dim3(static_cast<unsigned>(BHk)), dim3(1024), 0, st, mask, s.Hq, s.Hkv,
                        NT, w.hbits, w.list16, w.n16);
   if (e != cudaSuccess) return e;
