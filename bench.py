@@ -872,8 +872,10 @@ def run_ncu_case(args, dev):
       attention: quantise and select once at --rho, then the attention
                  kernel 3 times (warm-up) and once more (the captured launch:
                  -k regex:thrift_attention -s 3 -c 1);
-      stages:    the quantisers of Q, K, V and the selection at --rho, twice
-                 in the same order (capture the second round)."""
+      stages:    the step's launches before attention (Q and K quantised and
+                 pooled in one pass each, V quantised, the selection from the
+                 block means at --rho), twice in the same order (capture the
+                 second round)."""
     import torch
 
     import fp16_block_attention_b200 as thrift
@@ -892,11 +894,13 @@ def run_ncu_case(args, dev):
             thrift.attention(Qd, Kd, Vd, mask, qz, sh, Od)
     else:
         ws = torch.empty(thrift.select_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        qm = torch.empty((w.B, w.Hq, sh.nb, w.D), dtype=torch.float32, device=dev)
+        km = torch.empty((w.B, w.Hkv, sh.nb, w.D), dtype=torch.float32, device=dev)
         for _ in range(2):
-            thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs)
-            thrift.quantize_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks)
+            thrift.quantize_pool_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, qm)
+            thrift.quantize_pool_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, km)
             thrift.quantize_nvfp4(Vd, thrift.V, sh, qz.v4, qz.vs)
-            thrift.select_blocks(Qd, Kd, sh, rho, mask, ws)
+            thrift.select_blocks_pooled(qm, km, sh, rho, mask, ws)
     torch.cuda.synchronize()
     if thrift.last_device_error() != 0:
         raise RuntimeError("a kernel reported a bounded-wait timeout")

@@ -109,43 +109,59 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __half* __rest
   }
 }
 
-// grid (ceil(nb/32), ceil(nb/32), B*Hq), block 256: a 32x32 tile of scores,
-// each thread a 2x2 sub-tile.
+// score[i][j] = fl32(sm_scale * fl32(qmean_i . kmean_j)) for one (batch,
+// query head) and a 64 x 64 tile of block pairs (tiles wholly above the causal
+// diagonal skipped).  The products of two FP32 means are exact in FP64 and
+// each dot is summed over the channels in order, in FP64, and rounded once.
+// 256 threads, thread (ty, tx) owning the 4 x 4 pairs (bi + ty + 16 a,
+// bj + tx + 16 c): per channel it reads four query and four key means (FP64,
+// widened once as 32-channel slices are staged) for sixteen FMAs.  The key
+// rows sit 33 doubles apart, so the sixteen rows a half-warp reads fall in
+// distinct bank pairs.
+constexpr int kScoreTile = 64;
+constexpr int kScoreSlice = 32;  // channels staged at a time
 __global__ void __launch_bounds__(256) score_kernel(const float* __restrict__ qm, const float* __restrict__ km,
                                                     int Hq, int Hkv, int nb, int D, int causal, float sm_scale,
                                                     float* __restrict__ scores) {
-  // The two 32-row slices of block means, widened to FP64 once (exact) as
-  // they are staged, so the inner loop is loads and FP64 FMAs only.
-  extern __shared__ double score_smem[];
-  double* qs = score_smem;               // [32][D + 1]
-  double* ks = score_smem + 32 * (D + 1);
-  const int bi = blockIdx.y * 32, bj = blockIdx.x * 32;
-  if (causal && bj > bi + 31) return;
+  __shared__ double qs[kScoreTile][kScoreSlice + 1];
+  __shared__ double ks[kScoreTile][kScoreSlice + 1];
+  const int bi = blockIdx.y * kScoreTile, bj = blockIdx.x * kScoreTile;
+  if (causal && bj > bi + kScoreTile - 1) return;
   const size_t bh = blockIdx.z;
   const size_t b = bh / Hq, hq = bh % Hq;
   const size_t bhk = b * Hkv + hq / (Hq / Hkv);
-  for (int t = threadIdx.x; t < 32 * D; t += blockDim.x) {
-    const int r = t / D, d = t % D;
-    qs[r * (D + 1) + d] = (bi + r < nb) ? static_cast<double>(qm[(bh * nb + bi + r) * D + d]) : 0.0;
-    ks[r * (D + 1) + d] = (bj + r < nb) ? static_cast<double>(km[(bhk * nb + bj + r) * D + d]) : 0.0;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0;
+  for (int d0 = 0; d0 < D; d0 += kScoreSlice) {
+    __syncthreads();  // the previous slice has been read
+    for (int t = threadIdx.x; t < kScoreTile * kScoreSlice; t += blockDim.x) {
+      const int r = t / kScoreSlice, d = t % kScoreSlice;
+      qs[r][d] = (bi + r < nb) ? static_cast<double>(qm[(bh * nb + bi + r) * D + d0 + d]) : 0.0;
+      ks[r][d] = (bj + r < nb) ? static_cast<double>(km[(bhk * nb + bj + r) * D + d0 + d]) : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int d = 0; d < kScoreSlice; ++d) {
+      double qv[4], kv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) qv[a] = qs[ty + 16 * a][d];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kv[c] = ks[tx + 16 * c][d];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fma(qv[a], kv[c], acc[a][c]);
+    }
   }
-  __syncthreads();
-  const int ti = (threadIdx.x / 16) * 2, tj = (threadIdx.x % 16) * 2;
-  const double* q0p = qs + ti * (D + 1);
-  const double* q1p = q0p + (D + 1);
-  const double* k0p = ks + tj * (D + 1);
-  const double* k1p = k0p + (D + 1);
-  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
-  for (int d = 0; d < D; ++d) {
-    const double q0 = q0p[d], q1 = q1p[d], k0 = k0p[d], k1 = k1p[d];
-    acc[0][0] = fma(q0, k0, acc[0][0]);
-    acc[0][1] = fma(q0, k1, acc[0][1]);
-    acc[1][0] = fma(q1, k0, acc[1][0]);
-    acc[1][1] = fma(q1, k1, acc[1][1]);
-  }
-  for (int a = 0; a < 2; ++a)
-    for (int c = 0; c < 2; ++c) {
-      const int i = bi + ti + a, j = bj + tj + c;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = bi + ty + 16 * a, j = bj + tx + 16 * c;
       if (i < nb && j < nb && (!causal || j <= i))
         scores[(bh * nb + i) * nb + j] = __fmul_rn(sm_scale, static_cast<float>(acc[a][c]));
     }
@@ -407,11 +423,9 @@ void launch_pool_and_scores(const void* Q, const void* K, const thrift_shape& s,
     pool_kernel<<<dim3(nb, s.B * s.Hq), kPoolThreads, 0, st>>>(static_cast<const __half*>(Q), s.N, s.D, s.blk, w.qm);
     pool_kernel<<<dim3(nb, s.B * s.Hkv), kPoolThreads, 0, st>>>(static_cast<const __half*>(K), s.N, s.D, s.blk, w.km);
   }
-  const int tiles = (nb + 31) / 32;
-  const int smem = 2 * 32 * (s.D + 1) * static_cast<int>(sizeof(double));
-  cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, smem, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
-                                                                  s.sm_scale, w.scores);
+  const int tiles = (nb + kScoreTile - 1) / kScoreTile;
+  score_kernel<<<dim3(tiles, tiles, s.B * s.Hq), 256, 0, st>>>(w.qm, w.km, s.Hq, s.Hkv, nb, s.D, s.causal,
+                                                               s.sm_scale, w.scores);
 }
 }  // namespace
 
