@@ -566,7 +566,18 @@ def run_sweep(args):
     q8 = thrift.quantize_mxfp8(Qd, thrift.Q, sh)      # buffers for the MXFP8 stages, allocated once
     k8 = thrift.quantize_mxfp8(Kd, thrift.K, sh)
     v8 = thrift.quantize_mxfp8(Vd, thrift.V, sh)
+    qm = torch.empty((w.B, w.Hq, sh.nb, w.D), dtype=torch.float32, device=dev)
+    km = torch.empty((w.B, w.Hkv, sh.nb, w.D), dtype=torch.float32, device=dev)
+    thrift.quantize_pool_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, qm, stream)
+    thrift.quantize_pool_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, km, stream)
     stages = [
+        ("step: quantise and pool Q (NVFP4 along D, FP32 block means)",
+         lambda: thrift.quantize_pool_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, qm, stream),
+         q_el * (2 + 0.5625) + qm.numel() * 4),
+        ("step: quantise and pool K", lambda: thrift.quantize_pool_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, km, stream),
+         kv_el * (2 + 0.5625) + km.numel() * 4),
+        ("step: select from the block means (FP64 scores, top-k)",
+         lambda: thrift.select_blocks_pooled(qm, km, sh, w.rho, mask, sel_ws, stream), (qm.numel() + km.numel()) * 4),
         ("quantise Q (NVFP4 along D)", lambda: thrift.quantize_nvfp4(Qd, thrift.Q, sh, qz.q4, qz.qs, stream),
          q_el * (2 + 0.5625)),
         ("quantise K (NVFP4 along D)", lambda: thrift.quantize_nvfp4(Kd, thrift.K, sh, qz.k4, qz.ks, stream),
@@ -603,7 +614,7 @@ def run_sweep(args):
         ms = e0.elapsed_time(e1) / 10
         print(f"| {name} | {ms:.4f} | {nbytes / 1e9:.3f} | {nbytes / (ms * 1e-3) / 1e9:.0f} |", flush=True)
     print()
-    del Qd, Kd, Vd, qz, mask, sel_ws
+    del Qd, Kd, Vd, qz, mask, sel_ws, qm, km
     torch.cuda.empty_cache()
 
     print("| workload | rho | blk | attention ms | effective TFLOP/s | roofline frac | MUFU frac |")
