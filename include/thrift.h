@@ -313,7 +313,8 @@ THRIFT_API thrift_status thrift_decode_select(const void* q, const float* km, co
                                               uint8_t* mask, void* stream);
 
 /* Workspace bytes of thrift_decode_attention and thrift_decode_step (the
- * mask of thrift_decode_step and per-chunk partial results). */
+ * mask of thrift_decode_step, per-chunk partial results of both passes, and
+ * per (batch, kv head) the key tiles some query head keeps in FP16). */
 THRIFT_API thrift_status thrift_decode_workspace_bytes(const thrift_shape* shape, size_t* bytes);
 
 /* Decode attention with a given mask [B][Hq][nb] (1 = FP16 block). */
