@@ -164,7 +164,9 @@ struct DParams {
   float* part_l;           // [B][Hq][cap]
   float* part_m;           // [B][Hq][cap]
   uint32_t* err;
-  uint64_t wait_ns;
+  uint64_t wait_ns;        // bound of every wait in the kernel (thrift_set_wait_limit)
+  int withhold;            // failure-detection test only: the K tile (counted per CTA and pass) whose
+                           // copies the K producer does not issue, so its consumers' waits run out; or -1
   int Hq, Hkv, NT, G;
   int units;               // B * Hkv
   int C;                   // key tiles per NVFP4 chunk (a unit's last chunk may be shorter)
@@ -400,6 +402,10 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
             ok = false;
             break;
           }
+          if (!is_v && u == p.withhold) {  // take the slot, issue nothing
+            ++u;
+            continue;
+          }
           uint8_t* st = ring + slot * L::kSlot;
           mbar_arrive_expect_tx(&full[slot], L::kSlot);
           if constexpr (PASS == kPassFp4) {
@@ -419,9 +425,10 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
           ++u;
         }
       }
-      // Let every copy this thread issued land before the CTA can exit.
+      // Let every copy this thread issued land before the CTA can exit (a
+      // withheld slot's wait runs out after the same limit).
       for (int s = 0; s < slots; ++s)
-        if (u > s) mbar_wait(&full[s], ((u - 1 - s) / slots) & 1, kWaitNs);
+        if (u > s) mbar_wait(&full[s], ((u - 1 - s) / slots) & 1, wns);
     }
     __syncwarp();
   } else if (warp == Cfg::kIssueS) {
@@ -477,7 +484,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
       }
       // drain: every tensor-core operation this thread issued completes before exit
       mma_commit(&ms.drain_s);
-      mbar_wait(&ms.drain_s, 0, kWaitNs);
+      mbar_wait(&ms.drain_s, 0, wns);
     }
     __syncwarp();
   } else if (warp == Cfg::kIssuePV) {
@@ -542,7 +549,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
         mma_commit(&ms.bar_o[r]);
       }
       mma_commit(&ms.drain_pv);
-      mbar_wait(&ms.drain_pv, 0, kWaitNs);
+      mbar_wait(&ms.drain_pv, 0, wns);
     }
     __syncwarp();
   } else if (Cfg::kCopier && warp == Cfg::kCopyV) {
@@ -573,7 +580,7 @@ __device__ __forceinline__ void decode_pass(const CUtensorMap* mK, const CUtenso
           }
         }
         mma_commit(&ms.drain_cp);
-        mbar_wait(&ms.drain_cp, 0, kWaitNs);
+        mbar_wait(&ms.drain_cp, 0, wns);
       }
     }
     __syncwarp();
@@ -1272,6 +1279,7 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
   prm.part_m = w.part_m;
   prm.err = err;
   prm.wait_ns = wait_limit_ns();
+  prm.withhold = test_withhold_tile();
   prm.Hq = s.Hq;
   prm.Hkv = s.Hkv;
   prm.NT = NT;

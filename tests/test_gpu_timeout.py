@@ -1,6 +1,6 @@
 """Failure detection on the GPU: a bounded wait that runs out (no GPU fault).
 
-Every wait inside the attention kernels is bounded (thrift_set_wait_limit).
+Every wait inside the attention and decode kernels is bounded (thrift_set_wait_limit).
 Here the wait limit is set to 1 ms and the producer of every CTA withholds the
 copies of one key tile (THRIFT_TEST_WITHHOLD_TILE: its ring slot is taken but
 nothing is ever copied into it, so the barrier its consumers wait on is never
@@ -104,3 +104,50 @@ def test_wait_limit_is_checked_on_the_host():
     assert lib.thrift_set_wait_limit(999) == 1
     assert lib.thrift_set_wait_limit(60_000_000_001) == 1
     assert lib.thrift_set_wait_limit(thrift.WAIT_LIMIT_DEFAULT_NS) == 0
+
+
+# Decode: both passes' K producers withhold their third K tile; with a 32k
+# cache every CTA of both passes takes at least three K tiles.  4, 8 and 16
+# query heads per kv head: two softmax groups and a V scale copier, one group
+# and a copier, one group without a copier.
+DECODE_CASES = [synth.GQA_N32K.with_(Hq=8, Hkv=2), synth.GQA_N32K.with_(Hq=16, Hkv=2),
+                synth.GQA_N32K.with_(Hq=32, Hkv=2)]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("w", DECODE_CASES, ids=lambda w: f"G{w.Hq // w.Hkv}")
+def test_a_decode_wait_that_runs_out_is_reported_and_the_next_call_is_unaffected(w, monkeypatch):
+    from oracle import decode
+
+    Q, K, V = synth.generate(w)
+    q = np.ascontiguousarray(Q[:, :, -1])
+    del Q
+    qd, Kd, Vd = to_dev(q, K, V)
+    sh = shape_of(w)
+    rho = 0.3
+    m_ref = decode.select(q, K, w.blk, w.sm_scale, rho, oracle.budget)
+    md, = to_dev(m_ref)
+    kq = thrift.quantize_kv(Kd, Vd, sh)
+    assert thrift.last_device_error() == 0
+    try:
+        thrift.set_wait_limit(1_000_000)  # 1 ms
+        monkeypatch.setenv("THRIFT_TEST_WITHHOLD_TILE", str(WITHHELD))
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        thrift.decode_attention(qd, Kd, Vd, kq, md, sh)
+        status = thrift.last_device_error()  # synchronises
+        elapsed = time.perf_counter() - t0
+    finally:
+        monkeypatch.delenv("THRIFT_TEST_WITHHOLD_TILE", raising=False)
+        thrift.set_wait_limit(thrift.WAIT_LIMIT_DEFAULT_NS)
+    assert status == THRIFT_ERR_TIMEOUT
+    assert elapsed < 1.0, elapsed
+
+    # the next call, with the defaults restored, is correct
+    out = thrift.decode_attention(qd, Kd, Vd, kq, md, sh)
+    assert thrift.last_device_error() == 0
+    heads = [(0, h) for h in range(w.Hq)]
+    ref = oracle.to_f16(decode.attention(q, K, V, m_ref, w.blk, w.sm_scale, heads))
+    got = out.cpu().numpy().reshape(-1, w.D)
+    mx, mean = compare_o(got, ref)
+    assert mx <= ATOL_MAX and mean <= ATOL_MEAN, (mx, mean)
