@@ -45,7 +45,7 @@ FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF / 2.25 PF)
 FP8_OVER_BF16 = 2.0          # nominal dense ratio (4.5 PF / 2.25 PF)
 PROFILE_FILE = os.path.join(ROOT, "profiles", "attention_gqa_n32k_traffic.json")
 KERNEL_SOURCES = ["attention.cu", "attention_db.cu", "attention_common.cuh", "ptx.cuh", "tmap.h"]
-LAUNCHES_PER_STEP = 8        # quantize Q, K, V; pool Q, K; scores; top-k; attention
+LAUNCHES_PER_STEP = 6        # quantise-and-pool Q, K; quantise V; scores; top-k; attention
 
 
 # ---------------------------------------------------------------- helpers ---
