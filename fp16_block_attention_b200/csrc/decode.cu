@@ -15,12 +15,15 @@
 // unquantised P.  Supported: D = 128, blk = 128, Hq / Hkv <= 16.
 //
 // Kernels:
-//   decode_select     one CTA per (batch, query head): the nb scores, then the
-//                     top k by rank of a unique 64-bit key.
+//   decode_select     one CTA per (batch, query head): the nb scores (one warp
+//                     per key block, coalesced), then the top k of unique
+//                     64-bit keys by a bitonic sort.
 //   decode_compact    one CTA per (batch, kv head) "unit": per key tile the
 //                     bits of the group's query heads that keep it in FP16,
 //                     and the list of the tiles some head keeps, in order.
-//   decode_attention  two passes, each a persistent kernel (one CTA per SM)
+//   thrift_decode_kernel  both passes in one persistent launch (the FP16
+//                     pass on the first SMs' worth of CTAs, the NVFP4 pass on
+//                     the rest, starting on the SMs the first leave), each CTA
 //                     walking chunks of one unit's key tiles with all its G
 //                     query heads, keys on the 128 tensor-memory lanes:
 //                       NVFP4 pass: chunks of <= 16 consecutive tiles;
@@ -34,14 +37,15 @@
 //                     Within a chunk two sweeps: every S first (one integer
 //                     maximum per head and chunk, so O is never rescaled),
 //                     then P and the P V products.  S, O and the query copies
-//                     are double-buffered across chunks and the loads stream
-//                     through one ring per pass (23 NVFP4 slots of 9 KB, or 6
-//                     fp16 slots of 32 KB), so one chunk's products overlap the
-//                     next one's loads.  Each chunk writes its unnormalised O,
-//                     l and M per head.
-//   decode_combine    per (batch, query head) and 32 channels: O = sum_c
-//                     2^(M_c - M) O_c / sum_c 2^(M_c - M) l_c over both passes'
-//                     chunks (exact power-of-two rescales).
+//                     are double-buffered across chunks; K and V stream
+//                     through a ring each (NVFP4: 12 and 11 slots of 9 KB;
+//                     FP16: 3 and 3 slots of 32 KB), so one chunk's products
+//                     overlap the next one's loads.  Each chunk writes its
+//                     unnormalised O, l and M per head.
+//   decode_combine    per (batch, query head): O = sum_c 2^(M_c - M) O_c /
+//                     sum_c 2^(M_c - M) l_c over both passes' chunks, in one
+//                     online sweep (exact power-of-two rescales).
+// The kernels of a step are chained by programmatic dependent launch.
 // The chunk's own maximum leaves every NVFP4 code of P as under the global
 // one while the group scales stay E4M3 normals (the prefill's argument for
 // its running maximum).
