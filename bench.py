@@ -925,7 +925,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=4096)
-    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=256)  # oracle rows per reference step (60 steps: about a minute on 16 cores)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--split", default="problems", choices=["problems", "heads"],
                     help="N > 1: an independent problem per rank (weak scaling, the default) or one problem "
